@@ -1,0 +1,383 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention hot path on B200.
+
+One step = one training pass of attention over one batch of the GQA workload
+(B=1, Hq=32, Hkv=8, N=8192, d=128, causal): fa_fwd then fa_bwd, through the C
+ABI, inputs resident in HBM.  The decode workload (B=64, Hq=32, Hkv=8, Nq=1,
+Nk=8192) is timed in the same run and reported under "parts".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl libfa|reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own replica of
+the workload on its own seeded batch (weak scaling, no collective on the data
+path); the timed region is bracketed by a barrier and synchronize and the
+reported time is the max over ranks.  Rank 0 prints one JSON line.
+
+FLOP rule: fwd = 4 B Hq Nq Nk d (halved when causal), bwd = 2.5 x fwd.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+STEP_WORKLOAD = "gqa_8k"
+DECODE_WORKLOAD = "gqa_decode"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing (host side; covered by CPU gloo tests)
+# ----------------------------------------------------------------------------
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own batch: a distinct seed per rank."""
+    return base_seed + 1000 * rank
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------
+# measured peaks and clocks
+# ----------------------------------------------------------------------------
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return dict(hbm_gbs=float(pk["hbm_gbs"]), bf16_tflops=float(pk["bf16_tflops"]),
+                    bf16_tflops_sustained=float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                    source="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                    source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.out = open(os.devnull, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# CPU reference arm: the oracle on a bounded sample
+# ----------------------------------------------------------------------------
+def oracle_sample_workload():
+    """One kv group (4 query heads) of the step workload at N = 2048: 15 GFLOP
+    of fwd + bwd by the FLOP rule, a few seconds of oracle time per step."""
+    w = synth.WORKLOADS[STEP_WORKLOAD]
+    return w.with_(B=1, Hq=w.G, Hkv=1, Nq=2048, Nk=2048)
+
+
+def time_oracle_step(w):
+    import oracle
+    x = synth.make_inputs(w)
+    t0 = time.perf_counter()
+    oracle.fwd(x["q"], x["k"], x["v"], w.scale, w.causal)
+    oracle.bwd(x["q"], x["k"], x["v"], x["dout"], w.scale, w.causal)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline_leg(reps=3):
+    w = oracle_sample_workload()
+    dt = sum(time_oracle_step(w) for _ in range(reps)) / reps
+    flops = w.fwd_flops() + w.bwd_flops()
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
+            "kind": "oracle",
+            "sample": (f"fwd+bwd of one kv group (B=1, Hq=4, Hkv=1, N=2048, d=128, causal) "
+                       f"of the {STEP_WORKLOAD} workload, {flops / 1e9:.1f} GFLOP by the FLOP "
+                       f"rule, mean of {reps} runs of {dt:.1f} s, fp64 oracle on all host cores")}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    w = oracle_sample_workload()
+    flops = w.fwd_flops() + w.bwd_flops()
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm-up state; its first step is timed like the rest
+    times = [time_oracle_step(w) for _ in range(args.steps)]
+    dt = sum(times) / len(times)
+    value = flops / dt / 1e12
+    line = {
+        "impl": "reference", "metric": "attention fwd+bwd TFLOP/s (causal GQA, N=8192, d=128)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{STEP_WORKLOAD} (oracle sample: one kv group at N=2048)",
+                   "B": 1, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.Nq, "d": w.d, "causal": True},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": "fwd+bwd of one kv group (Hq=4, Hkv=1) at N=2048, per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+def run_libfa(args, rank, world, local):
+    import torch
+    import exact_attention_114_b200 as fa
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+
+    w = synth.WORKLOADS[STEP_WORKLOAD]
+    w = w.with_(seed=rank_seed(w.seed, rank))
+    x = synth.make_inputs(w, pinned=True)
+    xd = {k: v.to(dev, non_blocking=True) for k, v in x.items()}
+    o = torch.empty_like(xd["q"])
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(xd["q"]), torch.empty_like(xd["k"]), torch.empty_like(xd["v"])
+    ws = torch.empty(fa.fa_bwd_workspace_size(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def fwd():
+        fa.fa_fwd(xd["q"], xd["k"], xd["v"], o, lse, causal=True, scale=w.scale)
+
+    def bwd():
+        fa.fa_bwd(xd["q"], xd["k"], xd["v"], o, xd["dout"], lse, dq, dk, dv, causal=True,
+                  scale=w.scale, workspace=ws)
+
+    def timed(fn, k):
+        """Per-call CUDA-event times (ms), L2 flushed before each call."""
+        ts = []
+        for _ in range(k):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in ts]
+
+    for _ in range(args.warmup):
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    fa.fa_check_device_status()
+
+    # ---- the timed steps
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        step_ms, fwd_ms, bwd_ms = [], [], []
+        for _ in range(args.steps):
+            flush.zero_()
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            e[0].record(stream)
+            fwd()
+            e[1].record(stream)
+            bwd()
+            e[2].record(stream)
+            step_ms.append(e)
+        torch.cuda.synchronize()
+    barrier(world)
+    for e in step_ms:
+        fwd_ms.append(e[0].elapsed_time(e[1]))
+        bwd_ms.append(e[1].elapsed_time(e[2]))
+    fa.fa_check_device_status()
+    total_ms = sum(fwd_ms) + sum(bwd_ms)
+    total_ms = max_over_ranks(total_ms, world, dev)
+    ms_step = total_ms / args.steps
+    flops_step = w.fwd_flops() + w.bwd_flops()
+    value = world * flops_step / (ms_step * 1e-3) / 1e12
+    fwd_med, bwd_med = statistics.median(fwd_ms), statistics.median(bwd_ms)
+    fwd_tf = w.fwd_flops() / (fwd_med * 1e-3) / 1e12
+    bwd_tf = w.bwd_flops() / (bwd_med * 1e-3) / 1e12
+
+    # ---- end to end through the public API: pinned host in, gradients out
+    hx = x
+    hdq = torch.empty_like(x["q"], pin_memory=True)
+    hdk = torch.empty_like(x["k"], pin_memory=True)
+    hdv = torch.empty_like(x["v"], pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in hx.values())
+    d2h = sum(t.numel() * t.element_size() for t in (hdq, hdk, hdv))
+
+    def e2e_step():
+        for kk in ("q", "k", "v", "dout"):
+            xd[kk].copy_(hx[kk], non_blocking=True)
+        fwd()
+        bwd()
+        hdq.copy_(dq, non_blocking=True)
+        hdk.copy_(dk, non_blocking=True)
+        hdv.copy_(dv, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e2e_ms = statistics.median(timed(e2e_step, max(3, min(args.steps, 10))))
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
+    e2e_value = world * flops_step / (e2e_ms * 1e-3) / 1e12
+
+    # ---- decode workload (HBM-bound path)
+    wd = synth.WORKLOADS[DECODE_WORKLOAD]
+    wd = wd.with_(seed=rank_seed(wd.seed, rank))
+    dx = synth.make_inputs(wd)
+    dxd = {k: v.to(dev) for k, v in dx.items()}
+    del dx
+    od = torch.empty_like(dxd["q"])
+    lsed = torch.empty((wd.B, wd.Hq, 1), dtype=torch.float32, device=dev)
+
+    def dec():
+        fa.fa_fwd(dxd["q"], dxd["k"], dxd["v"], od, lsed, causal=False, scale=wd.scale)
+
+    for _ in range(max(3, args.warmup)):
+        dec()
+    torch.cuda.synchronize()
+    dec_ms = statistics.median(timed(dec, max(10, args.steps)))
+    dec_bytes = (2 * wd.B * wd.Hkv * wd.Nk * wd.d * 2 + 2 * wd.B * wd.Hq * wd.d * 2
+                 + wd.B * wd.Hq * 4)
+    dec_gbs = dec_bytes / (dec_ms * 1e-3) / 1e9
+    fa.fa_check_device_status()
+
+    clocks = clk.summary()
+    line = {
+        "metric": "attention fwd+bwd TFLOP/s (causal GQA, N=8192, d=128)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{STEP_WORKLOAD}: B=1, Hq=32, Hkv=8, N=8192, d=128, causal, "
+                               f"bf16 N(0,1) inputs (seed {w.seed})",
+                   "global_batch": world * w.B, "seq_len": w.Nq, "parallelism": f"replicas x{world}",
+                   "l2": "flushed before every timed call (2 x 126 MiB write)"},
+        "parts": {
+            "fwd": {"ms": fwd_med, "tflops": fwd_tf, "frac_of_peak": fwd_tf / peaks["bf16_tflops_sustained"]},
+            "bwd": {"ms": bwd_med, "tflops": bwd_tf, "frac_of_peak": bwd_tf / peaks["bf16_tflops_sustained"]},
+            "decode": {"workload": f"{DECODE_WORKLOAD}: B=64, Hq=32, Hkv=8, Nq=1, Nk=8192, d=128",
+                       "ms": dec_ms, "gbs": dec_gbs, "frac_of_hbm": dec_gbs / peaks["hbm_gbs"],
+                       "algorithmic_bytes": dec_bytes},
+        },
+        "roofline": {"kernel": "fa_bwd (bwd_main dominant; pre/post included in the time)",
+                     "bound": "tensor", "achieved": bwd_tf,
+                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": bwd_tf / peaks["bf16_tflops_sustained"], "traffic": None,
+                     "peak_source": peaks["source"] + " (sustained bf16 cuBLAS)"},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps * 4,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_leg()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["libfa", "reference"], default="libfa")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        # the CPU oracle: rank 0 alone measures it; other ranks have no work
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        import torch
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        return run_libfa(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

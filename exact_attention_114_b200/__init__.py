@@ -1,0 +1,184 @@
+"""Python binding of libfa (exact attention for B200, sm_100a).
+
+Argument marshalling only: every function here forwards torch device tensors
+(as raw pointers, sizes and the current CUDA stream) to the C ABI declared in
+``include/fa.h`` and raises ``FaError`` on a non-OK status.  There is no
+fallback: if ``libfa.so`` has not been built, loading fails loudly.
+
+Layouts (BHSD, contiguous): q, o, dout, dq [B, Hq, Nq, d]; k, v, dk, dv
+[B, Hkv, Nk, d] in bf16; lse [B, Hq, Nq] in fp32.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+FA_OK = 0
+FA_ERR_INVALID_ARGUMENT = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_WORKSPACE = 3
+FA_ERR_CUDA = 4
+FA_ERR_TIMEOUT = 5
+
+_lock = threading.Lock()
+_lib = None
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{status_string(status)}: {message}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libfa.so (raises if it was not built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(
+                    f"libfa.so is missing at {LIB_PATH}; build it with "
+                    "`python -m exact_attention_114_b200.build` (needs nvcc)")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, ip, fl, sz, uip = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t,
+                                   ctypes.c_uint)
+            L.fa_abi_version.argtypes = []
+            L.fa_abi_version.restype = ip
+            L.fa_status_string.argtypes = [ip]
+            L.fa_status_string.restype = ctypes.c_char_p
+            L.fa_last_error_message.argtypes = []
+            L.fa_last_error_message.restype = ctypes.c_char_p
+            L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, fl, ip, vp]
+            L.fa_fwd.restype = ip
+            L.fa_fwd_splitkv_workspace_size.argtypes = [ip, ip, ip, ip, ip, ip, ip]
+            L.fa_fwd_splitkv_workspace_size.restype = sz
+            L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, fl, ip, ip, vp,
+                                         sz, vp]
+            L.fa_fwd_splitkv.restype = ip
+            L.fa_bwd_workspace_size.argtypes = [ip, ip, ip, ip, ip, ip]
+            L.fa_bwd_workspace_size.restype = sz
+            L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, fl, ip,
+                                 vp, sz, vp]
+            L.fa_bwd.restype = ip
+            L.fa_check_device_status.argtypes = [vp]
+            L.fa_check_device_status.restype = ip
+            L.fa_selftest_wait_timeout.argtypes = [uip, vp]
+            L.fa_selftest_wait_timeout.restype = ip
+            _lib = L
+        return _lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return lib().fa_status_string(int(status)).decode()
+    except ImportError:
+        return f"status {status}"
+
+
+def last_error_message() -> str:
+    return lib().fa_last_error_message().decode()
+
+
+def _check(status: int):
+    if status != FA_OK:
+        raise FaError(status, last_error_message())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dims(q, k):
+    B, Hq, Nq, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if B != Bk or d != dk:
+        raise ValueError(f"q {tuple(q.shape)} and k {tuple(k.shape)} disagree")
+    return B, Hq, Hkv, Nq, Nk, d
+
+
+def _require(t, name, dtype):
+    if not t.is_cuda or not t.is_contiguous() or t.dtype != dtype:
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+
+
+def abi_version() -> int:
+    return int(lib().fa_abi_version())
+
+
+def fa_fwd(q, k, v, o=None, lse=None, *, causal=False, scale=None, stream=None, want_lse=True):
+    """Forward: returns (o, lse).  Allocates o / lse when not given."""
+    import torch
+    B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _require(t, n, torch.bfloat16)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d,
+                        scale, int(bool(causal)), _stream(stream)))
+    return o, lse
+
+
+def fa_fwd_splitkv_workspace_size(B, Hq, Hkv, Nq, Nk, d, num_splits=0) -> int:
+    return int(lib().fa_fwd_splitkv_workspace_size(B, Hq, Hkv, Nq, Nk, d, num_splits))
+
+
+def fa_fwd_splitkv(q, k, v, o=None, lse=None, *, causal=False, scale=None, num_splits=0,
+                   workspace=None, stream=None):
+    """Split-KV (decode-shape) forward.  ``workspace`` is an optional device
+    tensor of at least ``fa_fwd_splitkv_workspace_size`` bytes."""
+    import torch
+    B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq,
+                                Nk, d, scale, int(bool(causal)), int(num_splits), _ptr(workspace),
+                                ws_bytes, _stream(stream)))
+    return o, lse
+
+
+def fa_bwd_workspace_size(B, Hq, Hkv, Nq, Nk, d) -> int:
+    return int(lib().fa_bwd_workspace_size(B, Hq, Hkv, Nq, Nk, d))
+
+
+def fa_bwd(q, k, v, o, dout, lse, dq=None, dk=None, dv=None, *, causal=False, scale=None,
+           workspace=None, stream=None):
+    """Backward: returns (dq, dk, dv).  Allocates the gradients when not given."""
+    import torch
+    B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                        _ptr(dk), _ptr(dv), B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)),
+                        _ptr(workspace), ws_bytes, _stream(stream)))
+    return dq, dk, dv
+
+
+def fa_check_device_status(stream=None):
+    _check(lib().fa_check_device_status(_stream(stream)))
+
+
+def fa_selftest_wait_timeout(timeout_us: int = 2000, stream=None) -> int:
+    """Runs the bounded-wait self-test; returns the raw status (5 = timeout seen)."""
+    return int(lib().fa_selftest_wait_timeout(int(timeout_us), _stream(stream)))

@@ -1,0 +1,529 @@
+// bwd.cuh -- backward pass by recomputation (page "FlashAttention：为什么少搬数据，
+// 反而算得更快", §05: rebuild each needed block of P from the saved row
+// statistic instead of reading a stored P).  For L = sum(dO * O):
+//   P = exp(scale q.k - LSE),  dV += P^T dO,  dP = dO V^T,  D = rowsum(dO * O),
+//   dS = P * (dP - D),  dK += scale dS^T Q,  dQ += scale dS K.
+//
+// Three kernels:
+//   bwd_pre   one warp per query row: D_i, LSE_i * log2(e) (+inf for rows that
+//             see no key, so their P is 0), and zero the fp32 dQ accumulator.
+//   bwd_main  one CTA per (batch, kv head, 128-key block), key-stationary:
+//             K and V stay in shared memory while the CTA walks every query
+//             head of the group and every 64-row query block that can see the
+//             keys (causal blocks above the diagonal are skipped).  dK and dV
+//             accumulate in tensor memory across the whole group, so the GQA
+//             reduction over query heads needs no atomics.
+//   bwd_post  dQ = bf16(scale * accumulator).
+//
+// bwd_main roles (384 threads = 3 warpgroups):
+//   warps 0-3  thread r = key r = TMEM lane r: read S^T and dP^T rows from TMEM,
+//              form P^T and dS^T (bf16) in shared memory; final dK/dV epilogue.
+//   warps 4-7  thread c = dQ^T row c (feature c): move dQ^T from TMEM to a
+//              shared [64 x d] fp32 tile and add it to the dQ accumulator with
+//              one bulk asynchronous reduce-add.
+//   warp 8     TMA loads (K, V once; Q, dO, LSE, D per step, two slots).
+//   warps 10-11 complete the third warpgroup (which gives registers away).
+//   warp 9     one thread issues the tcgen05.mma ops, per step `it`:
+//                S^T(it+1) = K Q^T, dP^T(it+1) = V dO^T      (after P/dS of it)
+//                dV += P^T(it) dO, dK += dS^T(it) Q, dQ^T(it) = K^T dS^T(it)
+//              so the softmax of step it+1 overlaps the gradient MMAs of it.
+// Tensor memory (512 columns): dK | dV (d each) | S^T 64 | dP^T 64 | dQ^T 64.
+#pragma once
+
+#include "sm100.cuh"
+#include "fa_kernels.h"
+
+namespace fa {
+
+// ----------------------------------------------------------------------------
+// bulk (non-tensor) async copies
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, const void* src, uint32_t bytes)
+{
+    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
+                 "r"(smem_u32(src)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// ----------------------------------------------------------------------------
+// bwd_pre: D = rowsum(dO * O), LSE in log2 units, zero the dQ accumulator
+// ----------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(BwdParams p)
+{
+    const int row = (int)(blockIdx.x * 8 + (threadIdx.x >> 5));   // over B * Hq * Nq_pad
+    const int lane = threadIdx.x & 31;
+    const int total = p.B * p.Hq * p.Nq_pad;
+    if (row >= total)
+        return;
+    const int bh = row / p.Nq_pad, i = row % p.Nq_pad;
+    constexpr int E = D / 32;   // elements per lane
+    float* acc = p.dq_acc + (size_t)row * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+        acc[e] = 0.f;
+    if (i >= p.Nq) {
+        if (lane == 0) {
+            p.delta[row] = 0.f;
+            p.lse_log2[row] = INFINITY;
+        }
+        return;
+    }
+    const size_t src = ((size_t)bh * p.Nq + i) * D + lane * E;
+    float s = 0.f;
+    if constexpr (E == 4) {
+        const uint2 a = *reinterpret_cast<const uint2*>(p.o + src);
+        const uint2 c = *reinterpret_cast<const uint2*>(p.dout + src);
+        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* c2 = reinterpret_cast<const __nv_bfloat162*>(&c);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const float2 x = __bfloat1622float2(a2[e]), y = __bfloat1622float2(c2[e]);
+            s = fmaf(x.x, y.x, s);
+            s = fmaf(x.y, y.y, s);
+        }
+    } else {
+        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(p.o + src);
+        const __nv_bfloat162 c = *reinterpret_cast<const __nv_bfloat162*>(p.dout + src);
+        const float2 x = __bfloat1622float2(a), y = __bfloat1622float2(c);
+        s = fmaf(x.x, y.x, s);
+        s = fmaf(x.y, y.y, s);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) {
+        p.delta[row] = s;
+        const float l = p.lse[(size_t)bh * p.Nq + i];
+        p.lse_log2[row] = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+    }
+}
+
+// ----------------------------------------------------------------------------
+// bwd_post: dQ = bf16(scale * accumulator)
+// ----------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) bwd_post_kernel(BwdParams p)
+{
+    const size_t n4 = (size_t)p.B * p.Hq * p.Nq * D / 4;
+    for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n4;
+         idx += (size_t)gridDim.x * blockDim.x) {
+        const size_t e = idx * 4;
+        const size_t row = e / D, c = e % D;
+        const size_t bh = row / p.Nq, i = row % p.Nq;
+        const float4 a = *reinterpret_cast<const float4*>(p.dq_acc + (bh * p.Nq_pad + i) * D + c);
+        uint2 w;
+        w.x = pack_bf16x2(a.x * p.scale, a.y * p.scale);
+        w.y = pack_bf16x2(a.z * p.scale, a.w * p.scale);
+        *reinterpret_cast<uint2*>(p.dq + e) = w;
+    }
+}
+
+// ----------------------------------------------------------------------------
+// bwd_main
+// ----------------------------------------------------------------------------
+template <int D>
+struct BwdCfg {
+    static constexpr int kThreads = 384;
+    // registers per thread after the split: 128 x (240 + 120 + 80) <= 384 x 168
+    static constexpr uint32_t kRegsDS = 240, kRegsDQ = 120, kRegsOther = 80;
+    static constexpr int kKPanel = 128 * 128;          // 128 keys x 64 bf16
+    static constexpr int kKTile = (D / 64) * kKPanel;  // K or V block
+    static constexpr int kQPanel = 64 * 128;           // 64 rows x 64 bf16
+    static constexpr int kQTile = (D / 64) * kQPanel;  // Q or dO block
+    static constexpr int kSlot = 2 * kQTile + 1024;    // Q, dO, lse_log2[64], delta[64] (1 KB-aligned)
+    static constexpr int kPTile = 128 * 128;           // P^T or dS^T: 128 keys x 64 q bf16
+    static constexpr int kOffK = 0;
+    static constexpr int kOffV = kOffK + kKTile;
+    static constexpr int kOffZero = kOffV + kKTile;                 // zero panel (D = 64 only)
+    static constexpr int kOffSlots = kOffZero + (D == 64 ? kKPanel : 0);
+    static constexpr int kOffP = kOffSlots + 2 * kSlot;
+    static constexpr int kOffDS = kOffP + kPTile;
+    static constexpr int kOffDQ = kOffDS + kPTile;                  // fp32 [64][D] staging
+    static constexpr int kOffBar = kOffDQ + 64 * D * 4;
+    static constexpr int kSmemBytes = kOffBar + 256 + 1024;
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kColDK = 0, kColDV = D, kColS = 2 * D, kColDP = 2 * D + 64,
+                              kColDQ = 2 * D + 128;
+};
+
+__device__ __forceinline__ void bwd_q_range(const BwdParams& p, int kb, int& qb0, int& nqb)
+{
+    const int nqb_all = p.Nq_pad / 64;
+    qb0 = 0;
+    if (p.causal) {
+        // first query block containing a row i with kb*128 <= i + (Nk - Nq)
+        const int first_row = kb * 128 - (p.Nk - p.Nq);
+        qb0 = first_row <= 0 ? 0 : first_row / 64;
+    }
+    nqb = max(0, nqb_all - qb0);
+}
+
+// byte offset of (row, 16-byte chunk) in a tile of 128-byte swizzled rows
+__device__ __forceinline__ uint32_t sw128_off(int row, int chunk)
+{
+    return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(384, 1)
+    bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                    BwdParams p)
+{
+    using C = BwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+    uint64_t* bar_kv = bars;            // K, V landed
+    uint64_t* bar_full = bars + 1;      // [2] step slot landed
+    uint64_t* bar_empty = bars + 3;     // [2] step slot released
+    uint64_t* bar_sdp = bars + 5;       // S^T and dP^T of a step in TMEM
+    uint64_t* bar_ds = bars + 6;        // P^T, dS^T of a step in smem (count 4)
+    uint64_t* bar_dsfree = bars + 7;    // gradient MMAs of a step done (smem P/dS free)
+    uint64_t* bar_dq = bars + 8;        // dQ^T of a step in TMEM
+    uint64_t* bar_dqfree = bars + 9;    // dQ^T read out of TMEM (count 4)
+    uint64_t* bar_final = bars + 10;    // all MMAs done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = warp_id(), lane = lane_id();
+    const int n_kb = (p.Nk + 127) / 128;
+    const int kb = (int)blockIdx.x / (p.B * p.Hkv);   // small key blocks (most work) first
+    const int kvh = (int)blockIdx.x % (p.B * p.Hkv);
+    const int b = kvh / p.Hkv, hk = kvh % p.Hkv;
+    int qb0, nqb;
+    bwd_q_range(p, kb, qb0, nqb);
+    if (!CAUSAL) {
+        qb0 = 0;
+        nqb = p.Nq_pad / 64;
+    }
+    const int n_it = p.G * nqb;
+    (void)n_kb;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_kv, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bar_full[s], 1);
+            mbar_init(&bar_empty[s], 1);
+        }
+        mbar_init(bar_sdp, 1);
+        mbar_init(bar_ds, 4);
+        mbar_init(bar_dsfree, 1);
+        mbar_init(bar_dq, 1);
+        mbar_init(bar_dqfree, 4);
+        mbar_init(bar_final, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (D == 64) {
+        // zero panel: rows 64..127 of K^T for the dQ^T MMA (M is 128)
+        uint4* z = reinterpret_cast<uint4*>(smem + C::kOffZero);
+        for (int i = threadIdx.x; i < C::kKPanel / 16; i += blockDim.x)
+            z[i] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
+    }
+    if (warp == 9) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    auto step_coords = [&](int it, int& h, int& qb) {
+        h = hk * p.G + it / nqb;
+        qb = qb0 + it % nqb;
+    };
+
+    // Each role runs inside the branch that sets its register budget.
+    if (warp >= 8) {
+      regs_dec<C::kRegsOther>();
+      if (warp == 8) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tensormap(&tmQ);
+            prefetch_tensormap(&tmDO);
+            mbar_arrive_expect_tx(bar_kv, 2 * C::kKTile);
+            for (int pn = 0; pn < D / 64; ++pn) {
+                tma_load_3d(smem + C::kOffK + pn * C::kKPanel, &tmK, bar_kv, pn * 64, kb * 128, kvh);
+                tma_load_3d(smem + C::kOffV + pn * C::kKPanel, &tmV, bar_kv, pn * 64, kb * 128, kvh);
+            }
+            int issued = 0;
+            for (int it = 0; it < n_it; ++it) {
+                const int s = it & 1;
+                if (!mbar_wait(&bar_empty[s], (uint32_t)((it >> 1) & 1) ^ 1u, abort_flag))
+                    break;
+                int h, qb;
+                step_coords(it, h, qb);
+                const int bh = b * p.Hq + h;
+                uint8_t* slot = smem + C::kOffSlots + s * C::kSlot;
+                mbar_arrive_expect_tx(&bar_full[s], 2 * C::kQTile + 512);
+                for (int pn = 0; pn < D / 64; ++pn) {
+                    tma_load_3d(slot + pn * C::kQPanel, &tmQ, &bar_full[s], pn * 64, qb * 64, bh);
+                    tma_load_3d(slot + C::kQTile + pn * C::kQPanel, &tmDO, &bar_full[s], pn * 64, qb * 64, bh);
+                }
+                const size_t vrow = (size_t)bh * p.Nq_pad + (size_t)qb * 64;
+                bulk_load(slot + 2 * C::kQTile, p.lse_log2 + vrow, 256, &bar_full[s]);
+                bulk_load(slot + 2 * C::kQTile + 256, p.delta + vrow, 256, &bar_full[s]);
+                ++issued;
+            }
+            if (*abort_flag) {
+                mbar_wait_limited(bar_kv, 0, FA_WAIT_LIMIT_CYCLES);
+                for (int i = max(0, issued - 2); i < issued; ++i)
+                    mbar_wait_limited(&bar_full[i & 1], (uint32_t)((i >> 1) & 1), FA_WAIT_LIMIT_CYCLES);
+            }
+        }
+      } else if (warp == 9) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_sdp = idesc_bf16_f32(128, 64, false, false);   // S^T, dP^T
+            const uint32_t id_grad = idesc_bf16_f32(128, D, false, true);    // dV, dK
+            const uint32_t id_dq = idesc_bf16_f32(128, 64, true, true);      // dQ^T
+            const uint32_t sK = smem_u32(smem + C::kOffK), sV = smem_u32(smem + C::kOffV);
+            const uint32_t sP = smem_u32(smem + C::kOffP), sDS = smem_u32(smem + C::kOffDS);
+            const uint32_t tDK = tmem + C::kColDK, tDV = tmem + C::kColDV, tS = tmem + C::kColS,
+                           tDP = tmem + C::kColDP, tDQ = tmem + C::kColDQ;
+            // K^T as the M = 128 operand of dQ^T: d panels are 16 KB apart (for d = 64
+            // the second "panel" is the zero panel right after V... placed at kOffZero)
+            const uint32_t lbo_kt = (D == 128) ? (uint32_t)C::kKPanel : (uint32_t)(C::kOffZero - C::kOffK);
+
+            auto issue_sdp = [&](int it) {
+                const uint32_t slot = smem_u32(smem + C::kOffSlots + (it & 1) * C::kSlot);
+                const uint32_t sQ = slot, sDO = slot + C::kQTile;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t ok_ = (uint32_t)((kk >> 2) * C::kKPanel + (kk & 3) * 32);
+                    const uint32_t oq = (uint32_t)((kk >> 2) * C::kQPanel + (kk & 3) * 32);
+                    mma_ss(tS, sdesc_sw128(sK + ok_, 16, 1024), sdesc_sw128(sQ + oq, 16, 1024), id_sdp,
+                           kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t ok_ = (uint32_t)((kk >> 2) * C::kKPanel + (kk & 3) * 32);
+                    const uint32_t oq = (uint32_t)((kk >> 2) * C::kQPanel + (kk & 3) * 32);
+                    mma_ss(tDP, sdesc_sw128(sV + ok_, 16, 1024), sdesc_sw128(sDO + oq, 16, 1024), id_sdp,
+                           kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar_sdp);
+            };
+
+            bool ok = mbar_wait(bar_kv, 0, abort_flag);
+            if (ok && n_it > 0) {
+                ok = mbar_wait(&bar_full[0], 0, abort_flag);
+                tc_fence_after();
+                if (ok)
+                    issue_sdp(0);
+            }
+            for (int it = 0; ok && it < n_it; ++it) {
+                if (!(ok = mbar_wait(bar_ds, (uint32_t)(it & 1), abort_flag)))
+                    break;
+                tc_fence_after();
+                if (it + 1 < n_it) {
+                    if (!(ok = mbar_wait(&bar_full[(it + 1) & 1], (uint32_t)(((it + 1) >> 1) & 1), abort_flag)))
+                        break;
+                    tc_fence_after();
+                    issue_sdp(it + 1);
+                }
+                if (it > 0) {
+                    if (!(ok = mbar_wait(bar_dqfree, (uint32_t)((it - 1) & 1), abort_flag)))
+                        break;
+                    tc_fence_after();
+                }
+                const uint32_t slot = smem_u32(smem + C::kOffSlots + (it & 1) * C::kSlot);
+                const uint32_t sQ = slot, sDO = slot + C::kQTile;
+                // dV += P^T dO ; dK += dS^T Q   (K dimension = 64 query rows)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+                    mma_ss(tDV, sdesc_sw128(sP + kk * 32, 16, 1024),
+                           sdesc_sw128(sDO + kk * 2048, C::kQPanel, 1024), id_grad, acc);
+                    mma_ss(tDK, sdesc_sw128(sDS + kk * 32, 16, 1024),
+                           sdesc_sw128(sQ + kk * 2048, C::kQPanel, 1024), id_grad, acc);
+                }
+                // dQ^T = K^T dS^T   (K dimension = 128 keys)
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tDQ, sdesc_sw128(sK + kk * 2048, lbo_kt, 1024), sdesc_sw128(sDS + kk * 2048, C::kPTile, 1024),
+                           id_dq, kk > 0 ? 1u : 0u);
+                mma_commit(bar_dq);
+                mma_commit(bar_dsfree);
+                mma_commit(&bar_empty[it & 1]);
+            }
+            mma_commit(bar_final);
+            if (!ok)
+                mbar_wait_limited(bar_final, 0, FA_WAIT_LIMIT_CYCLES);
+        }
+      }
+    } else if (warp < 4) {
+        regs_inc<C::kRegsDS>();
+        // ------------------------------------------------------------ P^T / dS^T
+        const int r = warp * 32 + lane;                 // key within the block
+        const int key = kb * 128 + r;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t tS = tmem + lane_off + C::kColS, tDP = tmem + lane_off + C::kColDP;
+        const float sl2 = p.scale_log2;
+        const int delta_q = p.Nk - p.Nq;
+        uint8_t* sP = smem + C::kOffP;
+        uint8_t* sDS = smem + C::kOffDS;
+        bool ok = true;
+        for (int it = 0; it < n_it; ++it) {
+            int h, qb;
+            step_coords(it, h, qb);
+            ok = mbar_wait(bar_sdp, (uint32_t)(it & 1), abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok)
+                break;
+            tc_fence_after();
+            const float* lse2 = reinterpret_cast<const float*>(smem + C::kOffSlots + (it & 1) * C::kSlot + 2 * C::kQTile);
+            const float* dlt = lse2 + 64;
+            uint32_t sr[64], dr[64];
+            tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+            tmem_ld32(tDP, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+            tmem_ld32(tDP + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+            tc_fence_before();
+            // query rows qb*64 + c see this key iff key < Nk and (causal) key <= row + Nk - Nq
+            const int q_first = qb * 64;
+            const int min_row = CAUSAL ? key - delta_q : INT_MIN;   // rows >= min_row see the key
+            const bool key_ok = key < p.Nk;
+            uint32_t pp[32], dd[32];
+#pragma unroll
+            for (int c = 0; c < 64; c += 2) {
+                float pv[2], dv_[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int cc = c + e;
+                    const bool vis = key_ok && (q_first + cc >= min_row);
+                    float pe = ex2_approx(fmaf(__uint_as_float(sr[cc]), sl2, -lse2[cc]));
+                    pe = vis ? pe : 0.f;
+                    pv[e] = pe;
+                    dv_[e] = pe * (__uint_as_float(dr[cc]) - dlt[cc]);
+                }
+                pp[c >> 1] = pack_bf16x2(pv[0], pv[1]);
+                dd[c >> 1] = pack_bf16x2(dv_[0], dv_[1]);
+            }
+            if (it > 0) {
+                ok = mbar_wait(bar_dsfree, (uint32_t)((it - 1) & 1), abort_flag);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok)
+                    break;
+            }
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                *reinterpret_cast<uint4*>(sP + sw128_off(r, ch)) =
+                    make_uint4(pp[4 * ch], pp[4 * ch + 1], pp[4 * ch + 2], pp[4 * ch + 3]);
+                *reinterpret_cast<uint4*>(sDS + sw128_off(r, ch)) =
+                    make_uint4(dd[4 * ch], dd[4 * ch + 1], dd[4 * ch + 2], dd[4 * ch + 3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar_ds);
+        }
+        // ---- epilogue: dK = scale * acc, dV = acc  (bf16)
+        if (ok) {
+            ok = mbar_wait(bar_final, 0, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+        }
+        if (ok) {
+            tc_fence_after();
+            const bool key_ok = key < p.Nk;
+            const size_t krow = ((size_t)kvh * p.Nk + key) * D;
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t a[32], v[32];
+                if (n_it > 0) {
+                    tmem_ld32(tmem + lane_off + C::kColDK + c0, a);
+                    tmem_ld32(tmem + lane_off + C::kColDV + c0, v);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        a[c] = v[c] = 0u;
+                }
+                if (key_ok) {
+                    uint32_t wk[16], wv[16];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        wk[c] = pack_bf16x2(__uint_as_float(a[2 * c]) * p.scale, __uint_as_float(a[2 * c + 1]) * p.scale);
+                        wv[c] = pack_bf16x2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1]));
+                    }
+                    uint4* dk4 = reinterpret_cast<uint4*>(p.dk + krow + c0);
+                    uint4* dv4 = reinterpret_cast<uint4*>(p.dv + krow + c0);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        dk4[c] = make_uint4(wk[4 * c], wk[4 * c + 1], wk[4 * c + 2], wk[4 * c + 3]);
+                        dv4[c] = make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
+                    }
+                }
+            }
+        }
+    } else {
+        regs_dec<C::kRegsDQ>();
+        // ------------------------------------------------------------ dQ^T drain (warps 4-7)
+        const int wq = warp - 4;
+        const int f = wq * 32 + lane;              // feature index = TMEM lane
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        const uint32_t tDQ = tmem + lane_off + C::kColDQ;
+        float* stage = reinterpret_cast<float*>(smem + C::kOffDQ);   // [64][D]
+        bool ok = true;
+        for (int it = 0; it < n_it; ++it) {
+            int h, qb;
+            step_coords(it, h, qb);
+            ok = mbar_wait(bar_dq, (uint32_t)(it & 1), abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok)
+                break;
+            tc_fence_after();
+            uint32_t a[64];
+            tmem_ld32(tDQ, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
+            tmem_ld32(tDQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar_dqfree);
+            // the previous bulk reduce must have finished reading the staging tile
+            if (threadIdx.x == 128)
+                bulk_wait_read0();
+            named_bar_sync(2, 128);
+            if (f < D) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                    stage[c * D + f] = __uint_as_float(a[c]);
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(2, 128);
+            if (threadIdx.x == 128) {
+                const size_t row0 = ((size_t)(b * p.Hq + h) * p.Nq_pad + (size_t)qb * 64) * D;
+                bulk_reduce_add_f32(p.dq_acc + row0, stage, 64 * D * 4);
+                bulk_commit();
+            }
+        }
+        if (threadIdx.x == 128)
+            bulk_wait0();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+}  // namespace fa

@@ -1,0 +1,610 @@
+// fa_api.cu -- the C ABI of libfa (declared in include/fa.h): argument checks,
+// TMA descriptor set-up, kernel selection and launches on the caller's stream.
+//
+// All kernels live in this one translation unit so that they share the device
+// status word g_status without relocatable device code.
+#include "fa.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "bwd.cuh"
+#include "decode.cuh"
+#include "fa_kernels.h"
+#include "fwd.cuh"
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+constexpr float kLog2e = 1.4426950408889634f;
+
+thread_local std::string t_error;
+
+void set_error(const char* fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    t_error = buf;
+}
+
+fa_status_t cuda_fail(cudaError_t e, const char* what)
+{
+    set_error("%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+    return FA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// argument checks (no CUDA call is made before these pass)
+// ---------------------------------------------------------------------------
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status_t check_ptr(const void* p, const char* name)
+{
+    if (p == nullptr) {
+        set_error("%s is NULL", name);
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    if (!aligned16(p)) {
+        set_error("%s is not 16-byte aligned", name);
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    return FA_OK;
+}
+
+fa_status_t check_shape(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) {
+        set_error("sizes must be >= 1 (B=%d Hq=%d Hkv=%d Nq=%d Nk=%d)", B, Hq, Hkv, Nq, Nk);
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    if (Hq % Hkv != 0) {
+        set_error("Hq=%d is not a multiple of Hkv=%d", Hq, Hkv);
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    if (d < 1) {
+        set_error("d=%d must be >= 1", d);
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    if (causal != 0 && causal != 1) {
+        set_error("causal=%d must be 0 or 1", causal);
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    if (!(std::isfinite(scale) && scale > 0.f)) {
+        set_error("scale must be finite and > 0");
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    // index ranges: row counts and TMA coordinates are 32-bit
+    if ((long long)B * Hq * ((long long)Nq + 256) > (1ll << 31) - 1 ||
+        (long long)B * Hkv * ((long long)Nk + 256) > (1ll << 31) - 1) {
+        set_error("problem too large for 32-bit row indices");
+        return FA_ERR_UNSUPPORTED;
+    }
+    if (d != 64 && d != 128) {
+        set_error("d=%d is not supported (64 or 128)", d);
+        return FA_ERR_UNSUPPORTED;
+    }
+    return FA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptors
+// ---------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode()
+{
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 3-D map over a [outer][rows][inner] bf16 tensor, box {64, box_rows, 1}, 128-byte
+// swizzle; rows past `rows` read as zero.
+fa_status_t make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
+                     uint32_t box_rows)
+{
+    EncodeTiledFn enc = get_encode();
+    if (!enc) {
+        set_error("cuTensorMapEncodeTiled is unavailable");
+        return FA_ERR_CUDA;
+    }
+    cuuint64_t dims[3] = {inner, rows, outer};
+    cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
+    cuuint32_t box[3] = {64, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("cuTensorMapEncodeTiled failed (%d)", (int)r);
+        return FA_ERR_CUDA;
+    }
+    return FA_OK;
+}
+
+// Raise a kernel's dynamic shared memory limit once per device.
+template <typename K>
+fa_status_t ensure_smem(K kernel, int bytes)
+{
+    static std::mutex mu;
+    static unsigned long long done = 0;   // bit per device ordinal (< 64)
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaGetDevice");
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev < 64 && (done >> dev) & 1ull)
+        return FA_OK;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaFuncSetAttribute");
+    if (dev < 64)
+        done |= 1ull << dev;
+    return FA_OK;
+}
+
+fa_status_t check_launch(const char* what)
+{
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return cuda_fail(e, what);
+    return FA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int sm_count()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        n <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    return n;
+}
+
+// ---------------------------------------------------------------------------
+// forward (tiled kernel)
+// ---------------------------------------------------------------------------
+template <int D, bool CAUSAL>
+fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                       int Nq, int Nk, float scale, cudaStream_t stream)
+{
+    using C = fa::FwdCfg<D>;
+    CUtensorMap mq, mk, mv;
+    fa_status_t st;
+    if ((st = make_map(&mq, q, D, Nq, (uint64_t)B * Hq, 128)) != FA_OK) return st;
+    if ((st = make_map(&mk, k, D, Nk, (uint64_t)B * Hkv, 128)) != FA_OK) return st;
+    if ((st = make_map(&mv, v, D, Nk, (uint64_t)B * Hkv, 128)) != FA_OK) return st;
+    auto kern = fa::fwd_kernel<D, CAUSAL>;
+    if ((st = ensure_smem(kern, C::kSmemBytes)) != FA_OK) return st;
+    fa::FwdParams p;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.G = Hq / Hkv;
+    p.n_pairs = (Nq + 255) / 256;
+    p.scale_log2 = scale * kLog2e;
+    const long long grid = (long long)p.n_pairs * B * Hq;
+    kern<<<(unsigned)grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
+    return check_launch("fwd_kernel launch");
+}
+
+fa_status_t fwd_tiled(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                      int Nq, int Nk, int d, float scale, int causal, cudaStream_t s)
+{
+    if (d == 128)
+        return causal ? launch_fwd<128, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, s)
+                      : launch_fwd<128, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, s);
+    return causal ? launch_fwd<64, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, s)
+                  : launch_fwd<64, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, s);
+}
+
+// ---------------------------------------------------------------------------
+// split-KV decode
+// ---------------------------------------------------------------------------
+constexpr int kDecodeMaxRows = 16;
+constexpr int kDecodeCtasPerSm = 2;
+
+bool decode_shape(int Hq, int Hkv, int Nq, int d) { return d == 128 && (long long)Nq * (Hq / Hkv) <= kDecodeMaxRows; }
+
+// Number of key chunks: the first count whose CTAs fill whole waves of the GPU
+// to 95% (at least 256 keys per chunk), else the best fill found.
+int decode_splits(int B, int Hkv, int Nk, int requested)
+{
+    const int max_splits = std::max(1, (Nk + fa::DecCfg::kKeys - 1) / fa::DecCfg::kKeys);
+    if (requested > 0)
+        return std::min(requested, max_splits);
+    const long long units = (long long)B * Hkv;
+    const long long slots = (long long)sm_count() * kDecodeCtasPerSm;
+    const int cap = std::max(1, std::min(64, Nk / 256));
+    int best = 1;
+    double best_eff = 0.0;
+    for (int s = 1; s <= cap; ++s) {
+        const long long ctas = units * s;
+        const long long waves = (ctas + slots - 1) / slots;
+        const double eff = (double)ctas / (double)(waves * slots);
+        if (eff >= 0.95)
+            return s;
+        if (eff > best_eff + 1e-9) {
+            best_eff = eff;
+            best = s;
+        }
+    }
+    return best;
+}
+
+struct DecodePlan {
+    int splits, chunk;
+    size_t o_bytes, lse_bytes;
+    size_t total() const { return splits > 1 ? align256(o_bytes) + align256(lse_bytes) : 0; }
+};
+
+DecodePlan decode_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, int requested)
+{
+    DecodePlan pl;
+    int s = decode_splits(B, Hkv, Nk, requested);
+    const int kt = fa::DecCfg::kKeys;
+    pl.chunk = ((Nk + s - 1) / s + kt - 1) / kt * kt;
+    pl.splits = (Nk + pl.chunk - 1) / pl.chunk;
+    const size_t R = (size_t)Nq * (Hq / Hkv);
+    pl.o_bytes = (size_t)B * Hkv * pl.splits * R * d * sizeof(float);
+    pl.lse_bytes = (size_t)B * Hkv * pl.splits * R * sizeof(float);
+    return pl;
+}
+
+fa_status_t launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                          int Nq, int Nk, int d, float scale, int causal, const DecodePlan& pl, void* ws,
+                          cudaStream_t stream)
+{
+    using C = fa::DecCfg;
+    CUtensorMap mk, mv;
+    fa_status_t st;
+    if ((st = make_map(&mk, k, d, Nk, (uint64_t)B * Hkv, 64)) != FA_OK) return st;
+    if ((st = make_map(&mv, v, d, Nk, (uint64_t)B * Hkv, 64)) != FA_OK) return st;
+    if ((st = ensure_smem(fa::decode_split_kernel, C::kSmemBytes)) != FA_OK) return st;
+    fa::DecodeParams p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.k = static_cast<const __nv_bfloat16*>(k);
+    p.v = static_cast<const __nv_bfloat16*>(v);
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.part_o = pl.splits > 1 ? static_cast<float*>(ws) : nullptr;
+    p.part_lse = pl.splits > 1 ? reinterpret_cast<float*>(static_cast<char*>(ws) + align256(pl.o_bytes)) : nullptr;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.G = Hq / Hkv;
+    p.R = Nq * p.G;
+    p.splits = pl.splits;
+    p.chunk = pl.chunk;
+    p.causal = causal;
+    p.scale_log2 = scale * kLog2e;
+    const long long grid = (long long)B * Hkv * pl.splits;
+    fa::decode_split_kernel<<<(unsigned)grid, C::kThreads, C::kSmemBytes, stream>>>(mk, mv, p);
+    if ((st = check_launch("decode_split_kernel launch")) != FA_OK) return st;
+    if (pl.splits > 1) {
+        const long long rows = (long long)B * Hkv * p.R;
+        fa::decode_combine_kernel<<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(p);
+        if ((st = check_launch("decode_combine_kernel launch")) != FA_OK) return st;
+    }
+    return FA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// backward
+// ---------------------------------------------------------------------------
+struct BwdPlan {
+    int Nq_pad;
+    size_t delta_off, lse_off, acc_off, total;
+};
+
+BwdPlan bwd_plan(int B, int Hq, int Nq, int d)
+{
+    BwdPlan pl;
+    pl.Nq_pad = (Nq + 63) / 64 * 64;
+    const size_t rows = (size_t)B * Hq * pl.Nq_pad;
+    pl.delta_off = 0;
+    pl.lse_off = align256(rows * 4);
+    pl.acc_off = pl.lse_off + align256(rows * 4);
+    pl.total = pl.acc_off + align256(rows * d * 4);
+    return pl;
+}
+
+template <int D, bool CAUSAL>
+fa_status_t launch_bwd(const fa::BwdParams& p, const void* q, const void* k, const void* v, const void* dout,
+                       cudaStream_t stream)
+{
+    using C = fa::BwdCfg<D>;
+    fa_status_t st;
+    const long long rows = (long long)p.B * p.Hq * p.Nq_pad;
+    fa::bwd_pre_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p);
+    if ((st = check_launch("bwd_pre_kernel launch")) != FA_OK) return st;
+
+    CUtensorMap mq, mk, mv, mdo;
+    if ((st = make_map(&mq, q, D, p.Nq, (uint64_t)p.B * p.Hq, 64)) != FA_OK) return st;
+    if ((st = make_map(&mdo, dout, D, p.Nq, (uint64_t)p.B * p.Hq, 64)) != FA_OK) return st;
+    if ((st = make_map(&mk, k, D, p.Nk, (uint64_t)p.B * p.Hkv, 128)) != FA_OK) return st;
+    if ((st = make_map(&mv, v, D, p.Nk, (uint64_t)p.B * p.Hkv, 128)) != FA_OK) return st;
+    auto kern = fa::bwd_main_kernel<D, CAUSAL>;
+    if ((st = ensure_smem(kern, C::kSmemBytes)) != FA_OK) return st;
+    const long long grid = (long long)((p.Nk + 127) / 128) * p.B * p.Hkv;
+    kern<<<(unsigned)grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mdo, p);
+    if ((st = check_launch("bwd_main_kernel launch")) != FA_OK) return st;
+
+    const long long n4 = (long long)p.B * p.Hq * p.Nq * D / 4;
+    const long long blocks = std::min<long long>((n4 + 255) / 256, (long long)sm_count() * 8);
+    fa::bwd_post_kernel<D><<<(unsigned)std::max<long long>(blocks, 1), 256, 0, stream>>>(p);
+    return check_launch("bwd_post_kernel launch");
+}
+
+// ---------------------------------------------------------------------------
+// timeout self-test
+// ---------------------------------------------------------------------------
+__global__ void selftest_wait_kernel(long long limit_cycles)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        fa::mbar_init(&bar, 1);
+        fa::fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // nothing arrives on this barrier: the wait must run out and report it
+        if (!fa::mbar_wait_limited(&bar, 0, limit_cycles))
+            atomicOr(&fa::g_status, fa::kStatusTimeout);
+    }
+}
+
+}  // namespace
+
+// ===========================================================================
+// exported entry points
+// ===========================================================================
+extern "C" {
+
+int fa_abi_version(void) { return kAbiVersion; }
+
+const char* fa_status_string(fa_status_t s)
+{
+    switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARGUMENT: return "FA_ERR_INVALID_ARGUMENT";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    }
+    return "FA_ERR_UNKNOWN";
+}
+
+const char* fa_last_error_message(void) { return t_error.c_str(); }
+
+fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                   int Nq, int Nk, int d, float scale, int causal, void* stream)
+{
+    t_error.clear();
+    fa_status_t st;
+    if ((st = check_ptr(q, "q")) || (st = check_ptr(k, "k")) || (st = check_ptr(v, "v")) ||
+        (st = check_ptr(o, "o")))
+        return st;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) {
+        set_error("lse is not 4-byte aligned");
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    if ((st = check_shape(B, Hq, Hkv, Nq, Nk, d, scale, causal)) != FA_OK)
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (!decode_shape(Hq, Hkv, Nq, d))
+        return fwd_tiled(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, s);
+    const DecodePlan pl = decode_plan(B, Hq, Hkv, Nq, Nk, d, 0);
+    void* ws = nullptr;
+    if (pl.total() > 0) {
+        cudaError_t e = cudaMallocAsync(&ws, pl.total(), s);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaMallocAsync (split-KV partials)");
+    }
+    st = launch_decode(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, pl, ws, s);
+    if (ws) {
+        cudaError_t e = cudaFreeAsync(ws, s);
+        if (e != cudaSuccess && st == FA_OK)
+            st = cuda_fail(e, "cudaFreeAsync");
+    }
+    return st;
+}
+
+size_t fa_fwd_splitkv_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || Hq % Hkv != 0 || d < 1 || num_splits < 0)
+        return 0;
+    return decode_plan(B, Hq, Hkv, Nq, Nk, d, num_splits).total();
+}
+
+fa_status_t fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                           int Hkv, int Nq, int Nk, int d, float scale, int causal, int num_splits,
+                           void* workspace, size_t workspace_bytes, void* stream)
+{
+    t_error.clear();
+    fa_status_t st;
+    if ((st = check_ptr(q, "q")) || (st = check_ptr(k, "k")) || (st = check_ptr(v, "v")) ||
+        (st = check_ptr(o, "o")))
+        return st;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) {
+        set_error("lse is not 4-byte aligned");
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    if ((st = check_shape(B, Hq, Hkv, Nq, Nk, d, scale, causal)) != FA_OK)
+        return st;
+    if (num_splits < 0 || num_splits > 256) {
+        set_error("num_splits=%d must be in [0, 256]", num_splits);
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    if (!decode_shape(Hq, Hkv, Nq, d)) {
+        set_error("split-KV needs d = 128 and Nq * Hq / Hkv <= %d", kDecodeMaxRows);
+        return FA_ERR_UNSUPPORTED;
+    }
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) {
+        set_error("workspace is not 256-byte aligned");
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const DecodePlan pl = decode_plan(B, Hq, Hkv, Nq, Nk, d, num_splits);
+    void* ws = workspace;
+    bool owned = false;
+    if (pl.total() > 0) {
+        if (ws == nullptr) {
+            cudaError_t e = cudaMallocAsync(&ws, pl.total(), s);
+            if (e != cudaSuccess)
+                return cuda_fail(e, "cudaMallocAsync (split-KV partials)");
+            owned = true;
+        } else if (workspace_bytes < pl.total()) {
+            set_error("workspace has %zu bytes, %zu needed", workspace_bytes, pl.total());
+            return FA_ERR_WORKSPACE;
+        }
+    }
+    st = launch_decode(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, pl, ws, s);
+    if (owned) {
+        cudaError_t e = cudaFreeAsync(ws, s);
+        if (e != cudaSuccess && st == FA_OK)
+            st = cuda_fail(e, "cudaFreeAsync");
+    }
+    return st;
+}
+
+size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || Hq % Hkv != 0 || d < 1)
+        return 0;
+    return bwd_plan(B, Hq, Nq, d).total;
+}
+
+fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                   void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                   int causal, void* workspace, size_t workspace_bytes, void* stream)
+{
+    t_error.clear();
+    fa_status_t st;
+    if ((st = check_ptr(q, "q")) || (st = check_ptr(k, "k")) || (st = check_ptr(v, "v")) ||
+        (st = check_ptr(o, "o")) || (st = check_ptr(dout, "dout")) || (st = check_ptr(lse, "lse")) ||
+        (st = check_ptr(dq, "dq")) || (st = check_ptr(dk, "dk")) || (st = check_ptr(dv, "dv")))
+        return st;
+    if ((st = check_shape(B, Hq, Hkv, Nq, Nk, d, scale, causal)) != FA_OK)
+        return st;
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) {
+        set_error("workspace is not 256-byte aligned");
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    const BwdPlan pl = bwd_plan(B, Hq, Nq, d);
+    if (workspace && workspace_bytes < pl.total) {
+        set_error("workspace has %zu bytes, %zu needed", workspace_bytes, pl.total);
+        return FA_ERR_WORKSPACE;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    void* ws = workspace;
+    bool owned = false;
+    if (!ws) {
+        cudaError_t e = cudaMallocAsync(&ws, pl.total, s);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaMallocAsync (backward workspace)");
+        owned = true;
+    }
+    fa::BwdParams p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.k = static_cast<const __nv_bfloat16*>(k);
+    p.v = static_cast<const __nv_bfloat16*>(v);
+    p.o = static_cast<const __nv_bfloat16*>(o);
+    p.dout = static_cast<const __nv_bfloat16*>(dout);
+    p.lse = lse;
+    p.dq = static_cast<__nv_bfloat16*>(dq);
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+    char* w = static_cast<char*>(ws);
+    p.delta = reinterpret_cast<float*>(w + pl.delta_off);
+    p.lse_log2 = reinterpret_cast<float*>(w + pl.lse_off);
+    p.dq_acc = reinterpret_cast<float*>(w + pl.acc_off);
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.G = Hq / Hkv;
+    p.Nq_pad = pl.Nq_pad;
+    p.causal = causal;
+    p.scale = scale;
+    p.scale_log2 = scale * kLog2e;
+    if (d == 128)
+        st = causal ? launch_bwd<128, true>(p, q, k, v, dout, s) : launch_bwd<128, false>(p, q, k, v, dout, s);
+    else
+        st = causal ? launch_bwd<64, true>(p, q, k, v, dout, s) : launch_bwd<64, false>(p, q, k, v, dout, s);
+    if (owned) {
+        cudaError_t e = cudaFreeAsync(ws, s);
+        if (e != cudaSuccess && st == FA_OK)
+            st = cuda_fail(e, "cudaFreeAsync");
+    }
+    return st;
+}
+
+fa_status_t fa_check_device_status(void* stream)
+{
+    t_error.clear();
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned int h = 0, zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&h, fa::g_status, sizeof h, 0, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyToSymbolAsync(fa::g_status, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "reading the device status word");
+    if (h & fa::kStatusTimeout) {
+        set_error("a bounded device wait ran out");
+        return FA_ERR_TIMEOUT;
+    }
+    return FA_OK;
+}
+
+fa_status_t fa_selftest_wait_timeout(unsigned timeout_us, void* stream)
+{
+    t_error.clear();
+    int dev = 0, khz = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess)
+        e = cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "querying the clock rate");
+    const long long cycles = (long long)timeout_us * (long long)(khz > 0 ? khz : 2000000) / 1000;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    selftest_wait_kernel<<<1, 32, 0, s>>>(cycles);
+    fa_status_t st = check_launch("selftest_wait_kernel launch");
+    if (st != FA_OK)
+        return st;
+    return fa_check_device_status(stream);
+}
+
+}  // extern "C"

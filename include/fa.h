@@ -1,0 +1,139 @@
+/*
+ * fa.h -- C ABI of libfa, exact scaled-dot-product attention for NVIDIA B200
+ * (sm_100a).
+ *
+ * The operation (page "FlashAttention：为什么少搬数据，反而算得更快", §02, the
+ * S = QK^T / P = softmax(S) / O = PV table, with scale and causal mask present):
+ *
+ *     O = softmax(scale * Q K^T + mask) V,   LSE_i = ln sum_j exp(scale q_i . k_j)
+ *
+ * computed tile by tile with the running statistics (m, l, U) of §04 so that S
+ * and P never reach device memory, and the backward of §05, which recomputes P
+ * block by block from the saved LSE.  MHA, MQA and GQA are selected by Hq / Hkv
+ * (page "FlashAttention技术原理详解"): query head h reads key/value head
+ * h / (Hq / Hkv).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Tensors are dense, row-major, "BHSD": q, o, dout, dq are [B, Hq, Nq, d];
+ *    k, v, dk, dv are [B, Hkv, Nk, d]; lse is [B, Hq, Nq].  q/k/v/o/dout/dq/dk/dv
+ *    hold bf16, lse holds fp32 (natural log of the scaled scores).
+ *  - Every tensor pointer is a DEVICE pointer, non-NULL and 16-byte aligned.
+ *  - d is 64 or 128.  Hq must be a multiple of Hkv.  B, Hq, Hkv, Nq, Nk >= 1.
+ *  - causal is 0 or 1.  With causal = 1, key j is visible to query i iff
+ *    j <= i + (Nk - Nq) (the mask is aligned to the bottom-right corner; for
+ *    Nq = Nk this is the usual lower triangle).  A query row that sees no key
+ *    gets O = 0, LSE = -inf and zero gradients.
+ *  - stream is a cudaStream_t (NULL = the legacy default stream).  All work is
+ *    enqueued on it; no call synchronises the stream or the device.
+ *  - Ownership: the caller owns every buffer; the library keeps no pointer
+ *    after a call returns and frees nothing it did not allocate.
+ *  - Errors: arguments are checked before anything is enqueued; a bad argument
+ *    returns FA_ERR_INVALID_ARGUMENT or FA_ERR_UNSUPPORTED with nothing launched.
+ *    A CUDA launch or allocation failure returns FA_ERR_CUDA;
+ *    fa_last_error_message() describes the last failure of the calling thread.
+ *  - Every wait inside a kernel is bounded.  A wait that runs out records
+ *    FA_ERR_TIMEOUT in a per-device status word and the kernel returns early;
+ *    fa_check_device_status() reads and clears it.
+ *  - Results are equal to the definition up to floating-point ordering, not
+ *    bit for bit (§04: "equivalent results" are not bitwise identical); the
+ *    dq accumulation uses atomics and is not run-to-run deterministic.
+ */
+#ifndef LIBFA_FA_H
+#define LIBFA_FA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARGUMENT = 1, /* NULL / misaligned pointer, bad size or flag */
+    FA_ERR_UNSUPPORTED = 2,      /* valid but not implemented (e.g. d = 96) */
+    FA_ERR_WORKSPACE = 3,        /* workspace given but smaller than required */
+    FA_ERR_CUDA = 4,             /* a CUDA runtime / driver call failed */
+    FA_ERR_TIMEOUT = 5           /* a bounded device wait ran out */
+} fa_status_t;
+
+/* Version of this ABI (incremented on any signature change). */
+int fa_abi_version(void);
+
+/* Static string for a status code. */
+const char* fa_status_string(fa_status_t status);
+
+/* Text of the last failure on the calling thread ("" if none). */
+const char* fa_last_error_message(void);
+
+/*
+ * Forward pass (§03 tiling, §04 online softmax).
+ *   q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] (bf16, read only)
+ *   o [B,Hq,Nq,d] bf16 (written), lse [B,Hq,Nq] fp32 (written; may be NULL when
+ *   the caller does not need it).
+ *   scale multiplies q.k (usually 1/sqrt(d)); it must be finite and > 0.
+ * Shapes with few query rows per kv head (Nq * Hq / Hkv <= 16, the decode shape
+ * of §09) run the split-KV kernels; their partial results need scratch, which
+ * this call allocates stream-ordered with cudaMallocAsync and frees with
+ * cudaFreeAsync on `stream`.  Use fa_fwd_splitkv() to pass the scratch instead.
+ */
+fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                   void* stream);
+
+/*
+ * Split-KV forward for the decode shape (§09: a single query position, scores
+ * of shape 1 x history).  The keys of every (batch, kv head) are cut into
+ * num_splits contiguous chunks; each chunk yields a partial (O_s, lse_s) for all
+ * Hq / Hkv query heads of the group, and a combine kernel merges them with the
+ * rescale-and-add rule of §04 in log form:
+ *     lse = ln sum_s exp(lse_s),   O = sum_s exp(lse_s - lse) O_s.
+ *   Requires Nq * (Hq / Hkv) <= 16.
+ *   num_splits: 0 picks a value from the shape; otherwise 1..256.
+ *   workspace: device scratch of at least fa_fwd_splitkv_workspace_size(...)
+ *   bytes, 256-byte aligned; NULL makes the call allocate it stream-ordered.
+ */
+size_t fa_fwd_splitkv_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                                     int num_splits);
+fa_status_t fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                           int causal, int num_splits, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/*
+ * Backward pass (§05: recompute each needed block of P from the saved LSE).
+ *   q, k, v, o, dout (bf16) and lse (fp32) as produced by fa_fwd with the same
+ *   scale and causal flag.
+ *   dq [B,Hq,Nq,d], dk/dv [B,Hkv,Nk,d] (bf16, written).  dk/dv are summed over
+ *   the Hq / Hkv query heads of each kv group.
+ *   workspace: device scratch of at least fa_bwd_workspace_size(...) bytes,
+ *   256-byte aligned (it holds D = rowsum(dout * o) and the fp32 dq
+ *   accumulator); NULL makes the call allocate it stream-ordered.
+ */
+size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d);
+fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o,
+                   const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                   int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Reads and clears the device status word of the current device.  Synchronises
+ * `stream` (the only call that does).  Returns FA_OK, or FA_ERR_TIMEOUT if a
+ * bounded wait in a kernel ran out since the last check, or FA_ERR_CUDA.
+ */
+fa_status_t fa_check_device_status(void* stream);
+
+/*
+ * Self-test of the bounded-wait machinery: launches one block that waits on a
+ * barrier nothing will arrive on, with a limit of timeout_us microseconds.
+ * The kernel gives up, records FA_ERR_TIMEOUT and returns; the device stays
+ * usable.  Returns what fa_check_device_status() then reports (FA_ERR_TIMEOUT
+ * when the machinery works).  Synchronises `stream`.
+ */
+fa_status_t fa_selftest_wait_timeout(unsigned timeout_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBFA_FA_H */

@@ -1,0 +1,107 @@
+"""Helpers for the GPU parity tests: run libfa on seeded inputs and compare it
+element by element with the fp64 oracle.
+
+Tolerances (fixed by the target statement for bf16 inputs with fp32
+accumulation): max |O - O_ref| <= 1e-2, max |LSE - LSE_ref| <= 1e-3 (rows that
+see no key must give -inf on both sides), and for each gradient
+max |dX - dX_ref| <= 2e-2 * max |dX_ref|.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import exact_attention_114_b200 as fa
+import oracle
+import synth
+
+O_TOL = 1e-2
+LSE_TOL = 1e-3
+GRAD_REL_TOL = 2e-2
+
+
+def to_gpu(x):
+    return {k: v.cuda() for k, v in x.items()}
+
+
+def gpu_forward(xd, w):
+    o, lse = fa.fa_fwd(xd["q"], xd["k"], xd["v"], causal=w.causal, scale=w.scale)
+    torch.cuda.synchronize()
+    fa.fa_check_device_status()
+    return o, lse
+
+
+def gpu_backward(xd, o, lse, w):
+    dq, dk, dv = fa.fa_bwd(xd["q"], xd["k"], xd["v"], o, xd["dout"], lse, causal=w.causal,
+                           scale=w.scale)
+    torch.cuda.synchronize()
+    fa.fa_check_device_status()
+    return dq, dk, dv
+
+
+def assert_o(o_gpu: np.ndarray, o_ref: np.ndarray, what="O"):
+    assert np.isfinite(o_gpu).all(), f"{what}: non-finite values"
+    err = np.max(np.abs(o_gpu - o_ref)) if o_ref.size else 0.0
+    assert err <= O_TOL, f"{what}: max |diff| {err:.3e} > {O_TOL}"
+    return err
+
+
+def assert_lse(l_gpu: np.ndarray, l_ref: np.ndarray):
+    ninf = np.isneginf(l_ref)
+    assert np.array_equal(np.isneginf(l_gpu), ninf), "LSE: -inf rows differ"
+    assert np.isfinite(l_gpu[~ninf]).all(), "LSE: non-finite values"
+    err = np.max(np.abs(l_gpu[~ninf] - l_ref[~ninf])) if (~ninf).any() else 0.0
+    assert err <= LSE_TOL, f"LSE: max |diff| {err:.3e} > {LSE_TOL}"
+    return err
+
+
+def assert_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str):
+    assert np.isfinite(g_gpu).all(), f"{what}: non-finite values"
+    scale = np.max(np.abs(g_ref)) if g_ref.size else 0.0
+    err = np.max(np.abs(g_gpu - g_ref)) if g_ref.size else 0.0
+    if scale == 0.0:
+        assert err == 0.0, f"{what}: expected zeros, max |value| {err}"
+        return 0.0
+    assert err <= GRAD_REL_TOL * scale, f"{what}: max |diff| {err:.3e} > {GRAD_REL_TOL} * {scale:.3e}"
+    return err / scale
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().double().numpy()
+
+
+def check_forward_full(w: synth.Workload):
+    x = synth.make_inputs(w)
+    xd = to_gpu(x)
+    o, lse = gpu_forward(xd, w)
+    o_ref, lse_ref = oracle.fwd(x["q"], x["k"], x["v"], w.scale, w.causal)
+    return assert_o(f64(o), o_ref), assert_lse(f64(lse), lse_ref), (x, xd, o, lse)
+
+
+def check_backward_full(w: synth.Workload, x, xd, o, lse):
+    dq, dk, dv = gpu_backward(xd, o, lse, w)
+    rq, rk, rv = oracle.bwd(x["q"], x["k"], x["v"], x["dout"], w.scale, w.causal)
+    return (assert_grad(f64(dq), rq, "dQ"), assert_grad(f64(dk), rk, "dK"),
+            assert_grad(f64(dv), rv, "dV"))
+
+
+def sample_rows(w: synth.Workload, n_random=16, seed=0):
+    """Flattened query rows (b * Hq + h) * Nq + i: tile edges, scaled rows, the
+    last row, and a few random ones, over a spread of heads and batches."""
+    rng = np.random.default_rng(seed)
+    cand_i = {0, 1, 63, 64, 65, 127, 128, 129, 255, 256, 257, w.Nq // 2, w.Nq - 1}
+    cand_i = sorted(i for i in cand_i if 0 <= i < w.Nq)
+    heads = sorted({0, w.Hq // 2, w.Hq - 1})
+    batches = sorted({0, w.B - 1})
+    rows = [(b * w.Hq + h) * w.Nq + i for b in batches for h in heads for i in cand_i]
+    rows += list(rng.integers(0, w.B * w.Hq * w.Nq, size=n_random))
+    return np.unique(np.array(rows, dtype=np.int64))
+
+
+def sample_keys_cheap(w: synth.Workload, kv_heads=(0,), seed=0):
+    """Flattened keys (b * Hkv + g) * Nk + j whose gradients the oracle can
+    compute quickly: with a causal mask only rows i >= j - (Nk - Nq) see key j,
+    so keys near the end are cheap."""
+    js = sorted({w.Nk - 1, w.Nk - 2, w.Nk - 64, w.Nk - 127, w.Nk - 128, w.Nk - 129})
+    js = [j for j in js if 0 <= j < w.Nk]
+    return np.array([(0 * w.Hkv + g) * w.Nk + j for g in kv_heads for j in js], dtype=np.int64)

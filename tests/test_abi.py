@@ -1,0 +1,128 @@
+"""CPU tests of the C ABI boundary: the library loads, exports every function
+declared in include/fa.h, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_attention_114_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+# a plausible, 16-byte aligned address; never dereferenced because every call
+# below fails validation first
+FAKE = ctypes.c_void_p(0x10000)
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+def declared_functions():
+    text = open(HEADER, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 10, names
+    L = fa.lib()
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in fa.h but not exported by libfa.so"
+
+
+def test_abi_version_and_status_strings():
+    assert fa.abi_version() == 1
+    for code, name in [(0, "FA_OK"), (1, "FA_ERR_INVALID_ARGUMENT"), (2, "FA_ERR_UNSUPPORTED"),
+                       (3, "FA_ERR_WORKSPACE"), (4, "FA_ERR_CUDA"), (5, "FA_ERR_TIMEOUT")]:
+        assert fa.status_string(code) == name
+        # the enum values in the header match
+        assert re.search(rf"\b{name}\s*=\s*{code}\b", open(HEADER, encoding="utf-8").read())
+
+
+def _fwd(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, Hq=2, Hkv=1, Nq=8, Nk=8, d=64,
+         scale=0.125, causal=0):
+    return fa.lib().fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(o=None), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(k=MISALIGNED), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(lse=ctypes.c_void_p(0x10002)), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(B=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(Nq=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(Nk=-3), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(Hq=3, Hkv=2), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(causal=2), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(scale=float("nan")), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(scale=0.0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=256), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=0), fa.FA_ERR_INVALID_ARGUMENT),
+    (dict(B=1 << 20, Hq=1 << 10, Hkv=1 << 10), fa.FA_ERR_UNSUPPORTED),
+])
+def test_fwd_rejects_bad_arguments(kw, status):
+    assert _fwd(**kw) == status
+    assert fa.last_error_message() != ""
+
+
+def test_bwd_rejects_bad_arguments():
+    L = fa.lib()
+    args = [FAKE] * 5 + [FAKE] + [FAKE] * 3
+    base = dict(B=1, Hq=2, Hkv=1, Nq=8, Nk=8, d=128, scale=0.1, causal=1)
+
+    def call(ptrs, ws=None, ws_bytes=0, **over):
+        p = dict(base, **over)
+        return L.fa_bwd(*ptrs, p["B"], p["Hq"], p["Hkv"], p["Nq"], p["Nk"], p["d"], p["scale"],
+                        p["causal"], ws, ws_bytes, None)
+
+    for i in range(9):
+        bad = list(args)
+        bad[i] = None
+        assert call(bad) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(args, d=80) == fa.FA_ERR_UNSUPPORTED
+    # a workspace that is too small is refused before any launch
+    need = fa.fa_bwd_workspace_size(1, 2, 1, 8, 8, 128)
+    assert call(args, ws=ctypes.c_void_p(0x100000), ws_bytes=need - 1) == fa.FA_ERR_WORKSPACE
+    assert call(args, ws=ctypes.c_void_p(0x100010), ws_bytes=need) == fa.FA_ERR_INVALID_ARGUMENT
+
+
+def test_splitkv_rejects_bad_arguments():
+    L = fa.lib()
+
+    def call(Hq=32, Hkv=8, Nq=1, d=128, splits=0, ws=None, ws_bytes=0):
+        return L.fa_fwd_splitkv(FAKE, FAKE, FAKE, FAKE, None, 2, Hq, Hkv, Nq, 4096, d, 0.1, 0,
+                                splits, ws, ws_bytes, None)
+
+    assert call(splits=-1) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(splits=257) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(Nq=8) == fa.FA_ERR_UNSUPPORTED       # 8 * 4 rows per kv head > 16
+    assert call(d=64) == fa.FA_ERR_UNSUPPORTED
+    need = fa.fa_fwd_splitkv_workspace_size(2, 32, 8, 1, 4096, 128, 4)
+    assert need > 0
+    assert call(splits=4, ws=ctypes.c_void_p(0x100000), ws_bytes=need - 16) == fa.FA_ERR_WORKSPACE
+    assert call(splits=4, ws=ctypes.c_void_p(0x100080), ws_bytes=need) == fa.FA_ERR_INVALID_ARGUMENT
+
+
+def test_workspace_sizes():
+    # backward: D and LSE rows (fp32) + fp32 dQ accumulator, rows padded to 64
+    n = fa.fa_bwd_workspace_size(1, 32, 8, 8192, 8192, 128)
+    rows = 32 * 8192
+    assert n == rows * 4 * 2 + rows * 128 * 4
+    assert fa.fa_bwd_workspace_size(1, 1, 1, 65, 65, 64) == 512 * 2 + 128 * 64 * 4  # 65 -> 128 rows
+    assert fa.fa_bwd_workspace_size(0, 1, 1, 1, 1, 64) == 0
+    # split-KV: one partial (O_s, lse_s) per (b, kv head, split, row); one split needs none
+    assert fa.fa_fwd_splitkv_workspace_size(4, 8, 2, 1, 4096, 128, 1) == 0
+    n4 = fa.fa_fwd_splitkv_workspace_size(4, 8, 2, 1, 4096, 128, 4)
+    part_rows = 4 * 2 * 4 * 4
+    assert n4 == part_rows * 128 * 4 + ((part_rows * 4 + 255) // 256) * 256
+
+
+def test_no_gpu_reports_cuda_error_without_crashing():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    st = _fwd(B=1, Hq=1, Hkv=1, Nq=128, Nk=128, d=64)
+    assert st == fa.FA_ERR_CUDA
+    assert fa.last_error_message()
