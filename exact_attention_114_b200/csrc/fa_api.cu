@@ -12,6 +12,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <string>
 
@@ -141,24 +142,24 @@ fa_status_t make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t 
     return FA_OK;
 }
 
-// Raise a kernel's dynamic shared memory limit once per device.
-template <typename K>
-fa_status_t ensure_smem(K kernel, int bytes)
+// Raise a kernel's dynamic shared memory limit once per (kernel, device).
+fa_status_t ensure_smem(const void* kernel, int bytes)
 {
     static std::mutex mu;
-    static unsigned long long done = 0;   // bit per device ordinal (< 64)
+    static std::map<const void*, unsigned long long> done;   // kernel -> bit per device (< 64)
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return cuda_fail(e, "cudaGetDevice");
     std::lock_guard<std::mutex> lk(mu);
-    if (dev < 64 && (done >> dev) & 1ull)
+    unsigned long long& mask = done[kernel];
+    if (dev < 64 && (mask >> dev) & 1ull)
         return FA_OK;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess)
         return cuda_fail(e, "cudaFuncSetAttribute");
     if (dev < 64)
-        done |= 1ull << dev;
+        mask |= 1ull << dev;
     return FA_OK;
 }
 
@@ -197,7 +198,7 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     if ((st = make_map(&mk, k, D, Nk, (uint64_t)B * Hkv, 128)) != FA_OK) return st;
     if ((st = make_map(&mv, v, D, Nk, (uint64_t)B * Hkv, 128)) != FA_OK) return st;
     auto kern = fa::fwd_kernel<D, CAUSAL>;
-    if ((st = ensure_smem(kern, C::kSmemBytes)) != FA_OK) return st;
+    if ((st = ensure_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes)) != FA_OK) return st;
     fa::FwdParams p;
     p.o = static_cast<__nv_bfloat16*>(o);
     p.lse = lse;
@@ -286,7 +287,7 @@ fa_status_t launch_decode(const void* q, const void* k, const void* v, void* o, 
     fa_status_t st;
     if ((st = make_map(&mk, k, d, Nk, (uint64_t)B * Hkv, 64)) != FA_OK) return st;
     if ((st = make_map(&mv, v, d, Nk, (uint64_t)B * Hkv, 64)) != FA_OK) return st;
-    if ((st = ensure_smem(fa::decode_split_kernel, C::kSmemBytes)) != FA_OK) return st;
+    if ((st = ensure_smem(reinterpret_cast<const void*>(fa::decode_split_kernel), C::kSmemBytes)) != FA_OK) return st;
     fa::DecodeParams p;
     p.q = static_cast<const __nv_bfloat16*>(q);
     p.k = static_cast<const __nv_bfloat16*>(k);
@@ -353,7 +354,7 @@ fa_status_t launch_bwd(const fa::BwdParams& p, const void* q, const void* k, con
     if ((st = make_map(&mk, k, D, p.Nk, (uint64_t)p.B * p.Hkv, 128)) != FA_OK) return st;
     if ((st = make_map(&mv, v, D, p.Nk, (uint64_t)p.B * p.Hkv, 128)) != FA_OK) return st;
     auto kern = fa::bwd_main_kernel<D, CAUSAL>;
-    if ((st = ensure_smem(kern, C::kSmemBytes)) != FA_OK) return st;
+    if ((st = ensure_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes)) != FA_OK) return st;
     const long long grid = (long long)((p.Nk + 127) / 128) * p.B * p.Hkv;
     kern<<<(unsigned)grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mdo, p);
     if ((st = check_launch("bwd_main_kernel launch")) != FA_OK) return st;

@@ -55,13 +55,16 @@ def assert_lse(l_gpu: np.ndarray, l_ref: np.ndarray):
     return err
 
 
+# When a reference gradient is identically zero (one key per row: dS = P (dP - D)
+# with P = 1 and dP = D), the relative bound has no scale; the GPU's value is then
+# a pure rounding residue of D = rowsum(dO * O) and is held to this absolute floor.
+ZERO_GRAD_FLOOR = 1e-4
+
+
 def assert_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str):
     assert np.isfinite(g_gpu).all(), f"{what}: non-finite values"
-    scale = np.max(np.abs(g_ref)) if g_ref.size else 0.0
+    scale = max(np.max(np.abs(g_ref)) if g_ref.size else 0.0, ZERO_GRAD_FLOOR)
     err = np.max(np.abs(g_gpu - g_ref)) if g_ref.size else 0.0
-    if scale == 0.0:
-        assert err == 0.0, f"{what}: expected zeros, max |value| {err}"
-        return 0.0
     assert err <= GRAD_REL_TOL * scale, f"{what}: max |diff| {err:.3e} > {GRAD_REL_TOL} * {scale:.3e}"
     return err / scale
 
