@@ -60,6 +60,9 @@ def lib() -> ctypes.CDLL:
             L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, fl, ip, ip, vp,
                                          sz, vp]
             L.fa_fwd_splitkv.restype = ip
+            L.fa_fwd_splitkv_noalloc.argtypes = [vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, fl, ip,
+                                                  ip, vp]
+            L.fa_fwd_splitkv_noalloc.restype = ip
             L.fa_bwd_workspace_size.argtypes = [ip, ip, ip, ip, ip, ip]
             L.fa_bwd_workspace_size.restype = sz
             L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, fl, ip,
@@ -152,6 +155,23 @@ def fa_fwd_splitkv(q, k, v, o=None, lse=None, *, causal=False, scale=None, num_s
     _check(lib().fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq,
                                 Nk, d, scale, int(bool(causal)), int(num_splits), _ptr(workspace),
                                 ws_bytes, _stream(stream)))
+    return o, lse
+
+
+NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024  # FA_SPLITKV_NOALLOC_SCRATCH_BYTES in fa.h
+
+
+def fa_fwd_splitkv_noalloc(q, k, v, o, lse, *, causal=False, scale=None, num_splits=0,
+                           stream=None):
+    """Split-KV forward that allocates nothing on the device: its partials use
+    a fixed array inside the library.  ``o`` and ``lse`` must be given (this
+    wrapper allocates nothing either).  Calls that overlap on the GPU race on
+    the shared array."""
+    B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(lib().fa_fwd_splitkv_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv,
+                                        Nq, Nk, d, scale, int(bool(causal)), int(num_splits),
+                                        _stream(stream)))
     return o, lse
 
 

@@ -319,6 +319,39 @@ fa_status_t launch_decode(const void* q, const void* k, const void* v, void* o, 
 }
 
 // ---------------------------------------------------------------------------
+// split-KV without allocation: partials live in a fixed device array
+// ---------------------------------------------------------------------------
+// Every GPU that loads the library holds this array until the process exits.
+static __device__ __align__(256) unsigned char g_splitkv_scratch[FA_SPLITKV_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_splitkv_scratch on the current device.  In host code the
+// symbol is only a host-side stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+fa_status_t noalloc_scratch(void** out)
+{
+    static std::mutex mu;
+    static void* addr[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) {
+        set_error("device ordinal %d out of range", dev);
+        return FA_ERR_UNSUPPORTED;
+    }
+    std::lock_guard<std::mutex> lk(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_splitkv_scratch);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaGetSymbolAddress (split-KV scratch)");
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return FA_OK;
+}
+
+// ---------------------------------------------------------------------------
 // backward
 // ---------------------------------------------------------------------------
 struct BwdPlan {
@@ -496,6 +529,45 @@ fa_status_t fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o,
             st = cuda_fail(e, "cudaFreeAsync");
     }
     return st;
+}
+
+fa_status_t fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                                   int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                                   int num_splits, void* stream)
+{
+    t_error.clear();
+    fa_status_t st;
+    if ((st = check_ptr(q, "q")) || (st = check_ptr(k, "k")) || (st = check_ptr(v, "v")) ||
+        (st = check_ptr(o, "o")))
+        return st;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) {
+        set_error("lse is not 4-byte aligned");
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    if ((st = check_shape(B, Hq, Hkv, Nq, Nk, d, scale, causal)) != FA_OK)
+        return st;
+    if (num_splits < 0 || num_splits > 256) {
+        set_error("num_splits=%d must be in [0, 256]", num_splits);
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    if (!decode_shape(Hq, Hkv, Nq, d)) {
+        set_error("split-KV needs d = 128 and Nq * Hq / Hkv <= %d", kDecodeMaxRows);
+        return FA_ERR_UNSUPPORTED;
+    }
+    const DecodePlan pl = decode_plan(B, Hq, Hkv, Nq, Nk, d, num_splits);
+    if (pl.total() > (size_t)FA_SPLITKV_NOALLOC_SCRATCH_BYTES) {
+        set_error("this shape needs %zu bytes of split-KV scratch but the fixed scratch holds %zu; "
+                  "use fewer splits or fa_fwd_splitkv with a caller workspace",
+                  pl.total(), (size_t)FA_SPLITKV_NOALLOC_SCRATCH_BYTES);
+        return FA_ERR_WORKSPACE;
+    }
+    void* ws = nullptr;
+    if (pl.total() > 0 && (st = noalloc_scratch(&ws)) != FA_OK)
+        return st;
+    // every partial the combine reads is written by the split pass of this same
+    // call, so nothing in the scratch has to be cleared first
+    return launch_decode(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, pl, ws,
+                         static_cast<cudaStream_t>(stream));
 }
 
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d)

@@ -101,6 +101,35 @@ fa_status_t fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o,
                            void* stream);
 
 /*
+ * Split-KV forward that allocates nothing (the paper has no counterpart; this
+ * is a deployment variant of fa_fwd_splitkv).
+ *
+ * For callers that may not allocate device memory on their call path -- for
+ * example an inference runtime's plugin whose enqueue step must not allocate,
+ * a host program whose allocator owns the whole device memory budget, or a
+ * latency-critical loop where growing a stream-ordered pool would stall.
+ * Arguments, shapes and results are those of fa_fwd_splitkv; only the
+ * workspace argument is gone.  The per-split partials go to one fixed device
+ * array of FA_SPLITKV_NOALLOC_SCRATCH_BYTES inside the library, which every GPU
+ * that loads the library holds until the process exits.
+ *   - No cudaMalloc, cudaFree or other allocating call is made.
+ *   - A shape whose partials need more than FA_SPLITKV_NOALLOC_SCRATCH_BYTES
+ *     (fa_fwd_splitkv_workspace_size() with the same arguments) is rejected
+ *     with FA_ERR_WORKSPACE before anything is launched; fewer splits need less.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current and caches it; make that
+ *     first call before any stream capture.
+ *   - All calls share the one array and it keeps the previous call's contents.
+ *     Nothing in it needs clearing (each call writes every partial it reads),
+ *     but calls that can overlap on the GPU -- on different streams, or on
+ *     different host threads -- race on it and must be serialised by the caller.
+ */
+#define FA_SPLITKV_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+fa_status_t fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                                   int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                                   int causal, int num_splits, void* stream);
+
+/*
  * Backward pass (§05: recompute each needed block of P from the saved LSE).
  *   q, k, v, o, dout (bf16) and lse (fp32) as produced by fa_fwd with the same
  *   scale and causal flag.
