@@ -22,7 +22,6 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -85,59 +84,66 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    """Samples SM clock, max SM clock and throttle reasons through NVML every
+    `period_s` seconds on a background thread while the timed region runs
+    (read-only queries; nothing about the GPU is changed)."""
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, period_s: float = 0.005):
         self.gpu = gpu_index
-        self.proc = None
-        self.out = None
+        self.period = period_s
+        self.samples = []
+        self._stop = None
+        self._thread = None
 
     def __enter__(self):
+        import threading
         try:
-            self.out = open(os.devnull, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
         except Exception:
-            self.proc = None
+            return self
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((sm, mx, rs))
+                except Exception:
+                    pass
+                self._stop.wait(self.period)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except Exception:
-                self.proc.kill()
-                out = ""
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
         return False
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+        if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        import pynvml
+        reasons = set()
+        for _, _, rs in self.samples:
+            for name, const in self.REASONS:
+                if rs & getattr(pynvml, const, 0):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(x[0] for x in self.samples),
+                "sm_max_mhz": max(x[1] for x in self.samples), "reasons": sorted(reasons),
+                "samples": len(self.samples)}
 
 
 # ----------------------------------------------------------------------------
@@ -351,6 +357,37 @@ def run_libfa(args, rank, world, local):
     return 0
 
 
+# ----------------------------------------------------------------------------
+# profiling mode: a few launches of one call on a reduced shape (for ncu)
+# ----------------------------------------------------------------------------
+PROFILE_CASES = {
+    # working sets above the 126 MB L2, a few hundred MB on the device
+    "fwd": ("gqa_8k", dict(Nq=4096, Nk=4096)),
+    "bwd": ("gqa_8k", dict(Nq=4096, Nk=4096)),
+    "decode": ("gqa_decode", dict(B=16)),
+}
+
+
+def run_profile(which: str, launches: int = 3) -> int:
+    """Runs `launches` calls of fa_fwd / fa_bwd / decode on the reduced shape in
+    PROFILE_CASES (the first ones are warm-up for an ncu -s skip)."""
+    import torch
+    import exact_attention_114_b200 as fa
+    name, over = PROFILE_CASES[which]
+    w = synth.WORKLOADS[name].with_(**over)
+    x = {k: v.cuda() for k, v in synth.make_inputs(w).items()}
+    o, lse = fa.fa_fwd(x["q"], x["k"], x["v"], causal=w.causal, scale=w.scale)
+    for _ in range(launches):
+        if which == "bwd":
+            fa.fa_bwd(x["q"], x["k"], x["v"], o, x["dout"], lse, causal=w.causal, scale=w.scale)
+        else:
+            fa.fa_fwd(x["q"], x["k"], x["v"], o, lse, causal=w.causal, scale=w.scale)
+    torch.cuda.synchronize()
+    fa.fa_check_device_status()
+    print(json.dumps({"profile": which, "workload": name, **over, "launches": launches}))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -358,9 +395,13 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["libfa", "reference"], default="libfa")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=sorted(PROFILE_CASES),
+                    help="run a few launches of one call on a reduced shape (for ncu) and exit")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
+    if args.profile:
+        return run_profile(args.profile)
     rank, world, local = dist_env()
     if args.impl == "reference":
         # the CPU oracle: rank 0 alone measures it; other ranks have no work

@@ -17,17 +17,23 @@
 //
 // bwd_main roles (384 threads = 3 warpgroups):
 //   warps 0-3  thread r = key r = TMEM lane r: read S^T and dP^T rows from TMEM,
-//              form P^T and dS^T (bf16) in shared memory; final dK/dV epilogue.
+//              write P^T (bf16) back over S^T in TMEM and dS^T (bf16) into
+//              shared memory; final dK/dV epilogue.
 //   warps 4-7  thread c = dQ^T row c (feature c): move dQ^T from TMEM to a
-//              shared [64 x d] fp32 tile and add it to the dQ accumulator with
-//              one bulk asynchronous reduce-add.
-//   warp 8     TMA loads (K, V once; Q, dO, LSE, D per step, two slots).
+//              shared [32 x d] fp32 tile (two halves per step) and add it to
+//              the dQ accumulator with bulk asynchronous reduce-adds.
+//   warp 8     TMA loads (K, V once; Q, dO, LSE, D per step, three slots so a
+//              step's loads are issued two steps ahead).
 //   warps 10-11 complete the third warpgroup (which gives registers away).
 //   warp 9     one thread issues the tcgen05.mma ops, per step `it`:
 //                S^T(it+1) = K Q^T, dP^T(it+1) = V dO^T      (after P/dS of it)
-//                dV += P^T(it) dO, dK += dS^T(it) Q, dQ^T(it) = K^T dS^T(it)
-//              so the softmax of step it+1 overlaps the gradient MMAs of it.
-// Tensor memory (512 columns): dK | dV (d each) | S^T 64 | dP^T 64 | dQ^T 64.
+//                dV += P^T(it) dO  (P^T read from tensor memory),
+//                dK += dS^T(it) Q, dQ^T(it) = K^T dS^T(it)
+//              so the softmax of step it+1 overlaps the gradient MMAs of it;
+//              S^T / P^T and dS^T are double-buffered so neither side waits
+//              for the other's previous step.
+// Tensor memory (512 columns): dK | dV (d each) | S^T/P^T x2 (64 each) | dP^T 64
+// | dQ^T 64  (for d = 64 the last 128 columns are unused).
 #pragma once
 
 #include "sm100.cuh"
@@ -138,26 +144,26 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(BwdParams p)
 template <int D>
 struct BwdCfg {
     static constexpr int kThreads = 384;
-    // registers per thread after the split: 128 x (240 + 120 + 80) <= 384 x 168
-    static constexpr uint32_t kRegsDS = 240, kRegsDQ = 120, kRegsOther = 80;
+    // registers per thread after the split: 128 x (208 + 112 + 144) <= 384 x 168
+    static constexpr uint32_t kRegsDS = 208, kRegsDQ = 112, kRegsOther = 144;
     static constexpr int kKPanel = 128 * 128;          // 128 keys x 64 bf16
     static constexpr int kKTile = (D / 64) * kKPanel;  // K or V block
     static constexpr int kQPanel = 64 * 128;           // 64 rows x 64 bf16
     static constexpr int kQTile = (D / 64) * kQPanel;  // Q or dO block
     static constexpr int kSlot = 2 * kQTile + 1024;    // Q, dO, lse_log2[64], delta[64] (1 KB-aligned)
-    static constexpr int kPTile = 128 * 128;           // P^T or dS^T: 128 keys x 64 q bf16
+    static constexpr int kSlots = 3;                   // step slots in flight (TMA latency cover)
+    static constexpr int kPTile = 128 * 128;           // dS^T: 128 keys x 64 q bf16
     static constexpr int kOffK = 0;
     static constexpr int kOffV = kOffK + kKTile;
     static constexpr int kOffZero = kOffV + kKTile;                 // zero panel (D = 64 only)
     static constexpr int kOffSlots = kOffZero + (D == 64 ? kKPanel : 0);
-    static constexpr int kOffP = kOffSlots + 2 * kSlot;
-    static constexpr int kOffDS = kOffP + kPTile;
-    static constexpr int kOffDQ = kOffDS + kPTile;                  // fp32 [64][D] staging
-    static constexpr int kOffBar = kOffDQ + 64 * D * 4;
+    static constexpr int kOffDS = kOffSlots + kSlots * kSlot;       // dS^T, two buffers
+    static constexpr int kOffDQ = kOffDS + 2 * kPTile;              // fp32 [32][D] staging (half a step)
+    static constexpr int kOffBar = kOffDQ + 32 * D * 4;
     static constexpr int kSmemBytes = kOffBar + 256 + 1024;
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kColDK = 0, kColDV = D, kColS = 2 * D, kColDP = 2 * D + 64,
-                              kColDQ = 2 * D + 128;
+    static constexpr uint32_t kColDK = 0, kColDV = D, kColS = 2 * D, kColDP = 2 * D + 128,
+                              kColDQ = 2 * D + 192;
 };
 
 __device__ __forceinline__ void bwd_q_range(const BwdParams& p, int kb, int& qb0, int& nqb)
@@ -190,15 +196,15 @@ __global__ void __launch_bounds__(384, 1)
     uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* bar_kv = bars;            // K, V landed
-    uint64_t* bar_full = bars + 1;      // [2] step slot landed
-    uint64_t* bar_empty = bars + 3;     // [2] step slot released
-    uint64_t* bar_sdp = bars + 5;       // S^T and dP^T of a step in TMEM
-    uint64_t* bar_ds = bars + 6;        // P^T, dS^T of a step in smem (count 4)
-    uint64_t* bar_dsfree = bars + 7;    // gradient MMAs of a step done (smem P/dS free)
-    uint64_t* bar_dq = bars + 8;        // dQ^T of a step in TMEM
-    uint64_t* bar_dqfree = bars + 9;    // dQ^T read out of TMEM (count 4)
-    uint64_t* bar_final = bars + 10;    // all MMAs done
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+    uint64_t* bar_full = bars + 1;      // [kSlots] step slot landed
+    uint64_t* bar_empty = bars + 4;     // [kSlots] step slot released
+    uint64_t* bar_sdp = bars + 7;       // S^T and dP^T of a step in TMEM
+    uint64_t* bar_ds = bars + 8;        // P^T (TMEM), dS^T (smem) of a step written (count 4)
+    uint64_t* bar_gdone = bars + 9;     // [2] gradient MMAs of a step done (its dS^T buffer free)
+    uint64_t* bar_dq = bars + 11;       // dQ^T of a step in TMEM
+    uint64_t* bar_dqfree = bars + 12;   // dQ^T read out of TMEM (count 4)
+    uint64_t* bar_final = bars + 13;    // all MMAs done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = warp_id(), lane = lane_id();
@@ -217,13 +223,14 @@ __global__ void __launch_bounds__(384, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(bar_kv, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < C::kSlots; ++s) {
             mbar_init(&bar_full[s], 1);
             mbar_init(&bar_empty[s], 1);
         }
         mbar_init(bar_sdp, 1);
         mbar_init(bar_ds, 4);
-        mbar_init(bar_dsfree, 1);
+        mbar_init(&bar_gdone[0], 1);
+        mbar_init(&bar_gdone[1], 1);
         mbar_init(bar_dq, 1);
         mbar_init(bar_dqfree, 4);
         mbar_init(bar_final, 1);
@@ -266,8 +273,8 @@ __global__ void __launch_bounds__(384, 1)
             }
             int issued = 0;
             for (int it = 0; it < n_it; ++it) {
-                const int s = it & 1;
-                if (!mbar_wait(&bar_empty[s], (uint32_t)((it >> 1) & 1) ^ 1u, abort_flag))
+                const int s = it % C::kSlots;
+                if (!mbar_wait(&bar_empty[s], (uint32_t)((it / C::kSlots) & 1) ^ 1u, abort_flag))
                     break;
                 int h, qb;
                 step_coords(it, h, qb);
@@ -285,8 +292,9 @@ __global__ void __launch_bounds__(384, 1)
             }
             if (*abort_flag) {
                 mbar_wait_limited(bar_kv, 0, FA_WAIT_LIMIT_CYCLES);
-                for (int i = max(0, issued - 2); i < issued; ++i)
-                    mbar_wait_limited(&bar_full[i & 1], (uint32_t)((i >> 1) & 1), FA_WAIT_LIMIT_CYCLES);
+                for (int i = max(0, issued - C::kSlots); i < issued; ++i)
+                    mbar_wait_limited(&bar_full[i % C::kSlots], (uint32_t)((i / C::kSlots) & 1),
+                                      FA_WAIT_LIMIT_CYCLES);
             }
         }
       } else if (warp == 9) {
@@ -295,30 +303,36 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t id_sdp = idesc_bf16_f32(128, 64, false, false);   // S^T, dP^T
             const uint32_t id_grad = idesc_bf16_f32(128, D, false, true);    // dV, dK
             const uint32_t id_dq = idesc_bf16_f32(128, 64, true, true);      // dQ^T
-            const uint32_t sK = smem_u32(smem + C::kOffK), sV = smem_u32(smem + C::kOffV);
-            const uint32_t sP = smem_u32(smem + C::kOffP), sDS = smem_u32(smem + C::kOffDS);
             const uint32_t tDK = tmem + C::kColDK, tDV = tmem + C::kColDV, tS = tmem + C::kColS,
                            tDP = tmem + C::kColDP, tDQ = tmem + C::kColDQ;
-            // K^T as the M = 128 operand of dQ^T: d panels are 16 KB apart (for d = 64
-            // the second "panel" is the zero panel right after V... placed at kOffZero)
+            // base descriptors; a byte offset `o` inside an operand is added as o >> 4
+            // to the start-address field (addresses stay below 256 KB, no carry)
+            const uint64_t dK_k = sdesc_sw128(smem_u32(smem + C::kOffK), 16, 1024);      // K as K-major A
+            const uint64_t dV_k = sdesc_sw128(smem_u32(smem + C::kOffV), 16, 1024);      // V as K-major A
+            // K^T as the M = 128 (feature) MN-major operand of dQ^T: the second 64-feature
+            // panel is 16 KB on for d = 128, the zero panel for d = 64
             const uint32_t lbo_kt = (D == 128) ? (uint32_t)C::kKPanel : (uint32_t)(C::kOffZero - C::kOffK);
+            const uint64_t dK_mn = sdesc_sw128(smem_u32(smem + C::kOffK), lbo_kt, 1024);
+            const uint64_t dSlot_k = sdesc_sw128(smem_u32(smem + C::kOffSlots), 16, 1024);   // Q / dO K-major
+            const uint64_t dSlot_mn = sdesc_sw128(smem_u32(smem + C::kOffSlots), C::kQPanel, 1024);
+            const uint64_t dDS_k = sdesc_sw128(smem_u32(smem + C::kOffDS), 16, 1024);
+            const uint64_t dDS_mn = sdesc_sw128(smem_u32(smem + C::kOffDS), C::kPTile, 1024);
+            auto off = [](uint32_t bytes) { return (uint64_t)(bytes >> 4); };
 
             auto issue_sdp = [&](int it) {
-                const uint32_t slot = smem_u32(smem + C::kOffSlots + (it & 1) * C::kSlot);
-                const uint32_t sQ = slot, sDO = slot + C::kQTile;
+                const uint32_t so = (uint32_t)((it % C::kSlots) * C::kSlot);
+                const uint32_t tSb = tS + (uint32_t)(64 * (it & 1));
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ok_ = (uint32_t)((kk >> 2) * C::kKPanel + (kk & 3) * 32);
                     const uint32_t oq = (uint32_t)((kk >> 2) * C::kQPanel + (kk & 3) * 32);
-                    mma_ss(tS, sdesc_sw128(sK + ok_, 16, 1024), sdesc_sw128(sQ + oq, 16, 1024), id_sdp,
-                           kk > 0 ? 1u : 0u);
+                    mma_ss(tSb, dK_k + off(ok_), dSlot_k + off(so + oq), id_sdp, kk > 0 ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ok_ = (uint32_t)((kk >> 2) * C::kKPanel + (kk & 3) * 32);
                     const uint32_t oq = (uint32_t)((kk >> 2) * C::kQPanel + (kk & 3) * 32);
-                    mma_ss(tDP, sdesc_sw128(sV + ok_, 16, 1024), sdesc_sw128(sDO + oq, 16, 1024), id_sdp,
-                           kk > 0 ? 1u : 0u);
+                    mma_ss(tDP, dV_k + off(ok_), dSlot_k + off(so + C::kQTile + oq), id_sdp, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar_sdp);
             };
@@ -335,35 +349,34 @@ __global__ void __launch_bounds__(384, 1)
                     break;
                 tc_fence_after();
                 if (it + 1 < n_it) {
-                    if (!(ok = mbar_wait(&bar_full[(it + 1) & 1], (uint32_t)(((it + 1) >> 1) & 1), abort_flag)))
+                    const int in = it + 1;
+                    if (!(ok = mbar_wait(&bar_full[in % C::kSlots], (uint32_t)((in / C::kSlots) & 1), abort_flag)))
                         break;
                     tc_fence_after();
-                    issue_sdp(it + 1);
+                    issue_sdp(in);
                 }
                 if (it > 0) {
                     if (!(ok = mbar_wait(bar_dqfree, (uint32_t)((it - 1) & 1), abort_flag)))
                         break;
                     tc_fence_after();
                 }
-                const uint32_t slot = smem_u32(smem + C::kOffSlots + (it & 1) * C::kSlot);
-                const uint32_t sQ = slot, sDO = slot + C::kQTile;
+                const uint32_t so = (uint32_t)((it % C::kSlots) * C::kSlot);
+                const uint32_t dso = (uint32_t)((it & 1) * C::kPTile);
+                const uint32_t tP = tS + (uint32_t)(64 * (it & 1));   // P^T: 32 columns of bf16 pairs
                 // dV += P^T dO ; dK += dS^T Q   (K dimension = 64 query rows)
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                    mma_ss(tDV, sdesc_sw128(sP + kk * 32, 16, 1024),
-                           sdesc_sw128(sDO + kk * 2048, C::kQPanel, 1024), id_grad, acc);
-                    mma_ss(tDK, sdesc_sw128(sDS + kk * 32, 16, 1024),
-                           sdesc_sw128(sQ + kk * 2048, C::kQPanel, 1024), id_grad, acc);
+                    mma_ts(tDV, tP + (uint32_t)(kk * 8), dSlot_mn + off(so + C::kQTile + kk * 2048), id_grad, acc);
+                    mma_ss(tDK, dDS_k + off(dso + kk * 32), dSlot_mn + off(so + kk * 2048), id_grad, acc);
                 }
                 // dQ^T = K^T dS^T   (K dimension = 128 keys)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tDQ, sdesc_sw128(sK + kk * 2048, lbo_kt, 1024), sdesc_sw128(sDS + kk * 2048, C::kPTile, 1024),
-                           id_dq, kk > 0 ? 1u : 0u);
+                    mma_ss(tDQ, dK_mn + off(kk * 2048), dDS_mn + off(dso + kk * 2048), id_dq, kk > 0 ? 1u : 0u);
                 mma_commit(bar_dq);
-                mma_commit(bar_dsfree);
-                mma_commit(&bar_empty[it & 1]);
+                mma_commit(&bar_gdone[it & 1]);
+                mma_commit(&bar_empty[it % C::kSlots]);
             }
             mma_commit(bar_final);
             if (!ok)
@@ -379,8 +392,6 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t tS = tmem + lane_off + C::kColS, tDP = tmem + lane_off + C::kColDP;
         const float sl2 = p.scale_log2;
         const int delta_q = p.Nk - p.Nq;
-        uint8_t* sP = smem + C::kOffP;
-        uint8_t* sDS = smem + C::kOffDS;
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
             int h, qb;
@@ -390,48 +401,51 @@ __global__ void __launch_bounds__(384, 1)
             if (!ok)
                 break;
             tc_fence_after();
-            const float* lse2 = reinterpret_cast<const float*>(smem + C::kOffSlots + (it & 1) * C::kSlot + 2 * C::kQTile);
+            const float* lse2 =
+                reinterpret_cast<const float*>(smem + C::kOffSlots + (it % C::kSlots) * C::kSlot + 2 * C::kQTile);
             const float* dlt = lse2 + 64;
+            const uint32_t tSb = tS + (uint32_t)(64 * (it & 1));
             uint32_t sr[64], dr[64];
-            tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-            tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-            tmem_ld32(tDP, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
-            tmem_ld32(tDP + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
-            tc_fence_before();
+            tmem_ld64x2(tSb, tDP, sr, dr);
             // query rows qb*64 + c see this key iff key < Nk and (causal) key <= row + Nk - Nq
             const int q_first = qb * 64;
             const int min_row = CAUSAL ? key - delta_q : INT_MIN;   // rows >= min_row see the key
             const bool key_ok = key < p.Nk;
             uint32_t pp[32], dd[32];
+            const float2 sl22 = make_float2(sl2, sl2);
+            // rows >= min_row see the key; whole 64-row block visible in most steps
+            const bool all_vis = key_ok && (q_first >= min_row);
 #pragma unroll
             for (int c = 0; c < 64; c += 2) {
-                float pv[2], dv_[2];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int cc = c + e;
-                    const bool vis = key_ok && (q_first + cc >= min_row);
-                    float pe = ex2_approx(fmaf(__uint_as_float(sr[cc]), sl2, -lse2[cc]));
-                    pe = vis ? pe : 0.f;
-                    pv[e] = pe;
-                    dv_[e] = pe * (__uint_as_float(dr[cc]) - dlt[cc]);
+                const float2 nl = make_float2(-lse2[c], -lse2[c + 1]);
+                const float2 x = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl22, nl);
+                float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                if (!all_vis) {
+                    pv.x = (key_ok && q_first + c >= min_row) ? pv.x : 0.f;
+                    pv.y = (key_ok && q_first + c + 1 >= min_row) ? pv.y : 0.f;
                 }
-                pp[c >> 1] = pack_bf16x2(pv[0], pv[1]);
-                dd[c >> 1] = pack_bf16x2(dv_[0], dv_[1]);
+                // dS = P * (dP - D)
+                const float2 dd2 = make_float2(__uint_as_float(dr[c]) - dlt[c], __uint_as_float(dr[c + 1]) - dlt[c + 1]);
+                pp[c >> 1] = pack_bf16x2(pv.x, pv.y);
+                dd[c >> 1] = pack_bf16x2(pv.x * dd2.x, pv.y * dd2.y);
             }
-            if (it > 0) {
-                ok = mbar_wait(bar_dsfree, (uint32_t)((it - 1) & 1), abort_flag);
+            // P^T over this step's S^T columns (the dV MMA reads it from there)
+            tmem_st32(tSb, pp);
+            // dS^T into this step's buffer, free once the gradient MMAs of step it-2 are done
+            if (it >= 2) {
+                ok = mbar_wait(&bar_gdone[it & 1], (uint32_t)((it >> 1) & 1) ^ 1u, abort_flag);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok)
                     break;
             }
+            uint8_t* sDS = smem + C::kOffDS + (it & 1) * C::kPTile;
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                *reinterpret_cast<uint4*>(sP + sw128_off(r, ch)) =
-                    make_uint4(pp[4 * ch], pp[4 * ch + 1], pp[4 * ch + 2], pp[4 * ch + 3]);
+            for (int ch = 0; ch < 8; ++ch)
                 *reinterpret_cast<uint4*>(sDS + sw128_off(r, ch)) =
                     make_uint4(dd[4 * ch], dd[4 * ch + 1], dd[4 * ch + 2], dd[4 * ch + 3]);
-            }
             fence_proxy_async_smem();
+            tmem_st_wait();
+            tc_fence_before();
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(bar_ds);
@@ -480,7 +494,7 @@ __global__ void __launch_bounds__(384, 1)
         const int f = wq * 32 + lane;              // feature index = TMEM lane
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
         const uint32_t tDQ = tmem + lane_off + C::kColDQ;
-        float* stage = reinterpret_cast<float*>(smem + C::kOffDQ);   // [64][D]
+        float* stage = reinterpret_cast<float*>(smem + C::kOffDQ);   // [32][D]
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
             int h, qb;
@@ -491,27 +505,30 @@ __global__ void __launch_bounds__(384, 1)
                 break;
             tc_fence_after();
             uint32_t a[64];
-            tmem_ld32(tDQ, *reinterpret_cast<uint32_t(*)[32]>(&a[0]));
-            tmem_ld32(tDQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32]));
+            tmem_ld64(tDQ, a);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(bar_dqfree);
-            // the previous bulk reduce must have finished reading the staging tile
-            if (threadIdx.x == 128)
-                bulk_wait_read0();
-            named_bar_sync(2, 128);
-            if (f < D) {
+            // two halves of 32 query rows through a 16 KB staging tile
 #pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    stage[c * D + f] = __uint_as_float(a[c]);
-            }
-            fence_proxy_async_smem();
-            named_bar_sync(2, 128);
-            if (threadIdx.x == 128) {
-                const size_t row0 = ((size_t)(b * p.Hq + h) * p.Nq_pad + (size_t)qb * 64) * D;
-                bulk_reduce_add_f32(p.dq_acc + row0, stage, 64 * D * 4);
-                bulk_commit();
+            for (int hf = 0; hf < 2; ++hf) {
+                // the previous bulk reduce must have finished reading the staging tile
+                if (threadIdx.x == 128)
+                    bulk_wait_read0();
+                named_bar_sync(2, 128);
+                if (f < D) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        stage[c * D + f] = __uint_as_float(a[32 * hf + c]);
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(2, 128);
+                if (threadIdx.x == 128) {
+                    const size_t row0 = ((size_t)(b * p.Hq + h) * p.Nq_pad + (size_t)qb * 64 + 32 * hf) * D;
+                    bulk_reduce_add_f32(p.dq_acc + row0, stage, 32 * D * 4);
+                    bulk_commit();
+                }
             }
         }
         if (threadIdx.x == 128)

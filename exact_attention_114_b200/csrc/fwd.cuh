@@ -39,8 +39,8 @@ constexpr float kLn2 = 0.69314718055994530942f;
 template <int D>
 struct FwdCfg {
     static constexpr int kThreads = 384;
-    // registers per thread after the split: 2 x 128 x 224 + 128 x 56 = 384 x 168
-    static constexpr uint32_t kRegsSoftmax = 224, kRegsOther = 56;
+    // registers per thread after the split: 2 x 128 x 208 + 128 x 80 <= 384 x 168
+    static constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 80;
     static constexpr int kTileBytes = 128 * D * 2;   // a 128-row Q, K or V tile
     static constexpr int kPanelBytes = 128 * 128;    // 128 rows x 64 bf16
     static constexpr int kStages = (D == 128) ? 4 : 8;
@@ -82,8 +82,8 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* bar_full = bar_q + 2;                    // [S]  ring slot landed
     uint64_t* bar_empty = bar_full + C::kStages;       // [S]  ring slot released
     uint64_t* bar_s = bar_empty + C::kStages;          // [2]  S tile ready in TMEM
-    uint64_t* bar_p = bar_s + 2;                       // [2]  P (and O rescale) written
-    uint64_t* bar_o = bar_p + 2;                       // [2]  last P.V of a tile done
+    uint64_t* bar_p = bar_s + 2;                       // [2][2] P half h (and O rescale) written
+    uint64_t* bar_o = bar_p + 4;                       // [2]  last P.V of a tile done
     uint64_t* bar_drain = bar_o + 2;                   // [1]  MMA drain on abort
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -107,7 +107,8 @@ __global__ void __launch_bounds__(384, 1)
         for (int t = 0; t < 2; ++t) {
             mbar_init(&bar_q[t], 1);
             mbar_init(&bar_s[t], 1);
-            mbar_init(&bar_p[t], 4);
+            mbar_init(&bar_p[2 * t], 4);
+            mbar_init(&bar_p[2 * t + 1], 4);
             mbar_init(&bar_o[t], 1);
         }
         for (int s = 0; s < C::kStages; ++s) {
@@ -191,25 +192,33 @@ __global__ void __launch_bounds__(384, 1)
                     ok = mbar_wait(&bar_q[t], 0, abort_flag);
             tc_fence_after();
 
-            auto slot_addr = [&](int idx) { return sKVa + (uint32_t)((idx % C::kStages) * C::kTileBytes); };
+            // base descriptors; a byte offset `o` inside an operand is added as o >> 4
+            // to the start-address field (addresses stay below 256 KB, no carry)
+            const uint64_t dQ_k = sdesc_sw128(sQa, 16, 1024);                   // Q tiles, K-major
+            const uint64_t dKV_k = sdesc_sw128(sKVa, 16, 1024);                 // ring as K (K-major)
+            const uint64_t dKV_mn = sdesc_sw128(sKVa, C::kPanelBytes, 1024);    // ring as V (MN-major)
+            auto off = [](uint32_t bytes) { return (uint64_t)(bytes >> 4); };
+            auto slot_off = [&](int idx) { return (uint32_t)((idx % C::kStages) * C::kTileBytes); };
             auto phase = [&](int idx) { return (uint32_t)((idx / C::kStages) & 1); };
             auto issue_S = [&](int t, int j) {
-                const uint32_t ka = slot_addr(2 * j);
-                const uint32_t qa = sQa + (uint32_t)(t * C::kTileBytes);
+                const uint32_t ko = slot_off(2 * j);
+                const uint32_t qo = (uint32_t)(t * C::kTileBytes);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (uint32_t)((kk >> 2) * C::kPanelBytes + (kk & 3) * 32);
-                    mma_ss(tS[t], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idS,
-                           kk > 0 ? 1u : 0u);
+                    const uint32_t o = (uint32_t)((kk >> 2) * C::kPanelBytes + (kk & 3) * 32);
+                    mma_ss(tS[t], dQ_k + off(qo + o), dKV_k + off(ko + o), idS, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(&bar_s[t]);
             };
-            auto issue_PV = [&](int t, int j) {
-                const uint32_t va = slot_addr(2 * j + 1);
+            // keys 64*half .. 64*half+63 of block j (P columns 32*half .. 32*half+31)
+            auto issue_PV = [&](int t, int j, int half) {
+                const uint32_t vo = slot_off(2 * j + 1);
 #pragma unroll
-                for (int kk = 0; kk < 128 / 16; ++kk)
-                    mma_ts(tO[t], tS[t] + (uint32_t)(kk * 8), sdesc_sw128(va + (uint32_t)(kk * 2048), C::kPanelBytes, 1024),
-                           idPV, (j > 0 || kk > 0) ? 1u : 0u);
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const int kk = 4 * half + k4;
+                    mma_ts(tO[t], tS[t] + (uint32_t)(kk * 8), dKV_mn + off(vo + (uint32_t)(kk * 2048)), idPV,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+                }
             };
 
             if (ok && n_iter > 0) {
@@ -230,10 +239,14 @@ __global__ void __launch_bounds__(384, 1)
                 bool k_ready = false;
                 for (int t = 0; t < 2 && ok; ++t) {
                     if (j < nblk[t]) {
-                        if (!(ok = mbar_wait(&bar_p[t], (uint32_t)(j & 1), abort_flag)))
+                        for (int hf = 0; hf < 2 && ok; ++hf) {
+                            if (!(ok = mbar_wait(&bar_p[2 * t + hf], (uint32_t)(j & 1), abort_flag)))
+                                break;
+                            tc_fence_after();
+                            issue_PV(t, j, hf);
+                        }
+                        if (!ok)
                             break;
-                        tc_fence_after();
-                        issue_PV(t, j);
                         if (j == nblk[t] - 1)
                             mma_commit(&bar_o[t]);
                     }
@@ -281,10 +294,7 @@ __global__ void __launch_bounds__(384, 1)
                 break;
             tc_fence_after();
             uint32_t sr[128];
-            tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-            tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-            tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-            tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+            tmem_ld128(tS, sr);
             float s[128];
 #pragma unroll
             for (int c = 0; c < 128; ++c)
@@ -299,11 +309,14 @@ __global__ void __launch_bounds__(384, 1)
                     if (kb + c > lim)
                         s[c] = -INFINITY;
             }
-            float mx = s[0];
+            // row max: two independent chains of three-input max
+            float mxa = fmaxf(s[0], s[1]), mxb = fmaxf(s[2], s[3]);
 #pragma unroll
-            for (int c = 1; c < 128; ++c)
-                mx = fmaxf(mx, s[c]);
-            const float m_blk = mx * sl2;
+            for (int c = 4; c < 128; c += 4) {
+                mxa = fmax3(mxa, s[c], s[c + 1]);
+                mxb = fmax3(mxb, s[c + 2], s[c + 3]);
+            }
+            const float m_blk = fmaxf(mxa, mxb) * sl2;
             float a = 1.f;
             bool resc = false;
             if (m_blk > m_ref + kRescaleLog2) {
@@ -324,23 +337,29 @@ __global__ void __launch_bounds__(384, 1)
                 }
             }
             const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-            float rs = 0.f;
-            uint32_t pk[64];
+            const float2 sl22 = make_float2(sl2, sl2), nm2 = make_float2(neg_m, neg_m);
+            float2 acc = make_float2(0.f, 0.f);
+            // P in two halves of 64 keys: the MMA warp starts P.V on the first
+            // half while the second is still being exponentiated
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                const float p0 = ex2_approx(fmaf(s[2 * c], sl2, neg_m));
-                const float p1 = ex2_approx(fmaf(s[2 * c + 1], sl2, neg_m));
-                rs += p0 + p1;
-                pk[c] = pack_bf16x2(p0, p1);
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const int e = 64 * hf + 2 * c;
+                    const float2 x = ffma2(make_float2(s[e], s[e + 1]), sl22, nm2);
+                    const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                    acc = fadd2(acc, pv);
+                    pk[c] = pack_bf16x2(pv.x, pv.y);
+                }
+                tmem_st32(tS + (uint32_t)(32 * hf), pk);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&bar_p[2 * t + hf]);
             }
-            tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-            tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&bar_p[t]);
-            l += rs;
+            l += acc.x + acc.y;
         }
 
         // ---- epilogue: O = U / l (bf16), LSE = (m + log2 l) ln 2
