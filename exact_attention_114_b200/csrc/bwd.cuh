@@ -26,7 +26,8 @@
 //              step's loads are issued two steps ahead).
 //   warps 10-11 complete the third warpgroup (which gives registers away).
 //   warp 9     one thread issues the tcgen05.mma ops, per step `it`:
-//                S^T(it+1) = K Q^T, dP^T(it+1) = V dO^T      (after P/dS of it)
+//                S^T(it+1) = K Q^T, dP^T(it+1) = V dO^T  (as soon as warps 0-3
+//                                                        have loaded step it's)
 //                dV += P^T(it) dO  (P^T read from tensor memory),
 //                dK += dS^T(it) Q, dQ^T(it) = K^T dS^T(it)
 //              so the softmax of step it+1 overlaps the gradient MMAs of it;
@@ -204,7 +205,8 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* bar_dq = bars + 11;       // dQ^T of a step in TMEM
     uint64_t* bar_dqfree = bars + 12;   // dQ^T read out of TMEM (count 4)
     uint64_t* bar_final = bars + 13;    // all MMAs done
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+    uint64_t* bar_sdp_read = bars + 14; // S^T, dP^T of a step loaded into registers (count 4)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = warp_id(), lane = lane_id();
@@ -229,6 +231,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         mbar_init(bar_sdp, 1);
         mbar_init(bar_ds, 4);
+        mbar_init(bar_sdp_read, 4);
         mbar_init(&bar_gdone[0], 1);
         mbar_init(&bar_gdone[1], 1);
         mbar_init(bar_dq, 1);
@@ -299,7 +302,8 @@ __global__ void __launch_bounds__(384, 1)
         }
       } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // (the whole warp runs this loop; one elected lane issues each MMA)
+        {
             const uint32_t id_sdp = idesc_bf16_f32(128, 64, false, false);   // S^T, dP^T
             const uint32_t id_grad = idesc_bf16_f32(128, D, false, true);    // dV, dK
             const uint32_t id_dq = idesc_bf16_f32(128, 64, true, true);      // dQ^T
@@ -326,37 +330,41 @@ __global__ void __launch_bounds__(384, 1)
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ok_ = (uint32_t)((kk >> 2) * C::kKPanel + (kk & 3) * 32);
                     const uint32_t oq = (uint32_t)((kk >> 2) * C::kQPanel + (kk & 3) * 32);
-                    mma_ss(tSb, dK_k + off(ok_), dSlot_k + off(so + oq), id_sdp, kk > 0 ? 1u : 0u);
+                    mma_ss_w(tSb, dK_k + off(ok_), dSlot_k + off(so + oq), id_sdp, kk > 0 ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ok_ = (uint32_t)((kk >> 2) * C::kKPanel + (kk & 3) * 32);
                     const uint32_t oq = (uint32_t)((kk >> 2) * C::kQPanel + (kk & 3) * 32);
-                    mma_ss(tDP, dV_k + off(ok_), dSlot_k + off(so + C::kQTile + oq), id_sdp, kk > 0 ? 1u : 0u);
+                    mma_ss_w(tDP, dV_k + off(ok_), dSlot_k + off(so + C::kQTile + oq), id_sdp, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(bar_sdp);
+                mma_commit_w(bar_sdp);
             };
 
-            bool ok = mbar_wait(bar_kv, 0, abort_flag);
+            bool ok = mbar_wait_w(bar_kv, 0, abort_flag);
             if (ok && n_it > 0) {
-                ok = mbar_wait(&bar_full[0], 0, abort_flag);
+                ok = mbar_wait_w(&bar_full[0], 0, abort_flag);
                 tc_fence_after();
                 if (ok)
                     issue_sdp(0);
             }
             for (int it = 0; ok && it < n_it; ++it) {
-                if (!(ok = mbar_wait(bar_ds, (uint32_t)(it & 1), abort_flag)))
-                    break;
-                tc_fence_after();
                 if (it + 1 < n_it) {
+                    // step it's S^T / dP^T are in registers: the next step's may overwrite
+                    // dP^T and the other S^T buffer
                     const int in = it + 1;
-                    if (!(ok = mbar_wait(&bar_full[in % C::kSlots], (uint32_t)((in / C::kSlots) & 1), abort_flag)))
+                    if (!(ok = mbar_wait_w(bar_sdp_read, (uint32_t)(it & 1), abort_flag)))
+                        break;
+                    if (!(ok = mbar_wait_w(&bar_full[in % C::kSlots], (uint32_t)((in / C::kSlots) & 1), abort_flag)))
                         break;
                     tc_fence_after();
                     issue_sdp(in);
                 }
+                if (!(ok = mbar_wait_w(bar_ds, (uint32_t)(it & 1), abort_flag)))
+                    break;
+                tc_fence_after();
                 if (it > 0) {
-                    if (!(ok = mbar_wait(bar_dqfree, (uint32_t)((it - 1) & 1), abort_flag)))
+                    if (!(ok = mbar_wait_w(bar_dqfree, (uint32_t)((it - 1) & 1), abort_flag)))
                         break;
                     tc_fence_after();
                 }
@@ -367,18 +375,18 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                    mma_ts(tDV, tP + (uint32_t)(kk * 8), dSlot_mn + off(so + C::kQTile + kk * 2048), id_grad, acc);
-                    mma_ss(tDK, dDS_k + off(dso + kk * 32), dSlot_mn + off(so + kk * 2048), id_grad, acc);
+                    mma_ts_w(tDV, tP + (uint32_t)(kk * 8), dSlot_mn + off(so + C::kQTile + kk * 2048), id_grad, acc);
+                    mma_ss_w(tDK, dDS_k + off(dso + kk * 32), dSlot_mn + off(so + kk * 2048), id_grad, acc);
                 }
                 // dQ^T = K^T dS^T   (K dimension = 128 keys)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tDQ, dK_mn + off(kk * 2048), dDS_mn + off(dso + kk * 2048), id_dq, kk > 0 ? 1u : 0u);
-                mma_commit(bar_dq);
-                mma_commit(&bar_gdone[it & 1]);
-                mma_commit(&bar_empty[it % C::kSlots]);
+                    mma_ss_w(tDQ, dK_mn + off(kk * 2048), dDS_mn + off(dso + kk * 2048), id_dq, kk > 0 ? 1u : 0u);
+                mma_commit_w(bar_dq);
+                mma_commit_w(&bar_gdone[it & 1]);
+                mma_commit_w(&bar_empty[it % C::kSlots]);
             }
-            mma_commit(bar_final);
+            mma_commit_w(bar_final);
             if (!ok)
                 mbar_wait_limited(bar_final, 0, FA_WAIT_LIMIT_CYCLES);
         }
@@ -407,6 +415,10 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t tSb = tS + (uint32_t)(64 * (it & 1));
             uint32_t sr[64], dr[64];
             tmem_ld64x2(tSb, tDP, sr, dr);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar_sdp_read);
             // query rows qb*64 + c see this key iff key < Nk and (causal) key <= row + Nk - Nq
             const int q_first = qb * 64;
             const int min_row = CAUSAL ? key - delta_q : INT_MIN;   // rows >= min_row see the key
@@ -425,9 +437,11 @@ __global__ void __launch_bounds__(384, 1)
                     pv.y = (key_ok && q_first + c + 1 >= min_row) ? pv.y : 0.f;
                 }
                 // dS = P * (dP - D)
-                const float2 dd2 = make_float2(__uint_as_float(dr[c]) - dlt[c], __uint_as_float(dr[c + 1]) - dlt[c + 1]);
+                const float2 dd2 = fadd2(make_float2(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])),
+                                         make_float2(-dlt[c], -dlt[c + 1]));
+                const float2 ds2 = fmul2(pv, dd2);
                 pp[c >> 1] = pack_bf16x2(pv.x, pv.y);
-                dd[c >> 1] = pack_bf16x2(pv.x * dd2.x, pv.y * dd2.y);
+                dd[c >> 1] = pack_bf16x2(ds2.x, ds2.y);
             }
             // P^T over this step's S^T columns (the dV MMA reads it from there)
             tmem_st32(tSb, pp);

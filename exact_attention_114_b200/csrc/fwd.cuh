@@ -28,6 +28,8 @@
 // same answer once numerator and denominator are rescaled together).
 #pragma once
 
+#include <type_traits>
+
 #include "sm100.cuh"
 #include "fa_kernels.h"
 
@@ -43,7 +45,7 @@ struct FwdCfg {
     static constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 80;
     static constexpr int kTileBytes = 128 * D * 2;   // a 128-row Q, K or V tile
     static constexpr int kPanelBytes = 128 * 128;    // 128 rows x 64 bf16
-    static constexpr int kStages = (D == 128) ? 4 : 8;
+    static constexpr int kStages = (D == 128) ? 5 : 8;
     static constexpr int kOffQ = 0;
     static constexpr int kOffKV = 2 * kTileBytes;
     static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
@@ -180,7 +182,8 @@ __global__ void __launch_bounds__(384, 1)
         }
       } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // (the whole warp runs this loop; one elected lane issues each MMA)
+        {
             const uint32_t idS = idesc_bf16_f32(128, 128, false, false);
             const uint32_t idPV = idesc_bf16_f32(128, D, false, true);
             const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
@@ -189,7 +192,7 @@ __global__ void __launch_bounds__(384, 1)
             bool ok = true;
             for (int t = 0; t < 2 && ok; ++t)
                 if (nblk[t] > 0)
-                    ok = mbar_wait(&bar_q[t], 0, abort_flag);
+                    ok = mbar_wait_w(&bar_q[t], 0, abort_flag);
             tc_fence_after();
 
             // base descriptors; a byte offset `o` inside an operand is added as o >> 4
@@ -206,9 +209,9 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t o = (uint32_t)((kk >> 2) * C::kPanelBytes + (kk & 3) * 32);
-                    mma_ss(tS[t], dQ_k + off(qo + o), dKV_k + off(ko + o), idS, kk > 0 ? 1u : 0u);
+                    mma_ss_w(tS[t], dQ_k + off(qo + o), dKV_k + off(ko + o), idS, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(&bar_s[t]);
+                mma_commit_w(&bar_s[t]);
             };
             // keys 64*half .. 64*half+63 of block j (P columns 32*half .. 32*half+31)
             auto issue_PV = [&](int t, int j, int half) {
@@ -216,31 +219,31 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                 for (int k4 = 0; k4 < 4; ++k4) {
                     const int kk = 4 * half + k4;
-                    mma_ts(tO[t], tS[t] + (uint32_t)(kk * 8), dKV_mn + off(vo + (uint32_t)(kk * 2048)), idPV,
+                    mma_ts_w(tO[t], tS[t] + (uint32_t)(kk * 8), dKV_mn + off(vo + (uint32_t)(kk * 2048)), idPV,
                            (j > 0 || kk > 0) ? 1u : 0u);
                 }
             };
 
             if (ok && n_iter > 0) {
-                ok = mbar_wait(&bar_full[0], 0, abort_flag);
+                ok = mbar_wait_w(&bar_full[0], 0, abort_flag);
                 tc_fence_after();
                 if (ok) {
                     for (int t = 0; t < 2; ++t)
                         if (nblk[t] > 0)
                             issue_S(t, 0);
-                    mma_commit(&bar_empty[0]);
+                    mma_commit_w(&bar_empty[0]);
                 }
             }
             for (int j = 0; ok && j < n_iter; ++j) {
                 const int iv = 2 * j + 1, ik = 2 * j + 2;
-                if (!(ok = mbar_wait(&bar_full[iv % C::kStages], phase(iv), abort_flag)))
+                if (!(ok = mbar_wait_w(&bar_full[iv % C::kStages], phase(iv), abort_flag)))
                     break;
                 tc_fence_after();
                 bool k_ready = false;
                 for (int t = 0; t < 2 && ok; ++t) {
                     if (j < nblk[t]) {
                         for (int hf = 0; hf < 2 && ok; ++hf) {
-                            if (!(ok = mbar_wait(&bar_p[2 * t + hf], (uint32_t)(j & 1), abort_flag)))
+                            if (!(ok = mbar_wait_w(&bar_p[2 * t + hf], (uint32_t)(j & 1), abort_flag)))
                                 break;
                             tc_fence_after();
                             issue_PV(t, j, hf);
@@ -248,11 +251,11 @@ __global__ void __launch_bounds__(384, 1)
                         if (!ok)
                             break;
                         if (j == nblk[t] - 1)
-                            mma_commit(&bar_o[t]);
+                            mma_commit_w(&bar_o[t]);
                     }
                     if (j + 1 < nblk[t]) {
                         if (!k_ready) {
-                            if (!(ok = mbar_wait(&bar_full[ik % C::kStages], phase(ik), abort_flag)))
+                            if (!(ok = mbar_wait_w(&bar_full[ik % C::kStages], phase(ik), abort_flag)))
                                 break;
                             tc_fence_after();
                             k_ready = true;
@@ -262,12 +265,12 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 if (!ok)
                     break;
-                mma_commit(&bar_empty[iv % C::kStages]);
+                mma_commit_w(&bar_empty[iv % C::kStages]);
                 if (k_ready)
-                    mma_commit(&bar_empty[ik % C::kStages]);
+                    mma_commit_w(&bar_empty[ik % C::kStages]);
             }
             if (!ok) {
-                mma_commit(bar_drain);
+                mma_commit_w(bar_drain);
                 mbar_wait_limited(bar_drain, 0, FA_WAIT_LIMIT_CYCLES);
             }
         }
@@ -339,16 +342,22 @@ __global__ void __launch_bounds__(384, 1)
             const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
             const float2 sl22 = make_float2(sl2, sl2), nm2 = make_float2(neg_m, neg_m);
             float2 acc = make_float2(0.f, 0.f);
-            // P in two halves of 64 keys: the MMA warp starts P.V on the first
-            // half while the second is still being exponentiated
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
+            // One exp2 per score: the MUFU unit would be as busy as the tensor
+            // core at d = 128, so in blocks without masked scores one pair in
+            // four goes to the FMA-pipe exp2 instead (masked -inf scores always
+            // take ex2.approx, which returns exactly 0 for them).
+            const bool soft = !__any_sync(0xffffffffu, need_mask);
+            auto half_block = [&](int hf, auto use_poly) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
                     const int e = 64 * hf + 2 * c;
                     const float2 x = ffma2(make_float2(s[e], s[e + 1]), sl22, nm2);
-                    const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                    float2 pv;
+                    if (decltype(use_poly)::value && (c & 3) == 3)
+                        pv = exp2_poly2(x);
+                    else
+                        pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                     acc = fadd2(acc, pv);
                     pk[c] = pack_bf16x2(pv.x, pv.y);
                 }
@@ -358,6 +367,15 @@ __global__ void __launch_bounds__(384, 1)
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&bar_p[2 * t + hf]);
+            };
+            // P in two halves of 64 keys: the MMA warp starts P.V on the first
+            // half while the second is still being exponentiated
+            if (soft) {
+                half_block(0, std::true_type{});
+                half_block(1, std::true_type{});
+            } else {
+                half_block(0, std::false_type{});
+                half_block(1, std::false_type{});
             }
             l += acc.x + acc.y;
         }

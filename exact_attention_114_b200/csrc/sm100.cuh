@@ -200,6 +200,48 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar)
         : "memory");
 }
 
+// Warp-wide forms: the whole warp executes the call (so the surrounding control
+// flow and the descriptors stay warp-uniform) and one elected lane issues.
+__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b32 l;\n\t"
+        "elect.sync l|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b32 l;\n\t"
+        "elect.sync l|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit_w(uint64_t* bar)
+{
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t.reg .b32 l;\n\t"
+        "elect.sync l|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+// Bounded wait executed by a whole warp; the result is the same on every lane.
+__device__ __forceinline__ bool mbar_wait_w(uint64_t* bar, uint32_t parity, volatile int* abort_flag)
+{
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+}
+
 // Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B.
 //   bits [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format,
 //   bit 15 A major (0 = K), bit 16 B major (0 = K, 1 = MN), [17,23) N >> 3,
@@ -350,6 +392,19 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b)
     asm("{\n\t.reg .b64 ra, rb;\n\t"
         "mov.b64 ra, {%1, %2};\n\tmov.b64 rb, {%3, %4};\n\t"
         "add.f32x2 %0, ra, rb;\n\t}"
+        : "=l"(r)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    float2 o;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(o.x), "=f"(o.y) : "l"(r));
+    return o;
+}
+
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b)
+{
+    uint64_t r;
+    asm("{\n\t.reg .b64 ra, rb;\n\t"
+        "mov.b64 ra, {%1, %2};\n\tmov.b64 rb, {%3, %4};\n\t"
+        "mul.f32x2 %0, ra, rb;\n\t}"
         : "=l"(r)
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     float2 o;
