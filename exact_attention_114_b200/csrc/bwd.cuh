@@ -198,11 +198,11 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* bar_kv = bars;            // K, V landed
     uint64_t* bar_full = bars + 1;      // [kSlots] step slot landed
-    uint64_t* bar_empty = bars + 4;     // [kSlots] step slot released
     uint64_t* bar_sdp = bars + 7;       // S^T and dP^T of a step in TMEM
     uint64_t* bar_ds = bars + 8;        // P^T (TMEM), dS^T (smem) of a step written (count 4)
-    uint64_t* bar_gdone = bars + 9;     // [2] gradient MMAs of a step done (its dS^T buffer free)
-    uint64_t* bar_dq = bars + 11;       // dQ^T of a step in TMEM
+    // [2] gradient MMAs of step `it` done (bar_gdone[it & 1]): dQ^T(it) is in TMEM,
+    // dS^T buffer (it & 1) and step slot (it % kSlots) are free again
+    uint64_t* bar_gdone = bars + 9;
     uint64_t* bar_dqfree = bars + 12;   // dQ^T read out of TMEM (count 4)
     uint64_t* bar_final = bars + 13;    // all MMAs done
     uint64_t* bar_sdp_read = bars + 14; // S^T, dP^T of a step loaded into registers (count 4)
@@ -225,16 +225,13 @@ __global__ void __launch_bounds__(384, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(bar_kv, 1);
-        for (int s = 0; s < C::kSlots; ++s) {
+        for (int s = 0; s < C::kSlots; ++s)
             mbar_init(&bar_full[s], 1);
-            mbar_init(&bar_empty[s], 1);
-        }
         mbar_init(bar_sdp, 1);
         mbar_init(bar_ds, 4);
         mbar_init(bar_sdp_read, 4);
         mbar_init(&bar_gdone[0], 1);
         mbar_init(&bar_gdone[1], 1);
-        mbar_init(bar_dq, 1);
         mbar_init(bar_dqfree, 4);
         mbar_init(bar_final, 1);
         *abort_flag = 0;
@@ -277,8 +274,12 @@ __global__ void __launch_bounds__(384, 1)
             int issued = 0;
             for (int it = 0; it < n_it; ++it) {
                 const int s = it % C::kSlots;
-                if (!mbar_wait(&bar_empty[s], (uint32_t)((it / C::kSlots) & 1) ^ 1u, abort_flag))
-                    break;
+                // the slot was last used by step it - kSlots: wait for its gradient MMAs
+                if (it >= C::kSlots) {
+                    const int prev = it - C::kSlots;
+                    if (!mbar_wait(&bar_gdone[prev & 1], (uint32_t)((prev >> 1) & 1), abort_flag))
+                        break;
+                }
                 int h, qb;
                 step_coords(it, h, qb);
                 const int bh = b * p.Hq + h;
@@ -344,7 +345,6 @@ __global__ void __launch_bounds__(384, 1)
             bool ok = mbar_wait_w(bar_kv, 0, abort_flag);
             if (ok && n_it > 0) {
                 ok = mbar_wait_w(&bar_full[0], 0, abort_flag);
-                tc_fence_after();
                 if (ok)
                     issue_sdp(0);
             }
@@ -357,7 +357,6 @@ __global__ void __launch_bounds__(384, 1)
                         break;
                     if (!(ok = mbar_wait_w(&bar_full[in % C::kSlots], (uint32_t)((in / C::kSlots) & 1), abort_flag)))
                         break;
-                    tc_fence_after();
                     issue_sdp(in);
                 }
                 if (!(ok = mbar_wait_w(bar_ds, (uint32_t)(it & 1), abort_flag)))
@@ -382,9 +381,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ss_w(tDQ, dK_mn + off(kk * 2048), dDS_mn + off(dso + kk * 2048), id_dq, kk > 0 ? 1u : 0u);
-                mma_commit_w(bar_dq);
                 mma_commit_w(&bar_gdone[it & 1]);
-                mma_commit_w(&bar_empty[it % C::kSlots]);
             }
             mma_commit_w(bar_final);
             if (!ok)
@@ -513,7 +510,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int it = 0; it < n_it; ++it) {
             int h, qb;
             step_coords(it, h, qb);
-            ok = mbar_wait(bar_dq, (uint32_t)(it & 1), abort_flag);
+            ok = mbar_wait(&bar_gdone[it & 1], (uint32_t)((it >> 1) & 1), abort_flag);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok)
                 break;

@@ -237,8 +237,12 @@ __device__ __forceinline__ void mma_commit_w(uint64_t* bar)
 }
 
 // Bounded wait executed by a whole warp; the result is the same on every lane.
+// The common case (phase already complete) costs one try_wait; the warp vote
+// is only taken on the slow path.
 __device__ __forceinline__ bool mbar_wait_w(uint64_t* bar, uint32_t parity, volatile int* abort_flag)
 {
+    if (__all_sync(0xffffffffu, mbar_try_wait(smem_u32(bar), parity)))
+        return true;
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
 }
 
