@@ -165,7 +165,7 @@ def time_oracle_step(w):
     return time.perf_counter() - t0
 
 
-def cpu_baseline_leg(reps=3):
+def cpu_baseline_leg(reps=10):
     w = oracle_sample_workload()
     dt = sum(time_oracle_step(w) for _ in range(reps)) / reps
     flops = w.fwd_flops() + w.bwd_flops()
