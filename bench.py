@@ -323,6 +323,34 @@ def run_libfa(args, rank, world, local):
     dec_gbs = dec_bytes / (dec_ms * 1e-3) / 1e9
     fa.fa_check_device_status()
 
+    # ---- the same decode over a paged KV cache: 64-key pages handed out in a
+    # seeded random order (same bytes, one block-table lookup per tile)
+    ps = 64
+    pages = wd.Nk // ps
+    gen = torch.Generator().manual_seed(wd.seed)
+    perm = torch.randperm(wd.B * pages, generator=gen).to(dev)
+    pool_k = torch.empty((wd.B * pages, ps, wd.Hkv, wd.d), dtype=torch.bfloat16, device=dev)
+    pool_v = torch.empty_like(pool_k)
+    pool_k[perm] = dxd["k"].permute(0, 2, 1, 3).reshape(wd.B * pages, ps, wd.Hkv, wd.d)
+    pool_v[perm] = dxd["v"].permute(0, 2, 1, 3).reshape(wd.B * pages, ps, wd.Hkv, wd.d)
+    table = perm.to(torch.int32).reshape(wd.B, pages).contiguous()
+    lens = torch.full((wd.B,), wd.Nk, dtype=torch.int32, device=dev)
+    del dxd["k"], dxd["v"]
+    torch.cuda.empty_cache()
+    pws = torch.empty(max(1, fa.fa_fwd_paged_workspace_size(wd.B, wd.Hq, wd.Hkv, 1, ps, pages, wd.d)),
+                      dtype=torch.uint8, device=dev)
+
+    def dec_paged():
+        fa.fa_fwd_paged(dxd["q"], pool_k, pool_v, table, lens, od, lsed, scale=wd.scale,
+                        workspace=pws)
+
+    for _ in range(3):
+        dec_paged()
+    torch.cuda.synchronize()
+    pag_ms = statistics.median(timed(dec_paged, max(10, args.steps)))
+    pag_gbs = dec_bytes / (pag_ms * 1e-3) / 1e9
+    fa.fa_check_device_status()
+
     clocks = clk.summary()
     line = {
         "metric": "attention fwd+bwd TFLOP/s (causal GQA, N=8192, d=128)",
@@ -339,6 +367,9 @@ def run_libfa(args, rank, world, local):
             "decode": {"workload": f"{DECODE_WORKLOAD}: B=64, Hq=32, Hkv=8, Nq=1, Nk=8192, d=128",
                        "ms": dec_ms, "gbs": dec_gbs, "frac_of_hbm": dec_gbs / peaks["hbm_gbs"],
                        "algorithmic_bytes": dec_bytes},
+            "decode_paged": {"workload": f"{DECODE_WORKLOAD} over 64-key pages in random order",
+                             "ms": pag_ms, "gbs": pag_gbs, "frac_of_hbm": pag_gbs / peaks["hbm_gbs"],
+                             "algorithmic_bytes": dec_bytes},
         },
         "roofline": {"kernel": "fa_bwd (bwd_main dominant; pre/post included in the time)",
                      "bound": "tensor", "achieved": bwd_tf,
@@ -347,7 +378,7 @@ def run_libfa(args, rank, world, local):
                      "peak_source": peaks["source"] + " (sustained bf16 cuBLAS)"},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": args.steps * 4,
+        "gpu_launches": args.steps * 4,  # timed region: fwd (1) + bwd (pre, main, post) per step
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -63,6 +63,11 @@ def lib() -> ctypes.CDLL:
             L.fa_fwd_splitkv_noalloc.argtypes = [vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, fl, ip,
                                                   ip, vp]
             L.fa_fwd_splitkv_noalloc.restype = ip
+            L.fa_fwd_paged_workspace_size.argtypes = [ip, ip, ip, ip, ip, ip, ip, ip]
+            L.fa_fwd_paged_workspace_size.restype = sz
+            L.fa_fwd_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, ip, ip, fl,
+                                       ip, ip, vp, sz, vp]
+            L.fa_fwd_paged.restype = ip
             L.fa_bwd_workspace_size.argtypes = [ip, ip, ip, ip, ip, ip]
             L.fa_bwd_workspace_size.restype = sz
             L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, fl, ip,
@@ -155,6 +160,37 @@ def fa_fwd_splitkv(q, k, v, o=None, lse=None, *, causal=False, scale=None, num_s
     _check(lib().fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq,
                                 Nk, d, scale, int(bool(causal)), int(num_splits), _ptr(workspace),
                                 ws_bytes, _stream(stream)))
+    return o, lse
+
+
+def fa_fwd_paged_workspace_size(B, Hq, Hkv, Nq, page_size, max_pages_per_seq, d, num_splits=0) -> int:
+    return int(lib().fa_fwd_paged_workspace_size(B, Hq, Hkv, Nq, page_size, max_pages_per_seq, d,
+                                                 num_splits))
+
+
+def fa_fwd_paged(q, k_cache, v_cache, block_table, seq_lens, o=None, lse=None, *, causal=False,
+                 scale=None, num_splits=0, workspace=None, stream=None):
+    """Decode over a paged KV cache.  k_cache/v_cache [num_pages, page_size, Hkv, d] bf16,
+    block_table int32 [B, max_pages_per_seq], seq_lens int32 [B], q [B, Hq, Nq, d]."""
+    import torch
+    B, Hq, Nq, d = q.shape
+    num_pages, page_size, Hkv, dk = k_cache.shape
+    if dk != d or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("k_cache / v_cache shapes disagree with q")
+    for t, n in ((block_table, "block_table"), (seq_lens, "seq_lens")):
+        if not t.is_cuda or t.dtype != torch.int32 or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous CUDA int32 tensor")
+    max_pages = block_table.shape[1]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().fa_fwd_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                              _ptr(seq_lens), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, d, page_size,
+                              num_pages, max_pages, scale, int(bool(causal)), int(num_splits),
+                              _ptr(workspace), ws_bytes, _stream(stream)))
     return o, lse
 
 

@@ -16,6 +16,12 @@
 //     final output when there is a single chunk.
 // Combine: lse = ln sum_s exp(lse_s), O = sum_s exp(lse_s - lse) O_s (§04 rule in
 // log form), one warp per output row.
+//
+// Paged variant (PAGED = true): the KV cache is a pool of pages, [num_pages,
+// page_size, Hkv, d], shared by all sequences (the pages are only "where the KV
+// is stored", §09); a block table maps each sequence's logical pages to
+// physical ones and every sequence has its own length.  Only the producer
+// changes: it looks up the page of each 64-key tile and issues a 4-D TMA load.
 #pragma once
 
 #include "sm100.cuh"
@@ -67,6 +73,7 @@ __device__ __forceinline__ uint32_t dec_tile_off(int key, int chunk)
     return (uint32_t)(panel * DecCfg::kPanelBytes + key * 128 + ((c ^ (key & 7)) << 4));
 }
 
+template <bool PAGED>
 __global__ void __launch_bounds__(160)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         DecodeParams p)
@@ -83,8 +90,10 @@ __global__ void __launch_bounds__(160)
     const int split = (int)blockIdx.x % p.splits;
     const int kvh = (int)blockIdx.x / p.splits;     // b * Hkv + kv head
     const int b = kvh / p.Hkv, hk = kvh % p.Hkv;
+    // keys of this sequence (a paged sequence's own length, clamped to what its table can hold)
+    const int Nk_b = PAGED ? max(0, min(__ldg(p.seq_lens + b), p.max_pages * p.page_size)) : p.Nk;
     const int k_begin = split * p.chunk;
-    const int k_end = min(p.Nk, k_begin + p.chunk);
+    const int k_end = min(Nk_b, k_begin + p.chunk);
     const int n_tiles = k_end > k_begin ? (k_end - k_begin + C::kKeys - 1) / C::kKeys : 0;
 
     if (threadIdx.x == 0) {
@@ -110,10 +119,21 @@ __global__ void __launch_bounds__(160)
                 uint8_t* dv = dk + C::kTileBytes;
                 mbar_arrive_expect_tx(&bar_full[slot], 2 * C::kTileBytes);
                 const int key0 = k_begin + t * C::kKeys;
-                tma_load_3d(dk, &tmK, &bar_full[slot], 0, key0, kvh);
-                tma_load_3d(dk + C::kPanelBytes, &tmK, &bar_full[slot], 64, key0, kvh);
-                tma_load_3d(dv, &tmV, &bar_full[slot], 0, key0, kvh);
-                tma_load_3d(dv + C::kPanelBytes, &tmV, &bar_full[slot], 64, key0, kvh);
+                if (PAGED) {
+                    // a 64-key tile never straddles a page (page_size is a multiple of 64);
+                    // an out-of-range page id reads zeros (TMA bounds), never another buffer
+                    const int page = __ldg(p.block_table + (size_t)b * p.max_pages + key0 / p.page_size);
+                    const int off = key0 % p.page_size;
+                    tma_load_4d(dk, &tmK, &bar_full[slot], 0, hk, off, page);
+                    tma_load_4d(dk + C::kPanelBytes, &tmK, &bar_full[slot], 64, hk, off, page);
+                    tma_load_4d(dv, &tmV, &bar_full[slot], 0, hk, off, page);
+                    tma_load_4d(dv + C::kPanelBytes, &tmV, &bar_full[slot], 64, hk, off, page);
+                } else {
+                    tma_load_3d(dk, &tmK, &bar_full[slot], 0, key0, kvh);
+                    tma_load_3d(dk + C::kPanelBytes, &tmK, &bar_full[slot], 64, key0, kvh);
+                    tma_load_3d(dv, &tmV, &bar_full[slot], 0, key0, kvh);
+                    tma_load_3d(dv + C::kPanelBytes, &tmV, &bar_full[slot], 64, key0, kvh);
+                }
             }
             if (*abort_flag) {
                 const int last = n_tiles;
@@ -152,7 +172,7 @@ __global__ void __launch_bounds__(160)
     for (int hr = 0; hr < 2; ++hr) {
         const int r = g + 8 * hr;
         const int i = (r < p.R) ? r % p.Nq : 0;
-        lim[hr] = p.causal ? min(k_end - 1, i + p.Nk - p.Nq) : k_end - 1;
+        lim[hr] = p.causal ? min(k_end - 1, i + Nk_b - p.Nq) : k_end - 1;
     }
 
     float o[16][4];

@@ -142,6 +142,30 @@ fa_status_t make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t 
     return FA_OK;
 }
 
+// 4-D map over a paged KV pool [pages][page_size][Hkv][d] (bf16), box {64, 1, 64, 1}
+// (one kv head, 64 keys of one page), 128-byte swizzle.
+fa_status_t make_map_paged(CUtensorMap* m, const void* base, uint64_t d, uint64_t Hkv, uint64_t page_size,
+                           uint64_t pages)
+{
+    EncodeTiledFn enc = get_encode();
+    if (!enc) {
+        set_error("cuTensorMapEncodeTiled is unavailable");
+        return FA_ERR_CUDA;
+    }
+    cuuint64_t dims[4] = {d, Hkv, page_size, pages};
+    cuuint64_t strides[3] = {d * 2, Hkv * d * 2, page_size * Hkv * d * 2};
+    cuuint32_t box[4] = {64, 1, 64, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("cuTensorMapEncodeTiled (paged) failed (%d)", (int)r);
+        return FA_ERR_CUDA;
+    }
+    return FA_OK;
+}
+
 // Raise a kernel's dynamic shared memory limit once per (kernel, device).
 fa_status_t ensure_smem(const void* kernel, int bytes)
 {
@@ -278,16 +302,28 @@ DecodePlan decode_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, int reques
     return pl;
 }
 
+struct PagedDesc {
+    const int* block_table;
+    const int* seq_lens;
+    int page_size, num_pages, max_pages;
+};
+
 fa_status_t launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                           int Nq, int Nk, int d, float scale, int causal, const DecodePlan& pl, void* ws,
-                          cudaStream_t stream)
+                          cudaStream_t stream, const PagedDesc* pg = nullptr)
 {
     using C = fa::DecCfg;
     CUtensorMap mk, mv;
     fa_status_t st;
-    if ((st = make_map(&mk, k, d, Nk, (uint64_t)B * Hkv, 64)) != FA_OK) return st;
-    if ((st = make_map(&mv, v, d, Nk, (uint64_t)B * Hkv, 64)) != FA_OK) return st;
-    if ((st = ensure_smem(reinterpret_cast<const void*>(fa::decode_split_kernel), C::kSmemBytes)) != FA_OK) return st;
+    if (pg) {
+        if ((st = make_map_paged(&mk, k, d, Hkv, pg->page_size, pg->num_pages)) != FA_OK) return st;
+        if ((st = make_map_paged(&mv, v, d, Hkv, pg->page_size, pg->num_pages)) != FA_OK) return st;
+    } else {
+        if ((st = make_map(&mk, k, d, Nk, (uint64_t)B * Hkv, 64)) != FA_OK) return st;
+        if ((st = make_map(&mv, v, d, Nk, (uint64_t)B * Hkv, 64)) != FA_OK) return st;
+    }
+    auto kern = pg ? fa::decode_split_kernel<true> : fa::decode_split_kernel<false>;
+    if ((st = ensure_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes)) != FA_OK) return st;
     fa::DecodeParams p;
     p.q = static_cast<const __nv_bfloat16*>(q);
     p.k = static_cast<const __nv_bfloat16*>(k);
@@ -307,8 +343,12 @@ fa_status_t launch_decode(const void* q, const void* k, const void* v, void* o, 
     p.chunk = pl.chunk;
     p.causal = causal;
     p.scale_log2 = scale * kLog2e;
+    p.block_table = pg ? pg->block_table : nullptr;
+    p.seq_lens = pg ? pg->seq_lens : nullptr;
+    p.page_size = pg ? pg->page_size : 0;
+    p.max_pages = pg ? pg->max_pages : 0;
     const long long grid = (long long)B * Hkv * pl.splits;
-    fa::decode_split_kernel<<<(unsigned)grid, C::kThreads, C::kSmemBytes, stream>>>(mk, mv, p);
+    kern<<<(unsigned)grid, C::kThreads, C::kSmemBytes, stream>>>(mk, mv, p);
     if ((st = check_launch("decode_split_kernel launch")) != FA_OK) return st;
     if (pl.splits > 1) {
         const long long rows = (long long)B * Hkv * p.R;
@@ -568,6 +608,79 @@ fa_status_t fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, 
     // call, so nothing in the scratch has to be cleared first
     return launch_decode(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, pl, ws,
                          static_cast<cudaStream_t>(stream));
+}
+
+size_t fa_fwd_paged_workspace_size(int B, int Hq, int Hkv, int Nq, int page_size, int max_pages_per_seq, int d,
+                                   int num_splits)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Hq % Hkv != 0 || d < 1 || num_splits < 0 || page_size < 1 ||
+        max_pages_per_seq < 1 || (long long)page_size * max_pages_per_seq > (1ll << 30))
+        return 0;
+    return decode_plan(B, Hq, Hkv, Nq, page_size * max_pages_per_seq, d, num_splits).total();
+}
+
+fa_status_t fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                         const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int d,
+                         int page_size, int num_pages, int max_pages_per_seq, float scale, int causal,
+                         int num_splits, void* workspace, size_t workspace_bytes, void* stream)
+{
+    t_error.clear();
+    fa_status_t st;
+    if ((st = check_ptr(q, "q")) || (st = check_ptr(k_cache, "k_cache")) || (st = check_ptr(v_cache, "v_cache")) ||
+        (st = check_ptr(o, "o")))
+        return st;
+    if (!block_table || !seq_lens || (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+        (reinterpret_cast<uintptr_t>(seq_lens) & 3u)) {
+        set_error("block_table and seq_lens must be non-NULL and 4-byte aligned");
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) {
+        set_error("lse is not 4-byte aligned");
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    if (page_size < 64 || page_size % 64 != 0 || num_pages < 1 || max_pages_per_seq < 1 ||
+        (long long)page_size * max_pages_per_seq > (1ll << 30) || (long long)num_pages * page_size > (1ll << 31)) {
+        set_error("page_size must be a positive multiple of 64; num_pages, max_pages_per_seq >= 1");
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    const int max_len = page_size * max_pages_per_seq;
+    if ((st = check_shape(B, Hq, Hkv, Nq, max_len, d, scale, causal)) != FA_OK)
+        return st;
+    if (num_splits < 0 || num_splits > 256) {
+        set_error("num_splits=%d must be in [0, 256]", num_splits);
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    if (!decode_shape(Hq, Hkv, Nq, d)) {
+        set_error("paged decode needs d = 128 and Nq * Hq / Hkv <= %d", kDecodeMaxRows);
+        return FA_ERR_UNSUPPORTED;
+    }
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) {
+        set_error("workspace is not 256-byte aligned");
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const DecodePlan pl = decode_plan(B, Hq, Hkv, Nq, max_len, d, num_splits);
+    void* ws = workspace;
+    bool owned = false;
+    if (pl.total() > 0) {
+        if (ws == nullptr) {
+            cudaError_t e = cudaMallocAsync(&ws, pl.total(), s);
+            if (e != cudaSuccess)
+                return cuda_fail(e, "cudaMallocAsync (paged split-KV partials)");
+            owned = true;
+        } else if (workspace_bytes < pl.total()) {
+            set_error("workspace has %zu bytes, %zu needed", workspace_bytes, pl.total());
+            return FA_ERR_WORKSPACE;
+        }
+    }
+    PagedDesc pg{block_table, seq_lens, page_size, num_pages, max_pages_per_seq};
+    st = launch_decode(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Nq, max_len, d, scale, causal, pl, ws, s, &pg);
+    if (owned) {
+        cudaError_t e = cudaFreeAsync(ws, s);
+        if (e != cudaSuccess && st == FA_OK)
+            st = cuda_fail(e, "cudaFreeAsync");
+    }
+    return st;
 }
 
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d)

@@ -31,6 +31,13 @@ struct DecodeParams {
     int chunk;               // keys per chunk (multiple of the key tile)
     int causal;
     float scale_log2;
+    // paged KV cache (decode_split_kernel<true>): K/V are [num_pages, page_size, Hkv, d];
+    // the keys of sequence b are block_table[b][key / page_size] * page_size + key % page_size,
+    // and sequence b has seq_lens[b] keys (Nk is then the longest allowed length)
+    const int* block_table;  // [B, max_pages]
+    const int* seq_lens;     // [B]
+    int page_size;
+    int max_pages;
 };
 
 struct BwdParams {

@@ -101,6 +101,31 @@ fa_status_t fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o,
                            void* stream);
 
 /*
+ * Decode over a paged KV cache (§09: paged KV management "orthogonal" to the
+ * attention computation -- it only decides where K and V are stored).
+ *   k_cache, v_cache: [num_pages, page_size, Hkv, d] bf16, one pool shared by
+ *     all sequences (heads innermost).
+ *   block_table: int32 [B, max_pages_per_seq] (device); logical page n of
+ *     sequence b is physical page block_table[b * max_pages_per_seq + n].
+ *   seq_lens: int32 [B] (device); sequence b has seq_lens[b] keys, at most
+ *     page_size * max_pages_per_seq (values are clamped to that range; a page id
+ *     outside [0, num_pages) reads zeros).
+ *   q, o: [B, Hq, Nq, d] bf16; lse [B, Hq, Nq] fp32 or NULL.  With causal = 1 the
+ *     Nq query rows of sequence b are its last Nq positions (bottom-right mask
+ *     against seq_lens[b]).
+ *   page_size: a multiple of 64.  d = 128, Nq * Hq / Hkv <= 16.
+ *   num_splits / workspace as for fa_fwd_splitkv, sized with
+ *   fa_fwd_paged_workspace_size().
+ */
+size_t fa_fwd_paged_workspace_size(int B, int Hq, int Hkv, int Nq, int page_size, int max_pages_per_seq,
+                                   int d, int num_splits);
+fa_status_t fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache,
+                         const int* block_table, const int* seq_lens, void* o, float* lse,
+                         int B, int Hq, int Hkv, int Nq, int d, int page_size, int num_pages,
+                         int max_pages_per_seq, float scale, int causal, int num_splits,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Split-KV forward that allocates nothing (the paper has no counterpart; this
  * is a deployment variant of fa_fwd_splitkv).
  *

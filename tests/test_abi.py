@@ -126,3 +126,22 @@ def test_no_gpu_reports_cuda_error_without_crashing():
     st = _fwd(B=1, Hq=1, Hkv=1, Nq=128, Nk=128, d=64)
     assert st == fa.FA_ERR_CUDA
     assert fa.last_error_message()
+
+
+def test_paged_rejects_bad_arguments():
+    L = fa.lib()
+
+    def call(page_size=64, num_pages=8, max_pages=4, table=FAKE, lens=FAKE, d=128, Nq=1, splits=0):
+        return L.fa_fwd_paged(FAKE, FAKE, FAKE, table, lens, FAKE, None, 2, 8, 2, Nq, d, page_size,
+                              num_pages, max_pages, 0.1, 0, splits, None, 0, None)
+
+    assert call(table=None) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(lens=ctypes.c_void_p(0x10002)) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(page_size=48) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(page_size=0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(num_pages=0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(max_pages=0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(d=64) == fa.FA_ERR_UNSUPPORTED
+    assert call(Nq=5) == fa.FA_ERR_UNSUPPORTED      # 5 * 4 rows per kv head > 16
+    assert call(splits=300) == fa.FA_ERR_INVALID_ARGUMENT
+    assert fa.fa_fwd_paged_workspace_size(2, 8, 2, 1, 64, 4, 128, 2) > 0
