@@ -74,6 +74,8 @@ def _load(path: str) -> ctypes.CDLL:
     L.oracle_full_row_f32.restype = None
     L.oracle_lse_merge.argtypes = [vp, vp, i64, i64, vp, vp]
     L.oracle_lse_merge.restype = None
+    L.oracle_e4m3_to_f64.argtypes = [vp, i64, vp]
+    L.oracle_e4m3_to_f64.restype = None
     return L
 
 
@@ -272,3 +274,14 @@ def lse_merge(o_parts, lse_parts):
     lse = ctypes.c_double()
     lib().oracle_lse_merge(_ptr(o_parts), _ptr(lse_parts), nparts, d, _ptr(o), ctypes.byref(lse))
     return o, lse.value
+
+
+def e4m3_to_f64(codes) -> np.ndarray:
+    """Values of e4m3 bytes (OCP FP8 E4M3, no infinities; 0x7F / 0xFF are NaN),
+    same shape as ``codes`` (uint8 array or tensor)."""
+    if hasattr(codes, "numpy"):
+        codes = codes.contiguous().view(dtype=__import__("torch").uint8).numpy()
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(c.shape, np.float64)
+    lib().oracle_e4m3_to_f64(_ptr(c), c.size, _ptr(out))
+    return out

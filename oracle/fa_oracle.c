@@ -744,4 +744,31 @@ void oracle_lse_merge(const double* o_parts, const double* lse_parts, int64_t np
     *lse = L;
 }
 
+/*
+ * e4m3 code -> double, from the definition of the OCP 8-bit floating point
+ * format E4M3 (the variant without infinities used for FP8 attention inputs):
+ *   bit 7 sign, bits 6..3 exponent e (bias 7), bits 2..0 mantissa m;
+ *   e = 0:            (-1)^sign * m * 2^-9          (subnormal; m = 0 is zero)
+ *   e = 15, m = 7:    NaN
+ *   otherwise:        (-1)^sign * (1 + m / 8) * 2^(e - 7)
+ * so the largest finite magnitude is 0x7E = 1.75 * 2^8 = 448.
+ */
+void oracle_e4m3_to_f64(const uint8_t* codes, int64_t n, double* out)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        const unsigned c = codes[i];
+        const int sign = (c >> 7) & 1;
+        const int e = (c >> 3) & 15;
+        const int m = c & 7;
+        double mag;
+        if (e == 15 && m == 7)
+            mag = NAN;
+        else if (e == 0)
+            mag = ldexp((double)m, -9);
+        else
+            mag = ldexp(1.0 + m / 8.0, e - 7);
+        out[i] = sign ? -mag : mag;
+    }
+}
+
 int oracle_abi_version(void) { return 1; }

@@ -1,8 +1,8 @@
 """Seeded synthetic workloads for exact attention.
 
-This module only draws inputs: iid N(0,1) samples rounded to bf16 from a
-counter-based SplitMix64 stream (see ``synth.c``), in the shapes of the five
-synthetic workloads below.  It contains no attention arithmetic and is shared
+This module only draws inputs: iid N(0,1) samples rounded to bf16 (or, on
+request, fp16) from a counter-based SplitMix64 stream (see ``synth.c``), in the
+shapes of the synthetic workloads below.  It contains no attention arithmetic and is shared
 by the tests, the benchmark, the smoke check and the oracle checks, so both
 sides of every comparison see identical input bits.
 
@@ -125,16 +125,24 @@ WORKLOADS = {
 }
 
 
-def make_inputs(w: Workload, nthreads: int = 0, pinned: bool = False, dout: bool = True):
-    """Return dict(q, k, v[, dout]) of CPU ``torch.bfloat16`` tensors for ``w``.
+def make_inputs(w: Workload, nthreads: int = 0, pinned: bool = False, dout: bool = True,
+                dtype=None):
+    """Return dict(q, k, v[, dout]) of CPU 16-bit tensors for ``w``: bf16 by
+    default, or fp16 with ``dtype=torch.float16`` (the same fp32 samples rounded
+    to nearest even in the other format).
 
     Shapes: q/dout [B, Hq, Nq, d], k/v [B, Hkv, Nk, d].  With
     ``w.scaled_q_rows`` query rows i % 64 == 0 of every head are multiplied by 8
-    (exact in bf16)."""
+    (exact in either format)."""
     import torch
+    dtype = torch.bfloat16 if dtype is None else dtype
 
     def draw(tid, shape):
         n = int(np.prod(shape))
+        if dtype == torch.float16:
+            f = normal_f32(w.seed, tid, n, nthreads).astype(np.float16)   # IEEE round to nearest even
+            t = torch.from_numpy(f).reshape(shape)
+            return t.pin_memory() if pinned else t
         t = torch.empty(shape, dtype=torch.bfloat16, pin_memory=pinned)
         bits = t.view(torch.int16).numpy().view(np.uint16).reshape(-1)
         normal_bf16_bits(w.seed, tid, n, nthreads, out=bits)
@@ -148,3 +156,28 @@ def make_inputs(w: Workload, nthreads: int = 0, pinned: bool = False, dout: bool
     if dout and w.backward:
         out["dout"] = draw(TENSOR_DO, (w.B, w.Hq, w.Nq, w.d))
     return out
+
+
+# Per-tensor descale factors of the e4m3 inputs (value = code * descale).  Not
+# powers of two, so a descale applied to the wrong tensor changes the result.
+FP8_DESCALE = {"q": 0.0173, "k": 0.0191, "v": 0.0137}
+E4M3_MAX = 448.0
+
+
+def make_inputs_fp8(w: Workload, nthreads: int = 0, pinned: bool = False):
+    """Return dict(q, k, v) of CPU uint8 tensors of e4m3 codes for ``w``: the
+    same N(0,1) fp32 samples as ``make_inputs`` divided by FP8_DESCALE[name],
+    clamped to +-448 and rounded to nearest even e4m3 (torch's float8_e4m3fn
+    cast).  The dequantised inputs are code * FP8_DESCALE[name]."""
+    import torch
+
+    def draw(tid, shape, descale):
+        n = int(np.prod(shape))
+        f = torch.from_numpy(normal_f32(w.seed, tid, n, nthreads)).div_(descale)
+        f.clamp_(-E4M3_MAX, E4M3_MAX)
+        t = f.to(torch.float8_e4m3fn).view(torch.uint8).reshape(shape)
+        return t.pin_memory() if pinned else t
+
+    return dict(q=draw(TENSOR_Q, (w.B, w.Hq, w.Nq, w.d), FP8_DESCALE["q"]),
+                k=draw(TENSOR_K, (w.B, w.Hkv, w.Nk, w.d), FP8_DESCALE["k"]),
+                v=draw(TENSOR_V, (w.B, w.Hkv, w.Nk, w.d), FP8_DESCALE["v"]))

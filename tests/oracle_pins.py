@@ -378,6 +378,38 @@ def pin_bf16_input_path():
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
 
 
+# Values fixed by the definition of OCP FP8 E4M3 (bias 7, 3 mantissa bits,
+# exponent field 0 subnormal with step 2^-9, 0x7F / 0xFF NaN, no infinities).
+E4M3_TABLE = {
+    0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x0F: 1.875 * 2.0 ** -6,
+    0x30: 0.5, 0x38: 1.0, 0x39: 1.125, 0x3F: 1.875, 0x40: 2.0, 0x54: 12.0, 0x77: 240.0,
+    0x78: 256.0, 0x7E: 448.0, 0x81: -(2.0 ** -9), 0xB8: -1.0, 0xC4: -3.0, 0xFE: -448.0,
+}
+
+
+def pin_e4m3_table():
+    v = oracle.e4m3_to_f64(np.arange(256, dtype=np.uint8))
+    for code, want in E4M3_TABLE.items():
+        assert v[code] == want, (hex(code), v[code], want)
+    assert np.isnan(v[0x7F]) and np.isnan(v[0xFF])
+    assert v[0x80] == 0.0 and np.signbit(v[0x80])
+    assert np.isfinite(np.delete(v, [0x7F, 0xFF])).all()
+
+
+def pin_e4m3_library_and_order():
+    """All 256 codes agree with torch's float8_e4m3fn, the positive codes are
+    strictly increasing and the negative ones mirror them."""
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    v = oracle.e4m3_to_f64(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    same = (v == ref) | (np.isnan(v) & np.isnan(ref))
+    assert same.all(), np.nonzero(~same)[0][:8]
+    pos = v[:0x7F]
+    assert (np.diff(pos) > 0).all()
+    assert np.array_equal(v[0x80:0xFF], -pos)
+
+
 ALL_PINS = [
     pin_worked_example_recurrence,
     pin_worked_example_fp32,
@@ -396,4 +428,6 @@ ALL_PINS = [
     pin_backward_invariants,
     pin_sampled_backward_matches_full,
     pin_bf16_input_path,
+    pin_e4m3_table,
+    pin_e4m3_library_and_order,
 ]

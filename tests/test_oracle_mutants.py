@@ -36,6 +36,11 @@ MUTANTS = [
     ("scale_squared", "s[j] = pb->scale * acc;", "s[j] = pb->scale * pb->scale * acc;", None),
     ("dq_transposed_operand", "dqi[t] += pb->scale * ds * kvec[t];",
      "dqi[t] += pb->scale * ds * qi[t];", None),
+    ("e4m3_bias_8", "mag = ldexp(1.0 + m / 8.0, e - 7);", "mag = ldexp(1.0 + m / 8.0, e - 8);", None),
+    ("e4m3_subnormal_step", "mag = ldexp((double)m, -9);", "mag = ldexp((double)m, -10);", None),
+    ("e4m3_mantissa_width", "mag = ldexp(1.0 + m / 8.0, e - 7);", "mag = ldexp(1.0 + m / 16.0, e - 7);",
+     None),
+    ("e4m3_no_nan", "if (e == 15 && m == 7)", "if (e == 16)", None),
 ]
 
 
