@@ -302,6 +302,44 @@ def run_libfa(args, rank, world, local):
     e2e_ms = max_over_ranks(e2e_ms, world, dev)
     e2e_value = world * flops_step / (e2e_ms * 1e-3) / 1e12
 
+    # ---- the same workload with fp16 inputs, and the e4m3 forward (kind::f8f6f4)
+    x16 = {k: v.to(dev) for k, v in synth.make_inputs(w, dtype=torch.float16).items()}
+    o16, dq16 = torch.empty_like(x16["q"]), torch.empty_like(x16["q"])
+    dk16, dv16 = torch.empty_like(x16["k"]), torch.empty_like(x16["v"])
+
+    def fwd16():
+        fa.fa_fwd(x16["q"], x16["k"], x16["v"], o16, lse, causal=True, scale=w.scale)
+
+    def bwd16():
+        fa.fa_bwd(x16["q"], x16["k"], x16["v"], o16, x16["dout"], lse, dq16, dk16, dv16, causal=True,
+                  scale=w.scale, workspace=ws)
+
+    for _ in range(3):
+        fwd16()
+        bwd16()
+    torch.cuda.synchronize()
+    f16_ms = statistics.median(timed(fwd16, max(10, args.steps)))
+    b16_ms = statistics.median(timed(bwd16, max(10, args.steps)))
+    fa.fa_check_device_status()
+    del x16, o16, dq16, dk16, dv16
+
+    DS = synth.FP8_DESCALE
+    x8 = {k: v.to(dev) for k, v in synth.make_inputs_fp8(w).items()}
+    ws8 = torch.empty(fa.fa_fwd_fp8_workspace_size(w.B, w.Hkv, w.Nk, w.d), dtype=torch.uint8,
+                      device=dev)
+
+    def fwd8():
+        fa.fa_fwd_fp8(x8["q"], x8["k"], x8["v"], DS["q"], DS["k"], DS["v"], o, lse, causal=True,
+                      scale=w.scale, workspace=ws8)
+
+    for _ in range(3):
+        fwd8()
+    torch.cuda.synchronize()
+    f8_ms = statistics.median(timed(fwd8, max(10, args.steps)))
+    f8_tf = w.fwd_flops() / (f8_ms * 1e-3) / 1e12
+    fa.fa_check_device_status()
+    del x8, ws8
+
     # ---- decode workload (HBM-bound path)
     wd = synth.WORKLOADS[DECODE_WORKLOAD]
     wd = wd.with_(seed=rank_seed(wd.seed, rank))
@@ -364,6 +402,13 @@ def run_libfa(args, rank, world, local):
         "parts": {
             "fwd": {"ms": fwd_med, "tflops": fwd_tf, "frac_of_peak": fwd_tf / peaks["bf16_tflops_sustained"]},
             "bwd": {"ms": bwd_med, "tflops": bwd_tf, "frac_of_peak": bwd_tf / peaks["bf16_tflops_sustained"]},
+            "fwd_fp16": {"ms": f16_ms, "tflops": w.fwd_flops() / (f16_ms * 1e-3) / 1e12},
+            "bwd_fp16": {"ms": b16_ms, "tflops": w.bwd_flops() / (b16_ms * 1e-3) / 1e12},
+            "fwd_fp8": {"ms": f8_ms, "tflops": f8_tf,
+                        "peak": 2 * peaks["bf16_tflops"],
+                        "frac_of_peak": f8_tf / (2 * peaks["bf16_tflops"]),
+                        "peak_source": "measured burst bf16 x 2 (nominal e4m3 / bf16 dense ratio)",
+                        "includes": "V transpose kernel + forward kernel"},
             "decode": {"workload": f"{DECODE_WORKLOAD}: B=64, Hq=32, Hkv=8, Nq=1, Nk=8192, d=128",
                        "ms": dec_ms, "gbs": dec_gbs, "frac_of_hbm": dec_gbs / peaks["hbm_gbs"],
                        "algorithmic_bytes": dec_bytes},
@@ -396,6 +441,7 @@ PROFILE_CASES = {
     "fwd": ("gqa_8k", dict(Nq=4096, Nk=4096)),
     "bwd": ("gqa_8k", dict(Nq=4096, Nk=4096)),
     "decode": ("gqa_decode", dict(B=16)),
+    "fwd_fp8": ("gqa_8k", dict(Nq=4096, Nk=4096)),
 }
 
 
@@ -408,9 +454,15 @@ def run_profile(which: str, launches: int = 3) -> int:
     w = synth.WORKLOADS[name].with_(**over)
     x = {k: v.cuda() for k, v in synth.make_inputs(w).items()}
     o, lse = fa.fa_fwd(x["q"], x["k"], x["v"], causal=w.causal, scale=w.scale)
+    if which == "fwd_fp8":
+        DS = synth.FP8_DESCALE
+        x = {k: v.cuda() for k, v in synth.make_inputs_fp8(w).items()}
     for _ in range(launches):
         if which == "bwd":
             fa.fa_bwd(x["q"], x["k"], x["v"], o, x["dout"], lse, causal=w.causal, scale=w.scale)
+        elif which == "fwd_fp8":
+            fa.fa_fwd_fp8(x["q"], x["k"], x["v"], DS["q"], DS["k"], DS["v"], o, lse, causal=w.causal,
+                          scale=w.scale)
         else:
             fa.fa_fwd(x["q"], x["k"], x["v"], o, lse, causal=w.causal, scale=w.scale)
     torch.cuda.synchronize()

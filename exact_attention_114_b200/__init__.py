@@ -25,6 +25,9 @@ FA_ERR_WORKSPACE = 3
 FA_ERR_CUDA = 4
 FA_ERR_TIMEOUT = 5
 
+FA_DTYPE_BF16 = 0
+FA_DTYPE_FP16 = 1
+
 _lock = threading.Lock()
 _lib = None
 
@@ -55,6 +58,16 @@ def lib() -> ctypes.CDLL:
             L.fa_last_error_message.restype = ctypes.c_char_p
             L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, fl, ip, vp]
             L.fa_fwd.restype = ip
+            L.fa_fwd_ex.argtypes = [ip, vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, fl, ip, vp]
+            L.fa_fwd_ex.restype = ip
+            L.fa_bwd_ex.argtypes = [ip, vp, vp, vp, vp, vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, fl, ip,
+                                    vp, sz, vp]
+            L.fa_bwd_ex.restype = ip
+            L.fa_fwd_fp8_workspace_size.argtypes = [ip, ip, ip, ip]
+            L.fa_fwd_fp8_workspace_size.restype = sz
+            L.fa_fwd_fp8.argtypes = [vp, vp, vp, fl, fl, fl, vp, vp, ip, ip, ip, ip, ip, ip, fl, ip, vp,
+                                     sz, vp]
+            L.fa_fwd_fp8.restype = ip
             L.fa_fwd_splitkv_workspace_size.argtypes = [ip, ip, ip, ip, ip, ip, ip]
             L.fa_fwd_splitkv_workspace_size.restype = sz
             L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, fl, ip, ip, vp,
@@ -121,23 +134,74 @@ def _require(t, name, dtype):
         raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
 
 
+def _dtype_code(t):
+    """FA_DTYPE_* of a 16-bit tensor."""
+    import torch
+    if t.dtype == torch.bfloat16:
+        return FA_DTYPE_BF16
+    if t.dtype == torch.float16:
+        return FA_DTYPE_FP16
+    raise ValueError(f"unsupported dtype {t.dtype} (bf16 or fp16)")
+
+
 def abi_version() -> int:
     return int(lib().fa_abi_version())
 
 
 def fa_fwd(q, k, v, o=None, lse=None, *, causal=False, scale=None, stream=None, want_lse=True):
-    """Forward: returns (o, lse).  Allocates o / lse when not given."""
+    """Forward: returns (o, lse).  Allocates o / lse when not given.  bf16
+    tensors go to fa_fwd, fp16 tensors to fa_fwd_ex."""
     import torch
     B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
+    dt = _dtype_code(q)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _require(t, n, torch.bfloat16)
+        _require(t, n, q.dtype)
     if o is None:
         o = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    _check(lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d,
-                        scale, int(bool(causal)), _stream(stream)))
+    if dt == FA_DTYPE_BF16:
+        _check(lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d,
+                            scale, int(bool(causal)), _stream(stream)))
+    else:
+        _check(lib().fa_fwd_ex(dt, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk,
+                               d, scale, int(bool(causal)), _stream(stream)))
+    return o, lse
+
+
+def fa_fwd_fp8_workspace_size(B, Hkv, Nk, d) -> int:
+    return int(lib().fa_fwd_fp8_workspace_size(B, Hkv, Nk, d))
+
+
+def fa_fwd_fp8(q, k, v, descale_q, descale_k, descale_v, o=None, lse=None, *, causal=False,
+               scale=None, workspace=None, stream=None, want_lse=True):
+    """Forward with e4m3 inputs (uint8 or float8_e4m3fn CUDA tensors, d = 128)
+    and per-tensor descales.  Returns (o, lse) with o in bf16."""
+    import torch
+    B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if not t.is_cuda or not t.is_contiguous() or t.element_size() != 1:
+            raise ValueError(f"{n} must be a contiguous CUDA tensor of e4m3 bytes")
+    if o is None:
+        o = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    _require(o, "o", torch.bfloat16)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), float(descale_q), float(descale_k),
+                            float(descale_v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d, scale,
+                            int(bool(causal)), _ptr(workspace), ws_bytes, _stream(stream)))
+    return o, lse
+
+
+def fa_fwd_ex(dtype, q, k, v, o, lse, *, causal=False, scale=None, stream=None):
+    """The C call fa_fwd_ex with an explicit FA_DTYPE_* code."""
+    B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(lib().fa_fwd_ex(int(dtype), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq,
+                           Nk, d, scale, int(bool(causal)), _stream(stream)))
     return o, lse
 
 
@@ -225,9 +289,15 @@ def fa_bwd(q, k, v, o, dout, lse, dq=None, dk=None, dv=None, *, causal=False, sc
     dv = torch.empty_like(v) if dv is None else dv
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
-                        _ptr(dk), _ptr(dv), B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)),
-                        _ptr(workspace), ws_bytes, _stream(stream)))
+    dt = _dtype_code(q)
+    if dt == FA_DTYPE_BF16:
+        _check(lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                            _ptr(dk), _ptr(dv), B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)),
+                            _ptr(workspace), ws_bytes, _stream(stream)))
+    else:
+        _check(lib().fa_bwd_ex(dt, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                               _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv, Nq, Nk, d, scale,
+                               int(bool(causal)), _ptr(workspace), ws_bytes, _stream(stream)))
     return dq, dk, dv
 
 

@@ -68,7 +68,7 @@ __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_
 // ----------------------------------------------------------------------------
 // bwd_pre: D = rowsum(dO * O), LSE in log2 units, zero the dQ accumulator
 // ----------------------------------------------------------------------------
-template <int D>
+template <int D, typename T = __nv_bfloat16>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdParams p)
 {
     const int row = (int)(blockIdx.x * 8 + (threadIdx.x >> 5));   // over B * Hq * Nq_pad
@@ -89,23 +89,25 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdParams p)
         }
         return;
     }
-    const size_t src = ((size_t)bh * p.Nq + i) * D + lane * E;
+    const size_t src = ((size_t)bh * p.Nq + i) * p.d_io + lane * E;
     float s = 0.f;
-    if constexpr (E == 4) {
-        const uint2 a = *reinterpret_cast<const uint2*>(p.o + src);
-        const uint2 c = *reinterpret_cast<const uint2*>(p.dout + src);
-        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
-        const __nv_bfloat162* c2 = reinterpret_cast<const __nv_bfloat162*>(&c);
+    const T* po = static_cast<const T*>(p.o);
+    const T* pd = static_cast<const T*>(p.dout);
+    if (lane * E >= p.d_io) {
+        // padded columns of a narrower head: nothing to read
+    } else if constexpr (E == 4) {
+        const uint2 a = *reinterpret_cast<const uint2*>(po + src);
+        const uint2 c = *reinterpret_cast<const uint2*>(pd + src);
+        const uint32_t aw[2] = {a.x, a.y}, cw[2] = {c.x, c.y};
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            const float2 x = __bfloat1622float2(a2[e]), y = __bfloat1622float2(c2[e]);
+            const float2 x = Elt<T>::unpack(aw[e]), y = Elt<T>::unpack(cw[e]);
             s = fmaf(x.x, y.x, s);
             s = fmaf(x.y, y.y, s);
         }
     } else {
-        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(p.o + src);
-        const __nv_bfloat162 c = *reinterpret_cast<const __nv_bfloat162*>(p.dout + src);
-        const float2 x = __bfloat1622float2(a), y = __bfloat1622float2(c);
+        const float2 x = Elt<T>::unpack(*reinterpret_cast<const uint32_t*>(po + src));
+        const float2 y = Elt<T>::unpack(*reinterpret_cast<const uint32_t*>(pd + src));
         s = fmaf(x.x, y.x, s);
         s = fmaf(x.y, y.y, s);
     }
@@ -122,20 +124,20 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdParams p)
 // ----------------------------------------------------------------------------
 // bwd_post: dQ = bf16(scale * accumulator)
 // ----------------------------------------------------------------------------
-template <int D>
+template <int D, typename T = __nv_bfloat16>
 __global__ void __launch_bounds__(256) bwd_post_kernel(BwdParams p)
 {
-    const size_t n4 = (size_t)p.B * p.Hq * p.Nq * D / 4;
+    const size_t n4 = (size_t)p.B * p.Hq * p.Nq * p.d_io / 4;
     for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n4;
          idx += (size_t)gridDim.x * blockDim.x) {
         const size_t e = idx * 4;
-        const size_t row = e / D, c = e % D;
+        const size_t row = e / p.d_io, c = e % p.d_io;
         const size_t bh = row / p.Nq, i = row % p.Nq;
         const float4 a = *reinterpret_cast<const float4*>(p.dq_acc + (bh * p.Nq_pad + i) * D + c);
         uint2 w;
-        w.x = pack_bf16x2(a.x * p.scale, a.y * p.scale);
-        w.y = pack_bf16x2(a.z * p.scale, a.w * p.scale);
-        *reinterpret_cast<uint2*>(p.dq + e) = w;
+        w.x = Elt<T>::pack(a.x * p.scale, a.y * p.scale);
+        w.y = Elt<T>::pack(a.z * p.scale, a.w * p.scale);
+        *reinterpret_cast<uint2*>(static_cast<T*>(p.dq) + e) = w;
     }
 }
 
@@ -185,7 +187,7 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int chunk)
     return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, typename T = __nv_bfloat16>
 __global__ void __launch_bounds__(384, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -305,9 +307,10 @@ __global__ void __launch_bounds__(384, 1)
         // ------------------------------------------------------------ MMA issuer
         // (the whole warp runs this loop; one elected lane issues each MMA)
         {
-            const uint32_t id_sdp = idesc_bf16_f32(128, 64, false, false);   // S^T, dP^T
-            const uint32_t id_grad = idesc_bf16_f32(128, D, false, true);    // dV, dK
-            const uint32_t id_dq = idesc_bf16_f32(128, 64, true, true);      // dQ^T
+            constexpr uint32_t fmt = Elt<T>::kMmaFmt;
+            const uint32_t id_sdp = idesc_f16kind(fmt, 128, 64, false, false);   // S^T, dP^T
+            const uint32_t id_grad = idesc_f16kind(fmt, 128, D, false, true);    // dV, dK
+            const uint32_t id_dq = idesc_f16kind(fmt, 128, 64, true, true);      // dQ^T
             const uint32_t tDK = tmem + C::kColDK, tDV = tmem + C::kColDV, tS = tmem + C::kColS,
                            tDP = tmem + C::kColDP, tDQ = tmem + C::kColDQ;
             // base descriptors; a byte offset `o` inside an operand is added as o >> 4
@@ -437,8 +440,8 @@ __global__ void __launch_bounds__(384, 1)
                 const float2 dd2 = fadd2(make_float2(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])),
                                          make_float2(-dlt[c], -dlt[c + 1]));
                 const float2 ds2 = fmul2(pv, dd2);
-                pp[c >> 1] = pack_bf16x2(pv.x, pv.y);
-                dd[c >> 1] = pack_bf16x2(ds2.x, ds2.y);
+                pp[c >> 1] = Elt<T>::pack(pv.x, pv.y);
+                dd[c >> 1] = Elt<T>::pack(ds2.x, ds2.y);
             }
             // P^T over this step's S^T columns (the dV MMA reads it from there)
             tmem_st32(tSb, pp);
@@ -469,9 +472,12 @@ __global__ void __launch_bounds__(384, 1)
         if (ok) {
             tc_fence_after();
             const bool key_ok = key < p.Nk;
-            const size_t krow = ((size_t)kvh * p.Nk + key) * D;
+            const int d_io = p.d_io;
 #pragma unroll 1
             for (int c0 = 0; c0 < D; c0 += 32) {
+                if (c0 >= d_io)   // padded columns of a narrower head
+                    break;
+                const size_t krow = ((size_t)kvh * p.Nk + key) * d_io;
                 uint32_t a[32], v[32];
                 if (n_it > 0) {
                     tmem_ld32(tmem + lane_off + C::kColDK + c0, a);
@@ -485,11 +491,11 @@ __global__ void __launch_bounds__(384, 1)
                     uint32_t wk[16], wv[16];
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
-                        wk[c] = pack_bf16x2(__uint_as_float(a[2 * c]) * p.scale, __uint_as_float(a[2 * c + 1]) * p.scale);
-                        wv[c] = pack_bf16x2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1]));
+                        wk[c] = Elt<T>::pack(__uint_as_float(a[2 * c]) * p.scale, __uint_as_float(a[2 * c + 1]) * p.scale);
+                        wv[c] = Elt<T>::pack(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1]));
                     }
-                    uint4* dk4 = reinterpret_cast<uint4*>(p.dk + krow + c0);
-                    uint4* dv4 = reinterpret_cast<uint4*>(p.dv + krow + c0);
+                    uint4* dk4 = reinterpret_cast<uint4*>(static_cast<T*>(p.dk) + krow + c0);
+                    uint4* dv4 = reinterpret_cast<uint4*>(static_cast<T*>(p.dv) + krow + c0);
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         dk4[c] = make_uint4(wk[4 * c], wk[4 * c + 1], wk[4 * c + 2], wk[4 * c + 3]);

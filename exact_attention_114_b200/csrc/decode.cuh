@@ -40,13 +40,22 @@ struct DecCfg {
     static constexpr int kSmemBytes = kOffBar + 128 + 1024;
 };
 
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+// D += A B with 16-bit A/B (bf16 or fp16) and fp32 accumulators
+template <typename T>
+__device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
 {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    if constexpr (Elt<T>::kMmaFmt == 1u)
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+            "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+    else
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+            "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3)
@@ -73,7 +82,7 @@ __device__ __forceinline__ uint32_t dec_tile_off(int key, int chunk)
     return (uint32_t)(panel * DecCfg::kPanelBytes + key * 128 + ((c ^ (key & 7)) << 4));
 }
 
-template <bool PAGED>
+template <bool PAGED, typename T = __nv_bfloat16>
 __global__ void __launch_bounds__(160)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         DecodeParams p)
@@ -160,7 +169,7 @@ __global__ void __launch_bounds__(160)
                 continue;
             const int h = hk * p.G + r / p.Nq, i = r % p.Nq;
             const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-                p.q + (((size_t)b * p.Hq + h) * p.Nq + i) * 128);
+                static_cast<const T*>(p.q) + (((size_t)b * p.Hq + h) * p.Nq + i) * 128);
             for (int ks = 0; ks < 8; ++ks) {
                 qa[ks][hr] = __ldg(qrow + ks * 8 + tq);          // cols 16ks + 2tq, +1
                 qa[ks][hr + 2] = __ldg(qrow + ks * 8 + 4 + tq);  // cols 16ks + 8 + 2tq, +1
@@ -201,8 +210,8 @@ __global__ void __launch_bounds__(160)
             for (int ks = 0; ks < 8; ++ks) {
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4(kbase + dec_tile_off(key, 2 * ks + (mi & 1)), b0, b1, b2, b3);
-                mma_bf16_16816(s[0], qa[ks], b0, b1);
-                mma_bf16_16816(s[1], qa[ks], b2, b3);
+                mma_16816<T>(s[0], qa[ks], b0, b1);
+                mma_16816<T>(s[1], qa[ks], b2, b3);
             }
         }
         // mask: keys past the chunk / causal limit
@@ -231,8 +240,8 @@ __global__ void __launch_bounds__(160)
             const float p10 = ex2_approx(fmaf(s[1][2 * hr], sl2, neg_m));
             const float p11 = ex2_approx(fmaf(s[1][2 * hr + 1], sl2, neg_m));
             l[hr] = l[hr] * a + (p00 + p01 + p10 + p11);
-            pa[hr] = pack_bf16x2(p00, p01);       // keys 2tq, 2tq+1
-            pa[hr + 2] = pack_bf16x2(p10, p11);   // keys 8 + 2tq, +1
+            pa[hr] = Elt<T>::pack(p00, p01);       // keys 2tq, 2tq+1
+            pa[hr + 2] = Elt<T>::pack(p10, p11);   // keys 8 + 2tq, +1
 #pragma unroll
             for (int nd = 0; nd < 16; ++nd) {
                 o[nd][2 * hr] *= a;
@@ -247,8 +256,8 @@ __global__ void __launch_bounds__(160)
             for (int nd = 0; nd < 16; nd += 2) {
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4_t(vbase + dec_tile_off(key, nd + (mi >> 1)), b0, b1, b2, b3);
-                mma_bf16_16816(o[nd], pa, b0, b1);
-                mma_bf16_16816(o[nd + 1], pa, b2, b3);
+                mma_16816<T>(o[nd], pa, b0, b1);
+                mma_16816<T>(o[nd + 1], pa, b2, b3);
             }
         }
         __syncwarp();
@@ -301,7 +310,7 @@ __global__ void __launch_bounds__(160)
         if (p.splits == 1) {
             const int h = hk * p.G + r / p.Nq, i = r % p.Nq;
             const size_t row = ((size_t)b * p.Hq + h) * p.Nq + i;
-            p.o[row * 128 + dcol] = __float2bfloat16_rn(on);
+            static_cast<T*>(p.o)[row * 128 + dcol] = Elt<T>::from_float(on);
             if (dcol == 0 && p.lse)
                 p.lse[row] = lse;
         } else {
@@ -314,6 +323,7 @@ __global__ void __launch_bounds__(160)
 }
 
 // One warp per output row (b, kv head, r): merge the partials of all splits.
+template <typename T = __nv_bfloat16>
 __global__ void __launch_bounds__(128) decode_combine_kernel(DecodeParams p)
 {
     const int warp = (int)(blockIdx.x * 4 + (threadIdx.x >> 5));
@@ -350,9 +360,9 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(DecodeParams p)
     const int h = hk * p.G + r / p.Nq, i = r % p.Nq;
     const size_t row = ((size_t)b * p.Hq + h) * p.Nq + i;
     uint2 w2;
-    w2.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-    w2.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<uint2*>(p.o + row * 128 + lane * 4) = w2;
+    w2.x = Elt<T>::pack(acc[0] * inv, acc[1] * inv);
+    w2.y = Elt<T>::pack(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(static_cast<T*>(p.o) + row * 128 + lane * 4) = w2;
     if (lane == 0 && p.lse)
         p.lse[row] = (L > 0.f) ? M + __logf(L) : -INFINITY;
 }

@@ -15,10 +15,12 @@
 #include <map>
 #include <mutex>
 #include <string>
+#include <type_traits>
 
 #include "bwd.cuh"
 #include "decode.cuh"
 #include "fa_kernels.h"
+#include "fp8.cuh"
 #include "fwd.cuh"
 
 namespace {
@@ -90,8 +92,8 @@ fa_status_t check_shape(int B, int Hq, int Hkv, int Nq, int Nk, int d, float sca
         set_error("problem too large for 32-bit row indices");
         return FA_ERR_UNSUPPORTED;
     }
-    if (d != 64 && d != 128) {
-        set_error("d=%d is not supported (64 or 128)", d);
+    if (d != 32 && d != 64 && d != 96 && d != 128) {
+        set_error("d=%d is not supported (32, 64, 96 or 128)", d);
         return FA_ERR_UNSUPPORTED;
     }
     return FA_OK;
@@ -118,10 +120,17 @@ EncodeTiledFn get_encode()
     return fn;
 }
 
-// 3-D map over a [outer][rows][inner] bf16 tensor, box {64, box_rows, 1}, 128-byte
-// swizzle; rows past `rows` read as zero.
-fa_status_t make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
-                     uint32_t box_rows)
+template <typename T>
+constexpr CUtensorMapDataType tma_type()
+{
+    return std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+}
+
+// 3-D map over a [outer][rows][inner] tensor of `elt` -byte elements, box
+// {box_inner, box_rows, 1} with box_inner * elt = 128 bytes (the 128-byte
+// swizzle span); elements past `inner` or `rows` read as zero.
+fa_status_t make_map_box(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
+                         uint32_t elt, uint32_t box_inner, uint32_t box_rows, CUtensorMapDataType dt)
 {
     EncodeTiledFn enc = get_encode();
     if (!enc) {
@@ -129,10 +138,10 @@ fa_status_t make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t 
         return FA_ERR_CUDA;
     }
     cuuint64_t dims[3] = {inner, rows, outer};
-    cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
-    cuuint32_t box[3] = {64, box_rows, 1};
+    cuuint64_t strides[2] = {inner * elt, inner * rows * elt};
+    cuuint32_t box[3] = {box_inner, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+    CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
@@ -140,6 +149,13 @@ fa_status_t make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t 
         return FA_ERR_CUDA;
     }
     return FA_OK;
+}
+
+// 16-bit tensor [outer][rows][inner], box {64, box_rows, 1}
+fa_status_t make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
+                     uint32_t box_rows, CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)
+{
+    return make_map_box(m, base, inner, rows, outer, 2, 64, box_rows, dt);
 }
 
 // 4-D map over a paged KV pool [pages][page_size][Hkv][d] (bf16), box {64, 1, 64, 1}
@@ -211,20 +227,25 @@ int sm_count()
 // ---------------------------------------------------------------------------
 // forward (tiled kernel)
 // ---------------------------------------------------------------------------
-template <int D, bool CAUSAL>
+// Kernel head dim for a head dim d of the tensors: 32 runs on the 64 kernels and
+// 96 on the 128 kernels, the missing columns being zero fill of the TMA boxes
+// (zero columns add nothing to Q K^T, and P V gives zero there, never stored).
+int kernel_d(int d) { return d <= 64 ? 64 : 128; }
+
+template <int D, bool CAUSAL, typename T>
 fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
-                       int Nq, int Nk, float scale, cudaStream_t stream)
+                       int Nq, int Nk, int d, float scale, cudaStream_t stream)
 {
     using C = fa::FwdCfg<D>;
     CUtensorMap mq, mk, mv;
     fa_status_t st;
-    if ((st = make_map(&mq, q, D, Nq, (uint64_t)B * Hq, 128)) != FA_OK) return st;
-    if ((st = make_map(&mk, k, D, Nk, (uint64_t)B * Hkv, 128)) != FA_OK) return st;
-    if ((st = make_map(&mv, v, D, Nk, (uint64_t)B * Hkv, 128)) != FA_OK) return st;
-    auto kern = fa::fwd_kernel<D, CAUSAL>;
+    if ((st = make_map(&mq, q, d, Nq, (uint64_t)B * Hq, 128, tma_type<T>())) != FA_OK) return st;
+    if ((st = make_map(&mk, k, d, Nk, (uint64_t)B * Hkv, 128, tma_type<T>())) != FA_OK) return st;
+    if ((st = make_map(&mv, v, d, Nk, (uint64_t)B * Hkv, 128, tma_type<T>())) != FA_OK) return st;
+    auto kern = fa::fwd_kernel<D, CAUSAL, T>;
     if ((st = ensure_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes)) != FA_OK) return st;
     fa::FwdParams p;
-    p.o = static_cast<__nv_bfloat16*>(o);
+    p.o = o;
     p.lse = lse;
     p.B = B;
     p.Hq = Hq;
@@ -233,20 +254,77 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     p.Nk = Nk;
     p.G = Hq / Hkv;
     p.n_pairs = (Nq + 255) / 256;
+    p.d_io = d;
     p.scale_log2 = scale * kLog2e;
+    p.o_scale = 1.f;
     const long long grid = (long long)p.n_pairs * B * Hq;
     kern<<<(unsigned)grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
     return check_launch("fwd_kernel launch");
 }
 
-fa_status_t fwd_tiled(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
-                      int Nq, int Nk, int d, float scale, int causal, cudaStream_t s)
+// ---------------------------------------------------------------------------
+// forward with e4m3 inputs (d = 128): V^T into the workspace, then the tiled
+// kernel on kind::f8f6f4
+// ---------------------------------------------------------------------------
+constexpr int kF8D = 128;
+
+size_t fp8_nk_pad(int Nk) { return ((size_t)Nk + 15) / 16 * 16; }
+
+size_t fp8_workspace_bytes(int B, int Hkv, int Nk) { return align256((size_t)B * Hkv * kF8D * fp8_nk_pad(Nk)); }
+
+template <bool CAUSAL>
+fa_status_t launch_fwd_fp8(const void* q, const void* k, const void* v, void* vt, void* o, float* lse, int B,
+                           int Hq, int Hkv, int Nq, int Nk, float scale_log2, float o_scale, cudaStream_t stream)
 {
-    if (d == 128)
-        return causal ? launch_fwd<128, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, s)
-                      : launch_fwd<128, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, s);
-    return causal ? launch_fwd<64, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, s)
-                  : launch_fwd<64, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, s);
+    using C = fa::FwdCfg<kF8D, true>;
+    const int nk_pad = (int)fp8_nk_pad(Nk);
+    const dim3 tgrid((unsigned)((nk_pad + 63) / 64), (unsigned)(B * Hkv));
+    fa::fp8_vt_kernel<kF8D><<<tgrid, 256, 0, stream>>>(static_cast<const uint8_t*>(v), static_cast<uint8_t*>(vt),
+                                                      Nk, nk_pad);
+    fa_status_t st;
+    if ((st = check_launch("fp8_vt_kernel launch")) != FA_OK) return st;
+    constexpr CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    CUtensorMap mq, mk, mv;
+    if ((st = make_map_box(&mq, q, kF8D, Nq, (uint64_t)B * Hq, 1, 128, 128, u8)) != FA_OK) return st;
+    if ((st = make_map_box(&mk, k, kF8D, Nk, (uint64_t)B * Hkv, 1, 128, 128, u8)) != FA_OK) return st;
+    // V^T [B * Hkv][d][nk_pad]: box of 128 keys x d rows
+    if ((st = make_map_box(&mv, vt, nk_pad, kF8D, (uint64_t)B * Hkv, 1, 128, kF8D, u8)) != FA_OK) return st;
+    auto kern = fa::fwd_kernel<kF8D, CAUSAL, __nv_bfloat16, true>;
+    if ((st = ensure_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes)) != FA_OK) return st;
+    fa::FwdParams p;
+    p.o = o;
+    p.lse = lse;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.G = Hq / Hkv;
+    p.n_pairs = (Nq + 255) / 256;
+    p.d_io = kF8D;
+    p.scale_log2 = scale_log2;
+    p.o_scale = o_scale;
+    const long long grid = (long long)p.n_pairs * B * Hq;
+    kern<<<(unsigned)grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
+    return check_launch("fwd_kernel (e4m3) launch");
+}
+
+template <typename T>
+fa_status_t fwd_tiled_t(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                        int Nq, int Nk, int d, float scale, int causal, cudaStream_t s)
+{
+    if (kernel_d(d) == 128)
+        return causal ? launch_fwd<128, true, T>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, s)
+                      : launch_fwd<128, false, T>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, s);
+    return causal ? launch_fwd<64, true, T>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, s)
+                  : launch_fwd<64, false, T>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, s);
+}
+
+fa_status_t fwd_tiled(int dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                      int Hkv, int Nq, int Nk, int d, float scale, int causal, cudaStream_t s)
+{
+    return dtype == FA_DTYPE_FP16 ? fwd_tiled_t<__half>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, s)
+                                  : fwd_tiled_t<__nv_bfloat16>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -308,9 +386,10 @@ struct PagedDesc {
     int page_size, num_pages, max_pages;
 };
 
-fa_status_t launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
-                          int Nq, int Nk, int d, float scale, int causal, const DecodePlan& pl, void* ws,
-                          cudaStream_t stream, const PagedDesc* pg = nullptr)
+template <typename T>
+fa_status_t launch_decode_t(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                            int Hkv, int Nq, int Nk, int d, float scale, int causal, const DecodePlan& pl, void* ws,
+                            cudaStream_t stream, const PagedDesc* pg)
 {
     using C = fa::DecCfg;
     CUtensorMap mk, mv;
@@ -319,16 +398,16 @@ fa_status_t launch_decode(const void* q, const void* k, const void* v, void* o, 
         if ((st = make_map_paged(&mk, k, d, Hkv, pg->page_size, pg->num_pages)) != FA_OK) return st;
         if ((st = make_map_paged(&mv, v, d, Hkv, pg->page_size, pg->num_pages)) != FA_OK) return st;
     } else {
-        if ((st = make_map(&mk, k, d, Nk, (uint64_t)B * Hkv, 64)) != FA_OK) return st;
-        if ((st = make_map(&mv, v, d, Nk, (uint64_t)B * Hkv, 64)) != FA_OK) return st;
+        if ((st = make_map(&mk, k, d, Nk, (uint64_t)B * Hkv, 64, tma_type<T>())) != FA_OK) return st;
+        if ((st = make_map(&mv, v, d, Nk, (uint64_t)B * Hkv, 64, tma_type<T>())) != FA_OK) return st;
     }
-    auto kern = pg ? fa::decode_split_kernel<true> : fa::decode_split_kernel<false>;
+    auto kern = pg ? fa::decode_split_kernel<true, T> : fa::decode_split_kernel<false, T>;
     if ((st = ensure_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes)) != FA_OK) return st;
     fa::DecodeParams p;
-    p.q = static_cast<const __nv_bfloat16*>(q);
-    p.k = static_cast<const __nv_bfloat16*>(k);
-    p.v = static_cast<const __nv_bfloat16*>(v);
-    p.o = static_cast<__nv_bfloat16*>(o);
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.o = o;
     p.lse = lse;
     p.part_o = pl.splits > 1 ? static_cast<float*>(ws) : nullptr;
     p.part_lse = pl.splits > 1 ? reinterpret_cast<float*>(static_cast<char*>(ws) + align256(pl.o_bytes)) : nullptr;
@@ -352,10 +431,19 @@ fa_status_t launch_decode(const void* q, const void* k, const void* v, void* o, 
     if ((st = check_launch("decode_split_kernel launch")) != FA_OK) return st;
     if (pl.splits > 1) {
         const long long rows = (long long)B * Hkv * p.R;
-        fa::decode_combine_kernel<<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(p);
+        fa::decode_combine_kernel<T><<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(p);
         if ((st = check_launch("decode_combine_kernel launch")) != FA_OK) return st;
     }
     return FA_OK;
+}
+
+fa_status_t launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                          int Nq, int Nk, int d, float scale, int causal, const DecodePlan& pl, void* ws,
+                          cudaStream_t stream, const PagedDesc* pg = nullptr, int dtype = FA_DTYPE_BF16)
+{
+    if (dtype == FA_DTYPE_FP16)
+        return launch_decode_t<__half>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, pl, ws, stream, pg);
+    return launch_decode_t<__nv_bfloat16>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, pl, ws, stream, pg);
 }
 
 // ---------------------------------------------------------------------------
@@ -407,34 +495,35 @@ BwdPlan bwd_plan(int B, int Hq, int Nq, int d)
     pl.delta_off = 0;
     pl.lse_off = align256(rows * 4);
     pl.acc_off = pl.lse_off + align256(rows * 4);
-    pl.total = pl.acc_off + align256(rows * d * 4);
+    pl.total = pl.acc_off + align256(rows * kernel_d(d) * 4);   // accumulator rows of the kernel width
     return pl;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, typename T>
 fa_status_t launch_bwd(const fa::BwdParams& p, const void* q, const void* k, const void* v, const void* dout,
                        cudaStream_t stream)
 {
     using C = fa::BwdCfg<D>;
     fa_status_t st;
     const long long rows = (long long)p.B * p.Hq * p.Nq_pad;
-    fa::bwd_pre_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p);
+    fa::bwd_pre_kernel<D, T><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p);
     if ((st = check_launch("bwd_pre_kernel launch")) != FA_OK) return st;
 
     CUtensorMap mq, mk, mv, mdo;
-    if ((st = make_map(&mq, q, D, p.Nq, (uint64_t)p.B * p.Hq, 64)) != FA_OK) return st;
-    if ((st = make_map(&mdo, dout, D, p.Nq, (uint64_t)p.B * p.Hq, 64)) != FA_OK) return st;
-    if ((st = make_map(&mk, k, D, p.Nk, (uint64_t)p.B * p.Hkv, 128)) != FA_OK) return st;
-    if ((st = make_map(&mv, v, D, p.Nk, (uint64_t)p.B * p.Hkv, 128)) != FA_OK) return st;
-    auto kern = fa::bwd_main_kernel<D, CAUSAL>;
+    constexpr CUtensorMapDataType dt = tma_type<T>();
+    if ((st = make_map(&mq, q, p.d_io, p.Nq, (uint64_t)p.B * p.Hq, 64, dt)) != FA_OK) return st;
+    if ((st = make_map(&mdo, dout, p.d_io, p.Nq, (uint64_t)p.B * p.Hq, 64, dt)) != FA_OK) return st;
+    if ((st = make_map(&mk, k, p.d_io, p.Nk, (uint64_t)p.B * p.Hkv, 128, dt)) != FA_OK) return st;
+    if ((st = make_map(&mv, v, p.d_io, p.Nk, (uint64_t)p.B * p.Hkv, 128, dt)) != FA_OK) return st;
+    auto kern = fa::bwd_main_kernel<D, CAUSAL, T>;
     if ((st = ensure_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes)) != FA_OK) return st;
     const long long grid = (long long)((p.Nk + 127) / 128) * p.B * p.Hkv;
     kern<<<(unsigned)grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mdo, p);
     if ((st = check_launch("bwd_main_kernel launch")) != FA_OK) return st;
 
-    const long long n4 = (long long)p.B * p.Hq * p.Nq * D / 4;
+    const long long n4 = (long long)p.B * p.Hq * p.Nq * p.d_io / 4;
     const long long blocks = std::min<long long>((n4 + 255) / 256, (long long)sm_count() * 8);
-    fa::bwd_post_kernel<D><<<(unsigned)std::max<long long>(blocks, 1), 256, 0, stream>>>(p);
+    fa::bwd_post_kernel<D, T><<<(unsigned)std::max<long long>(blocks, 1), 256, 0, stream>>>(p);
     return check_launch("bwd_post_kernel launch");
 }
 
@@ -480,11 +569,15 @@ const char* fa_status_string(fa_status_t s)
 
 const char* fa_last_error_message(void) { return t_error.c_str(); }
 
-fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
-                   int Nq, int Nk, int d, float scale, int causal, void* stream)
+static fa_status_t fwd_entry(int dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                             int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, void* stream)
 {
     t_error.clear();
     fa_status_t st;
+    if (dtype != FA_DTYPE_BF16 && dtype != FA_DTYPE_FP16) {
+        set_error("dtype=%d is not FA_DTYPE_BF16 or FA_DTYPE_FP16", dtype);
+        return FA_ERR_INVALID_ARGUMENT;
+    }
     if ((st = check_ptr(q, "q")) || (st = check_ptr(k, "k")) || (st = check_ptr(v, "v")) ||
         (st = check_ptr(o, "o")))
         return st;
@@ -496,7 +589,7 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
         return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (!decode_shape(Hq, Hkv, Nq, d))
-        return fwd_tiled(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, s);
+        return fwd_tiled(dtype, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, s);
     const DecodePlan pl = decode_plan(B, Hq, Hkv, Nq, Nk, d, 0);
     void* ws = nullptr;
     if (pl.total() > 0) {
@@ -504,8 +597,87 @@ fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* 
         if (e != cudaSuccess)
             return cuda_fail(e, "cudaMallocAsync (split-KV partials)");
     }
-    st = launch_decode(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, pl, ws, s);
+    st = launch_decode(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, pl, ws, s, nullptr, dtype);
     if (ws) {
+        cudaError_t e = cudaFreeAsync(ws, s);
+        if (e != cudaSuccess && st == FA_OK)
+            st = cuda_fail(e, "cudaFreeAsync");
+    }
+    return st;
+}
+
+fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                   int Nq, int Nk, int d, float scale, int causal, void* stream)
+{
+    return fwd_entry(FA_DTYPE_BF16, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream);
+}
+
+fa_status_t fa_fwd_ex(fa_dtype_t dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                      int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, void* stream)
+{
+    return fwd_entry((int)dtype, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream);
+}
+
+size_t fa_fwd_fp8_workspace_size(int B, int Hkv, int Nk, int d)
+{
+    if (B < 1 || Hkv < 1 || Nk < 1 || d != kF8D)
+        return 0;
+    return fp8_workspace_bytes(B, Hkv, Nk);
+}
+
+fa_status_t fa_fwd_fp8(const void* q, const void* k, const void* v, float descale_q, float descale_k,
+                       float descale_v, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                       float scale, int causal, void* workspace, size_t workspace_bytes, void* stream)
+{
+    t_error.clear();
+    fa_status_t st;
+    if ((st = check_ptr(q, "q")) || (st = check_ptr(k, "k")) || (st = check_ptr(v, "v")) ||
+        (st = check_ptr(o, "o")))
+        return st;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) {
+        set_error("lse is not 4-byte aligned");
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    const float ds[3] = {descale_q, descale_k, descale_v};
+    for (float x : ds)
+        if (!(std::isfinite(x) && x > 0.f)) {
+            set_error("descale factors must be finite and > 0");
+            return FA_ERR_INVALID_ARGUMENT;
+        }
+    if ((st = check_shape(B, Hq, Hkv, Nq, Nk, d, scale, causal)) != FA_OK)
+        return st;
+    if (d != kF8D) {
+        set_error("the e4m3 forward takes d = 128 (got %d)", d);
+        return FA_ERR_UNSUPPORTED;
+    }
+    if ((long long)B * Hkv > 65535) {   // grid.y of the V transpose
+        set_error("the e4m3 forward takes B * Hkv <= 65535");
+        return FA_ERR_UNSUPPORTED;
+    }
+    const float scale_log2 = scale * descale_q * descale_k * kLog2e;
+    if (!(std::isfinite(scale_log2) && scale_log2 > 0.f)) {
+        set_error("scale * descale_q * descale_k is not a positive finite fp32 value");
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) {
+        set_error("workspace is not 256-byte aligned");
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    const size_t need = fp8_workspace_bytes(B, Hkv, Nk);
+    if (workspace && workspace_bytes < need) {
+        set_error("workspace has %zu bytes, %zu needed", workspace_bytes, need);
+        return FA_ERR_WORKSPACE;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    void* ws = workspace;
+    if (!ws) {
+        cudaError_t e = cudaMallocAsync(&ws, need, s);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaMallocAsync (V^T workspace)");
+    }
+    st = causal ? launch_fwd_fp8<true>(q, k, v, ws, o, lse, B, Hq, Hkv, Nq, Nk, scale_log2, descale_v, s)
+                : launch_fwd_fp8<false>(q, k, v, ws, o, lse, B, Hq, Hkv, Nq, Nk, scale_log2, descale_v, s);
+    if (!workspace) {
         cudaError_t e = cudaFreeAsync(ws, s);
         if (e != cudaSuccess && st == FA_OK)
             st = cuda_fail(e, "cudaFreeAsync");
@@ -690,12 +862,17 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d)
     return bwd_plan(B, Hq, Nq, d).total;
 }
 
-fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
-                   void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
-                   int causal, void* workspace, size_t workspace_bytes, void* stream)
+static fa_status_t bwd_entry(int dtype, const void* q, const void* k, const void* v, const void* o,
+                             const void* dout, const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv,
+                             int Nq, int Nk, int d, float scale, int causal, void* workspace,
+                             size_t workspace_bytes, void* stream)
 {
     t_error.clear();
     fa_status_t st;
+    if (dtype != FA_DTYPE_BF16 && dtype != FA_DTYPE_FP16) {
+        set_error("dtype=%d is not FA_DTYPE_BF16 or FA_DTYPE_FP16", dtype);
+        return FA_ERR_INVALID_ARGUMENT;
+    }
     if ((st = check_ptr(q, "q")) || (st = check_ptr(k, "k")) || (st = check_ptr(v, "v")) ||
         (st = check_ptr(o, "o")) || (st = check_ptr(dout, "dout")) || (st = check_ptr(lse, "lse")) ||
         (st = check_ptr(dq, "dq")) || (st = check_ptr(dk, "dk")) || (st = check_ptr(dv, "dv")))
@@ -721,15 +898,15 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
         owned = true;
     }
     fa::BwdParams p;
-    p.q = static_cast<const __nv_bfloat16*>(q);
-    p.k = static_cast<const __nv_bfloat16*>(k);
-    p.v = static_cast<const __nv_bfloat16*>(v);
-    p.o = static_cast<const __nv_bfloat16*>(o);
-    p.dout = static_cast<const __nv_bfloat16*>(dout);
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.o = o;
+    p.dout = dout;
     p.lse = lse;
-    p.dq = static_cast<__nv_bfloat16*>(dq);
-    p.dk = static_cast<__nv_bfloat16*>(dk);
-    p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
     char* w = static_cast<char*>(ws);
     p.delta = reinterpret_cast<float*>(w + pl.delta_off);
     p.lse_log2 = reinterpret_cast<float*>(w + pl.lse_off);
@@ -741,19 +918,48 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, c
     p.Nk = Nk;
     p.G = Hq / Hkv;
     p.Nq_pad = pl.Nq_pad;
+    p.d_io = d;
     p.causal = causal;
     p.scale = scale;
     p.scale_log2 = scale * kLog2e;
-    if (d == 128)
-        st = causal ? launch_bwd<128, true>(p, q, k, v, dout, s) : launch_bwd<128, false>(p, q, k, v, dout, s);
-    else
-        st = causal ? launch_bwd<64, true>(p, q, k, v, dout, s) : launch_bwd<64, false>(p, q, k, v, dout, s);
+    if (dtype == FA_DTYPE_FP16) {
+        if (kernel_d(d) == 128)
+            st = causal ? launch_bwd<128, true, __half>(p, q, k, v, dout, s)
+                        : launch_bwd<128, false, __half>(p, q, k, v, dout, s);
+        else
+            st = causal ? launch_bwd<64, true, __half>(p, q, k, v, dout, s)
+                        : launch_bwd<64, false, __half>(p, q, k, v, dout, s);
+    } else {
+        if (kernel_d(d) == 128)
+            st = causal ? launch_bwd<128, true, __nv_bfloat16>(p, q, k, v, dout, s)
+                        : launch_bwd<128, false, __nv_bfloat16>(p, q, k, v, dout, s);
+        else
+            st = causal ? launch_bwd<64, true, __nv_bfloat16>(p, q, k, v, dout, s)
+                        : launch_bwd<64, false, __nv_bfloat16>(p, q, k, v, dout, s);
+    }
     if (owned) {
         cudaError_t e = cudaFreeAsync(ws, s);
         if (e != cudaSuccess && st == FA_OK)
             st = cuda_fail(e, "cudaFreeAsync");
     }
     return st;
+}
+
+fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                   void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                   int causal, void* workspace, size_t workspace_bytes, void* stream)
+{
+    return bwd_entry(FA_DTYPE_BF16, q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                     workspace, workspace_bytes, stream);
+}
+
+fa_status_t fa_bwd_ex(fa_dtype_t dtype, const void* q, const void* k, const void* v, const void* o,
+                      const void* dout, const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv,
+                      int Nq, int Nk, int d, float scale, int causal, void* workspace, size_t workspace_bytes,
+                      void* stream)
+{
+    return bwd_entry((int)dtype, q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                     workspace, workspace_bytes, stream);
 }
 
 fa_status_t fa_check_device_status(void* stream)

@@ -8,19 +8,22 @@
 namespace fa {
 
 struct FwdParams {
-    __nv_bfloat16* o;   // [B, Hq, Nq, d]
+    void* o;            // [B, Hq, Nq, d] (bf16 or fp16)
     float* lse;         // [B, Hq, Nq] or nullptr
     int B, Hq, Hkv, Nq, Nk;
     int G;              // Hq / Hkv
     int n_pairs;        // ceil(Nq / 256): 256-row query tile pairs per head
-    float scale_log2;   // scale * log2(e)
+    int d_io;           // head dim of the tensors in memory (<= kernel D, multiple of 32); the
+                        // columns d_io..D-1 of the tiles are TMA zero fill and are never stored
+    float scale_log2;   // scale * log2(e) (times the Q and K descales for e4m3 inputs)
+    float o_scale;      // O = o_scale * U / l: 1, or the V descale for e4m3 inputs
 };
 
 struct DecodeParams {
-    const __nv_bfloat16* q;  // [B, Hq, Nq, d]
-    const __nv_bfloat16* k;  // [B, Hkv, Nk, d]
-    const __nv_bfloat16* v;
-    __nv_bfloat16* o;        // [B, Hq, Nq, d]
+    const void* q;           // [B, Hq, Nq, d]  (16-bit elements, bf16 or fp16)
+    const void* k;           // [B, Hkv, Nk, d]
+    const void* v;
+    void* o;                 // [B, Hq, Nq, d]
     float* lse;              // [B, Hq, Nq] or nullptr
     float* part_o;           // [B * Hkv, splits, R, d]  partial O_s (normalised)
     float* part_lse;         // [B * Hkv, splits, R]     partial lse_s
@@ -41,21 +44,22 @@ struct DecodeParams {
 };
 
 struct BwdParams {
-    const __nv_bfloat16* q;     // [B, Hq, Nq, d]
-    const __nv_bfloat16* k;     // [B, Hkv, Nk, d]
-    const __nv_bfloat16* v;
-    const __nv_bfloat16* o;     // [B, Hq, Nq, d]
-    const __nv_bfloat16* dout;  // [B, Hq, Nq, d]
+    const void* q;              // [B, Hq, Nq, d]  (16-bit elements, bf16 or fp16)
+    const void* k;              // [B, Hkv, Nk, d]
+    const void* v;
+    const void* o;              // [B, Hq, Nq, d]
+    const void* dout;           // [B, Hq, Nq, d]
     const float* lse;           // [B, Hq, Nq]
-    __nv_bfloat16* dq;          // [B, Hq, Nq, d]
-    __nv_bfloat16* dk;          // [B, Hkv, Nk, d]
-    __nv_bfloat16* dv;
+    void* dq;                   // [B, Hq, Nq, d]
+    void* dk;                   // [B, Hkv, Nk, d]
+    void* dv;
     float* delta;               // [B, Hq, Nq_pad]  D_i = rowsum(dout * o)
     float* lse_log2;            // [B, Hq, Nq_pad]  LSE_i * log2(e) (+inf for masked rows)
     float* dq_acc;              // [B, Hq, Nq_pad, d] fp32 accumulator
     int B, Hq, Hkv, Nq, Nk;
     int G;
     int Nq_pad;                 // Nq rounded up to the query block
+    int d_io;                   // head dim in memory (<= kernel D, multiple of 32); dq_acc keeps D
     int causal;
     float scale;
     float scale_log2;

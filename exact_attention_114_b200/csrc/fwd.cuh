@@ -38,19 +38,27 @@ namespace fa {
 constexpr float kRescaleLog2 = 8.0f;
 constexpr float kLn2 = 0.69314718055994530942f;
 
-template <int D>
+// F8: Q, K, V are e4m3 bytes and V arrives transposed (d rows of 128 keys),
+// see fp8_vt_kernel; otherwise they are 16-bit (T).
+template <int D, bool F8 = false>
 struct FwdCfg {
     static constexpr int kThreads = 384;
     // registers per thread after the split: 2 x 128 x 208 + 128 x 80 <= 384 x 168
     static constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 80;
-    static constexpr int kTileBytes = 128 * D * 2;   // a 128-row Q, K or V tile
-    static constexpr int kPanelBytes = 128 * 128;    // 128 rows x 64 bf16
-    static constexpr int kStages = (D == 128) ? 5 : 8;
+    static constexpr int kElt = F8 ? 1 : 2;              // bytes per Q/K/V element
+    static constexpr int kTileBytes = 128 * D * kElt;    // a 128-row Q or K tile, a V tile
+    static constexpr int kPanelBytes = 128 * 128;        // 128 rows x 128 bytes (one swizzle span)
+    static constexpr int kPanels = D * kElt / 128;
+    static constexpr int kPanelElems = 128 / kElt;
+    static constexpr int kKSteps = D * kElt / 32;        // Q.K^T instructions (32 bytes of d each)
+    static constexpr int kStages = F8 ? 10 : (D == 128) ? 5 : 8;
+    static constexpr int kBarBytes = F8 ? 512 : 256;
     static constexpr int kOffQ = 0;
     static constexpr int kOffKV = 2 * kTileBytes;
     static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
-    static constexpr int kSmemBytes = kOffBar + 256 + 1024;  // + barriers + alignment slack
+    static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + barriers + alignment slack
     static constexpr uint32_t kTmemCols = 512;
+    static_assert(!F8 || D == 128, "the e4m3 kernel is built for d = 128");
 };
 
 __device__ __forceinline__ int fwd_blocks_for_tile(int qt, int Nq, int Nk, bool causal)
@@ -67,12 +75,12 @@ __device__ __forceinline__ int fwd_blocks_for_tile(int qt, int Nq, int Nk, bool 
     return min(nkb, last_key / 128 + 1);
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, typename T = __nv_bfloat16, bool F8 = false>
 __global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, FwdParams p)
 {
-    using C = FwdCfg<D>;
+    using C = FwdCfg<D, F8>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -145,9 +153,9 @@ __global__ void __launch_bounds__(384, 1)
                 if (nblk[t] == 0)
                     continue;
                 mbar_arrive_expect_tx(&bar_q[t], C::kTileBytes);
-                for (int pn = 0; pn < D / 64; ++pn)
-                    tma_load_3d(sQ + t * C::kTileBytes + pn * C::kPanelBytes, &tmQ, &bar_q[t], pn * 64,
-                                q0 + 128 * t, bh);
+                for (int pn = 0; pn < C::kPanels; ++pn)
+                    tma_load_3d(sQ + t * C::kTileBytes + pn * C::kPanelBytes, &tmQ, &bar_q[t],
+                                pn * C::kPanelElems, q0 + 128 * t, bh);
             }
             int slot = 0;
             uint32_t round = 0;
@@ -161,9 +169,12 @@ __global__ void __launch_bounds__(384, 1)
                     }
                     uint8_t* dst = sKV + slot * C::kTileBytes;
                     mbar_arrive_expect_tx(&bar_full[slot], C::kTileBytes);
-                    for (int pn = 0; pn < D / 64; ++pn)
-                        tma_load_3d(dst + pn * C::kPanelBytes, kv ? &tmV : &tmK, &bar_full[slot], pn * 64,
-                                    j * 128, kvh);
+                    if (F8 && kv)   // V^T: d rows of keys j*128 .. j*128+127
+                        tma_load_3d(dst, &tmV, &bar_full[slot], j * 128, 0, kvh);
+                    else
+                        for (int pn = 0; pn < C::kPanels; ++pn)
+                            tma_load_3d(dst + pn * C::kPanelBytes, kv ? &tmV : &tmK, &bar_full[slot],
+                                        pn * C::kPanelElems, j * 128, kvh);
                     ++issued;
                     if (++slot == C::kStages) {
                         slot = 0;
@@ -184,8 +195,10 @@ __global__ void __launch_bounds__(384, 1)
         // ------------------------------------------------------------ MMA issuer
         // (the whole warp runs this loop; one elected lane issues each MMA)
         {
-            const uint32_t idS = idesc_bf16_f32(128, 128, false, false);
-            const uint32_t idPV = idesc_bf16_f32(128, D, false, true);
+            // e4m3 is format code 0 of kind::f8f6f4; V^T makes both P.V operands K-major
+            constexpr uint32_t fmt = F8 ? 0u : Elt<T>::kMmaFmt;
+            const uint32_t idS = idesc_f16kind(fmt, 128, 128, false, false);
+            const uint32_t idPV = idesc_f16kind(fmt, 128, D, false, !F8);
             const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
             const uint32_t tS[2] = {tmem, tmem + 128u};
             const uint32_t tO[2] = {tmem + 256u, tmem + 256u + (uint32_t)D};
@@ -207,20 +220,30 @@ __global__ void __launch_bounds__(384, 1)
                 const uint32_t ko = slot_off(2 * j);
                 const uint32_t qo = (uint32_t)(t * C::kTileBytes);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
+                for (int kk = 0; kk < C::kKSteps; ++kk) {
                     const uint32_t o = (uint32_t)((kk >> 2) * C::kPanelBytes + (kk & 3) * 32);
-                    mma_ss_w(tS[t], dQ_k + off(qo + o), dKV_k + off(ko + o), idS, kk > 0 ? 1u : 0u);
+                    mma_ss_k<F8>(tS[t], dQ_k + off(qo + o), dKV_k + off(ko + o), idS, kk > 0 ? 1u : 0u);
                 }
                 mma_commit_w(&bar_s[t]);
             };
             // keys 64*half .. 64*half+63 of block j (P columns 32*half .. 32*half+31)
             auto issue_PV = [&](int t, int j, int half) {
                 const uint32_t vo = slot_off(2 * j + 1);
+                if constexpr (F8) {
+                    // P: four e4m3 per column, 8 columns per 32 keys; V^T rows are 128 keys
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    const int kk = 4 * half + k4;
-                    mma_ts_w(tO[t], tS[t] + (uint32_t)(kk * 8), dKV_mn + off(vo + (uint32_t)(kk * 2048)), idPV,
-                           (j > 0 || kk > 0) ? 1u : 0u);
+                    for (int k2 = 0; k2 < 2; ++k2) {
+                        const int kk = 2 * half + k2;
+                        mma_ts_f8_w(tO[t], tS[t] + (uint32_t)(kk * 8), dKV_k + off(vo + (uint32_t)(kk * 32)),
+                                    idPV, (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                } else {
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const int kk = 4 * half + k4;
+                        mma_ts_w(tO[t], tS[t] + (uint32_t)(kk * 8), dKV_mn + off(vo + (uint32_t)(kk * 2048)),
+                                 idPV, (j > 0 || kk > 0) ? 1u : 0u);
+                    }
                 }
             };
 
@@ -347,7 +370,30 @@ __global__ void __launch_bounds__(384, 1)
             // four goes to the FMA-pipe exp2 instead (masked -inf scores always
             // take ex2.approx, which returns exactly 0 for them).
             const bool soft = !__any_sync(0xffffffffu, need_mask);
-            auto half_block = [&](int hf, auto use_poly) {
+            auto half_block_f8 = [&](int hf, auto use_poly) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const int e = 64 * hf + 4 * c;
+                    const float2 x0 = ffma2(make_float2(s[e], s[e + 1]), sl22, nm2);
+                    const float2 x1 = ffma2(make_float2(s[e + 2], s[e + 3]), sl22, nm2);
+                    const float2 p0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
+                    float2 p1;
+                    if (decltype(use_poly)::value && (c & 1) == 1)
+                        p1 = exp2_poly2(x1);
+                    else
+                        p1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+                    acc = fadd2(acc, fadd2(p0, p1));
+                    pk[c] = pack_e4m3x4(p0.x, p0.y, p1.x, p1.y);
+                }
+                tmem_st16(tS + (uint32_t)(16 * hf), pk);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&bar_p[2 * t + hf]);
+            };
+            auto half_block_16 = [&](int hf, auto use_poly) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
@@ -359,7 +405,7 @@ __global__ void __launch_bounds__(384, 1)
                     else
                         pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                     acc = fadd2(acc, pv);
-                    pk[c] = pack_bf16x2(pv.x, pv.y);
+                    pk[c] = Elt<T>::pack(pv.x, pv.y);
                 }
                 tmem_st32(tS + (uint32_t)(32 * hf), pk);
                 tmem_st_wait();
@@ -367,6 +413,12 @@ __global__ void __launch_bounds__(384, 1)
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&bar_p[2 * t + hf]);
+            };
+            auto half_block = [&](int hf, auto use_poly) {
+                if constexpr (F8)
+                    half_block_f8(hf, use_poly);
+                else
+                    half_block_16(hf, use_poly);
             };
             // P in two halves of 64 keys: the MMA warp starts P.V on the first
             // half while the second is still being exponentiated
@@ -388,18 +440,18 @@ __global__ void __launch_bounds__(384, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (ok) {
                 tc_fence_after();
-                const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+                const float inv_l = (l > 0.f) ? p.o_scale / l : 0.f;
 #pragma unroll 1
-                for (int c0 = 0; c0 < D; c0 += 32) {
+                for (int c0 = 0; c0 < p.d_io; c0 += 32) {
                     uint32_t o[32];
                     tmem_ld32(tO + (uint32_t)c0, o);
                     if (row_valid) {
                         uint32_t w[16];
 #pragma unroll
                         for (int c = 0; c < 16; ++c)
-                            w[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l,
+                            w[c] = Elt<T>::pack(__uint_as_float(o[2 * c]) * inv_l,
                                                __uint_as_float(o[2 * c + 1]) * inv_l);
-                        uint4* dst = reinterpret_cast<uint4*>(p.o + row * D + c0);
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(p.o) + row * p.d_io + c0);
 #pragma unroll
                         for (int c = 0; c < 4; ++c)
                             dst[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
@@ -410,9 +462,9 @@ __global__ void __launch_bounds__(384, 1)
             }
         } else if (nb == 0 && row_valid) {
             // no visible key for any row of this tile
-            uint4* dst = reinterpret_cast<uint4*>(p.o + row * D);
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(p.o) + row * p.d_io);
 #pragma unroll 1
-            for (int c = 0; c < D / 8; ++c)
+            for (int c = 0; c < p.d_io / 8; ++c)
                 dst[c] = make_uint4(0u, 0u, 0u, 0u);
             if (p.lse)
                 p.lse[row] = -INFINITY;

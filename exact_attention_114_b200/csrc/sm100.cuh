@@ -11,6 +11,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace fa {
 
@@ -236,6 +237,45 @@ __device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint6
         : "memory");
 }
 
+// kind::f8f6f4 with A and B both e4m3 (format code 0 in the instruction
+// descriptor), fp32 accumulate.  One instruction covers K = 32, which is 32
+// bytes of a row: the shared-memory descriptors step exactly as for kind::f16,
+// and an A operand in tensor memory holds four e4m3 values per 32-bit column.
+__device__ __forceinline__ void mma_ss_f8_w(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b32 l;\n\t"
+        "elect.sync l|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_ts_f8_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b32 l;\n\t"
+        "elect.sync l|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Both kinds behind one name: F8 selects kind::f8f6f4, else kind::f16.
+template <bool F8>
+__device__ __forceinline__ void mma_ss_k(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate)
+{
+    if constexpr (F8)
+        mma_ss_f8_w(d_tmem, adesc, bdesc, idesc, accumulate);
+    else
+        mma_ss_w(d_tmem, adesc, bdesc, idesc, accumulate);
+}
+
 __device__ __forceinline__ void mma_commit_w(uint64_t* bar)
 {
     asm volatile(
@@ -256,14 +296,20 @@ __device__ __forceinline__ bool mbar_wait_w(uint64_t* bar, uint32_t parity, vola
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
 }
 
-// Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B.
-//   bits [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format,
+// Instruction descriptor, kind::f16: fp32 accumulate, A and B of one 16-bit type
+// (fmt 1 = bf16, 0 = fp16).
+//   bits [4,6) D format (1 = f32), [7,10) A format, [10,13) B format,
 //   bit 15 A major (0 = K), bit 16 B major (0 = K, 1 = MN), [17,23) N >> 3,
 //   [24,29) M >> 4.
+__host__ __device__ constexpr uint32_t idesc_f16kind(uint32_t fmt, int M, int N, bool a_mn_major, bool b_mn_major)
+{
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+           ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major)
 {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
-           ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+    return idesc_f16kind(1u, M, N, a_mn_major, b_mn_major);
 }
 
 // Shared-memory matrix descriptor for the 128-byte swizzle layout.
@@ -468,6 +514,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Four fp32 values -> four e4m3 bytes (round to nearest even, saturating at
+// +-448), value k in byte k of the word.  cvt...e4m3x2 puts its first source
+// in the upper byte of the 16-bit result.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float p0, float p1, float p2, float p3)
+{
+    unsigned short lo, hi;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(p1), "f"(p0));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(p3), "f"(p2));
+    return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
 // Move registers between warpgroups of a block (all four warps of the
 // warpgroup execute it).  The per-thread counts of all warpgroups must add up
 // to no more than the block's registers at launch.
@@ -488,6 +545,42 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
+
+// ---------------------------------------------------------------------------
+// 16-bit element types: bf16 (default) and fp16
+// ---------------------------------------------------------------------------
+template <typename T>
+struct Elt;
+
+template <>
+struct Elt<__nv_bfloat16> {
+    static constexpr uint32_t kMmaFmt = 1u;   // instruction-descriptor A/B format
+    __device__ static __forceinline__ uint32_t pack(float lo, float hi)
+    {
+        __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&v);
+    }
+    __device__ static __forceinline__ float2 unpack(uint32_t w)
+    {
+        return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+    }
+    __device__ static __forceinline__ __nv_bfloat16 from_float(float x) { return __float2bfloat16_rn(x); }
+};
+
+template <>
+struct Elt<__half> {
+    static constexpr uint32_t kMmaFmt = 0u;
+    __device__ static __forceinline__ uint32_t pack(float lo, float hi)
+    {
+        __half2 v = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<uint32_t*>(&v);
+    }
+    __device__ static __forceinline__ float2 unpack(uint32_t w)
+    {
+        return __half22float2(*reinterpret_cast<const __half2*>(&w));
+    }
+    __device__ static __forceinline__ __half from_float(float x) { return __float2half_rn(x); }
+};
 
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }

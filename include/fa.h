@@ -17,9 +17,14 @@
  * --------------------------------
  *  - Tensors are dense, row-major, "BHSD": q, o, dout, dq are [B, Hq, Nq, d];
  *    k, v, dk, dv are [B, Hkv, Nk, d]; lse is [B, Hq, Nq].  q/k/v/o/dout/dq/dk/dv
- *    hold bf16, lse holds fp32 (natural log of the scaled scores).
+ *    hold bf16 (fp16 through the *_ex calls), lse holds fp32 (natural log of
+ *    the scaled scores).
  *  - Every tensor pointer is a DEVICE pointer, non-NULL and 16-byte aligned.
- *  - d is 64 or 128.  Hq must be a multiple of Hkv.  B, Hq, Hkv, Nq, Nk >= 1.
+ *  - d is 32, 64, 96 or 128 (page "AI infra 一层全看懂(五) Flash Attention",
+ *    §五, gives 64 to 128 as the usual head dimension; 32 and 96 run on the 64
+ *    and 128 kernels with the missing columns zero-filled on chip).  The
+ *    split-KV and paged calls take d = 128 only.  Hq must be a multiple of Hkv.
+ *    B, Hq, Hkv, Nq, Nk >= 1.
  *  - causal is 0 or 1.  With causal = 1, key j is visible to query i iff
  *    j <= i + (Nk - Nq) (the mask is aligned to the bottom-right corner; for
  *    Nq = Nk this is the usual lower triangle).  A query row that sees no key
@@ -57,6 +62,12 @@ typedef enum {
     FA_ERR_TIMEOUT = 5           /* a bounded device wait ran out */
 } fa_status_t;
 
+/* Element type of the 16-bit tensors (q, k, v, o, dout, dq, dk, dv). */
+typedef enum {
+    FA_DTYPE_BF16 = 0,
+    FA_DTYPE_FP16 = 1
+} fa_dtype_t;
+
 /* Version of this ABI (incremented on any signature change). */
 int fa_abi_version(void);
 
@@ -80,6 +91,43 @@ const char* fa_last_error_message(void);
 fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                    int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                    void* stream);
+
+/*
+ * fa_fwd for either 16-bit element type: q, k, v, o hold `dtype` elements
+ * (FA_DTYPE_BF16 is exactly fa_fwd).  Everything else as fa_fwd; an unknown
+ * dtype returns FA_ERR_INVALID_ARGUMENT.
+ */
+fa_status_t fa_fwd_ex(fa_dtype_t dtype, const void* q, const void* k, const void* v, void* o, float* lse,
+                      int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                      void* stream);
+
+/*
+ * Forward with e4m3 (FP8) inputs.  The pages list an FP8 path as the lower-
+ * precision trade-off of the Hopper-generation kernel that needs its error
+ * kept under control (page "FlashAttention：为什么少搬数据，反而算得更快",
+ * §07); they give no recipe, so this call takes the plainest one:
+ *   q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d]: one e4m3 byte per element (OCP FP8
+ *   E4M3: bias 7, no infinities), dense BHSD, read only.  The values are
+ *   code * descale_{q,k,v} (one fp32 scale per tensor, finite and > 0).
+ *   S = scale * (Q K^T) accumulates exactly in fp32; P = exp(S - m) is rounded
+ *   to e4m3 for the P.V product (fp32 accumulation); the row sum l uses the
+ *   fp32 P.  o [B,Hq,Nq,d] is bf16 (written); lse [B,Hq,Nq] fp32 (or NULL).
+ *   d must be 128 (else FA_ERR_UNSUPPORTED).  Masking and shapes as fa_fwd,
+ *   always on the tiled kernel.
+ *   workspace: device scratch of fa_fwd_fp8_workspace_size(B, Hkv, Nk, d)
+ *   bytes, 256-byte aligned, for V transposed to [B,Hkv,d,Nk rounded up to
+ *   16]; NULL makes the call allocate it stream-ordered.  A smaller one returns
+ *   FA_ERR_WORKSPACE with nothing launched.
+ * Error bound against exact attention of the dequantised inputs: |O - O_ref|
+ * <= sum_j err(p_ij) |v_j| / l_i per element, err(p) = max(p / 16, 2^-10) (the
+ * e4m3 rounding of P), plus fp32 and bf16 output rounding.
+ */
+size_t fa_fwd_fp8_workspace_size(int B, int Hkv, int Nk, int d);
+
+fa_status_t fa_fwd_fp8(const void* q, const void* k, const void* v, float descale_q, float descale_k,
+                       float descale_v, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk,
+                       int d, float scale, int causal, void* workspace, size_t workspace_bytes,
+                       void* stream);
 
 /*
  * Split-KV forward for the decode shape (§09: a single query position, scores
@@ -169,6 +217,16 @@ fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o,
                    const void* dout, const float* lse, void* dq, void* dk, void* dv,
                    int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_bwd for either 16-bit element type: q, k, v, o, dout, dq, dk, dv hold
+ * `dtype` elements (FA_DTYPE_BF16 is exactly fa_bwd).  The workspace size does
+ * not depend on the element type.
+ */
+fa_status_t fa_bwd_ex(fa_dtype_t dtype, const void* q, const void* k, const void* v, const void* o,
+                      const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                      int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Reads and clears the device status word of the current device.  Synchronises

@@ -57,7 +57,8 @@ def _fwd(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, Hq=2, Hkv=1, Nq=8, Nk=8,
     (dict(causal=2), fa.FA_ERR_INVALID_ARGUMENT),
     (dict(scale=float("nan")), fa.FA_ERR_INVALID_ARGUMENT),
     (dict(scale=0.0), fa.FA_ERR_INVALID_ARGUMENT),
-    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=80), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=48), fa.FA_ERR_UNSUPPORTED),
     (dict(d=256), fa.FA_ERR_UNSUPPORTED),
     (dict(d=0), fa.FA_ERR_INVALID_ARGUMENT),
     (dict(B=1 << 20, Hq=1 << 10, Hkv=1 << 10), fa.FA_ERR_UNSUPPORTED),
@@ -145,3 +146,49 @@ def test_paged_rejects_bad_arguments():
     assert call(Nq=5) == fa.FA_ERR_UNSUPPORTED      # 5 * 4 rows per kv head > 16
     assert call(splits=300) == fa.FA_ERR_INVALID_ARGUMENT
     assert fa.fa_fwd_paged_workspace_size(2, 8, 2, 1, 64, 4, 128, 2) > 0
+
+
+def test_dtype_codes_are_checked_first():
+    """fa_fwd_ex / fa_bwd_ex refuse a dtype code outside fa_dtype_t before any
+    other check, and accept both codes up to the pointer checks."""
+    L = fa.lib()
+    for bad in (-1, 2, 7):
+        st = L.fa_fwd_ex(bad, FAKE, FAKE, FAKE, FAKE, None, 1, 2, 1, 8, 8, 64, 0.1, 0, None)
+        assert st == fa.FA_ERR_INVALID_ARGUMENT
+        assert "dtype" in fa.last_error_message()
+        st = L.fa_bwd_ex(bad, *([FAKE] * 9), 1, 2, 1, 8, 8, 64, 0.1, 1, None, 0, None)
+        assert st == fa.FA_ERR_INVALID_ARGUMENT
+    for good in (fa.FA_DTYPE_BF16, fa.FA_DTYPE_FP16):
+        st = L.fa_fwd_ex(good, None, FAKE, FAKE, FAKE, None, 1, 2, 1, 8, 8, 64, 0.1, 0, None)
+        assert st == fa.FA_ERR_INVALID_ARGUMENT and "q" in fa.last_error_message()
+
+
+def test_padded_head_dims_share_the_kernel_workspace():
+    """d = 32 and 96 run on the 64 and 128 kernels, whose dQ accumulator rows
+    have the kernel width."""
+    ws = fa.fa_bwd_workspace_size
+    assert ws(1, 4, 2, 100, 100, 32) == ws(1, 4, 2, 100, 100, 64)
+    assert ws(1, 4, 2, 100, 100, 96) == ws(1, 4, 2, 100, 100, 128)
+    assert ws(1, 4, 2, 100, 100, 64) < ws(1, 4, 2, 100, 100, 128)
+
+
+def test_fp8_rejects_bad_arguments():
+    L = fa.lib()
+    base = dict(B=1, Hq=2, Hkv=1, Nq=8, Nk=8, d=128, scale=0.1, causal=1, ds=(0.5, 0.5, 0.5))
+
+    def call(q=FAKE, ws=None, ws_bytes=0, **over):
+        p = dict(base, **over)
+        return L.fa_fwd_fp8(q, FAKE, FAKE, *p["ds"], FAKE, None, p["B"], p["Hq"], p["Hkv"], p["Nq"],
+                            p["Nk"], p["d"], p["scale"], p["causal"], ws, ws_bytes, None)
+
+    assert call(q=None) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(d=64) == fa.FA_ERR_UNSUPPORTED
+    assert call(ds=(0.5, 0.0, 0.5)) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(ds=(0.5, 0.5, float("inf"))) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(ds=(1e30, 1e30, 1.0)) == fa.FA_ERR_INVALID_ARGUMENT   # scale * dq * dk overflows
+    need = fa.fa_fwd_fp8_workspace_size(1, 1, 8, 128)
+    assert need == 2048                     # 128 d rows x 16 padded keys
+    assert fa.fa_fwd_fp8_workspace_size(1, 1, 8, 64) == 0
+    assert call(ws=ctypes.c_void_p(0x100000), ws_bytes=need - 1) == fa.FA_ERR_WORKSPACE
+    assert call(ws=ctypes.c_void_p(0x100010), ws_bytes=need) == fa.FA_ERR_INVALID_ARGUMENT
+    assert fa.fa_fwd_fp8_workspace_size(2, 8, 8192, 128) == 2 * 8 * 128 * 8192
