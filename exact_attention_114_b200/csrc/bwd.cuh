@@ -517,7 +517,8 @@ __global__ void __launch_bounds__(384, 1)
             int h, qb;
             step_coords(it, h, qb);
             ok = mbar_wait(&bar_gdone[it & 1], (uint32_t)((it >> 1) & 1), abort_flag);
-            ok = __all_sync(0xffffffffu, ok);
+            // all four drain warps decide together: the named barriers below need all of them
+            ok = named_bar_and(2, 128, ok);
             if (!ok)
                 break;
             tc_fence_after();

@@ -307,7 +307,7 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_off + 128u * (uint32_t)t;
         const uint32_t tO = tmem + lane_off + 256u + (uint32_t)(D * t);
-        const int nb = nblk[t];
+        const int nb = t ? nblk[1] : nblk[0];
         const int qlim = qi + delta;
         const float sl2 = p.scale_log2;
         float m_ref = -INFINITY, l = 0.f;
