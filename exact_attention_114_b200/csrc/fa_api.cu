@@ -92,8 +92,8 @@ fa_status_t check_shape(int B, int Hq, int Hkv, int Nq, int Nk, int d, float sca
         set_error("problem too large for 32-bit row indices");
         return FA_ERR_UNSUPPORTED;
     }
-    if (d != 32 && d != 64 && d != 96 && d != 128) {
-        set_error("d=%d is not supported (32, 64, 96 or 128)", d);
+    if (d < 32 || d > 256 || d % 32 != 0) {
+        set_error("d=%d is not supported (a multiple of 32 up to 256)", d);
         return FA_ERR_UNSUPPORTED;
     }
     return FA_OK;
@@ -227,10 +227,10 @@ int sm_count()
 // ---------------------------------------------------------------------------
 // forward (tiled kernel)
 // ---------------------------------------------------------------------------
-// Kernel head dim for a head dim d of the tensors: 32 runs on the 64 kernels and
-// 96 on the 128 kernels, the missing columns being zero fill of the TMA boxes
-// (zero columns add nothing to Q K^T, and P V gives zero there, never stored).
-int kernel_d(int d) { return d <= 64 ? 64 : 128; }
+// Kernel head dim for a head dim d of the tensors (a multiple of 32): the next of
+// 64, 128, 256, the missing columns being zero fill of the TMA boxes (zero
+// columns add nothing to Q K^T, and P V gives zero there, never stored).
+int kernel_d(int d) { return d <= 64 ? 64 : d <= 128 ? 128 : 256; }
 
 template <int D, bool CAUSAL, typename T>
 fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
@@ -253,7 +253,7 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     p.Nq = Nq;
     p.Nk = Nk;
     p.G = Hq / Hkv;
-    p.n_pairs = (Nq + 255) / 256;
+    p.n_pairs = (Nq + 128 * C::kTiles - 1) / (128 * C::kTiles);
     p.d_io = d;
     p.scale_log2 = scale * kLog2e;
     p.o_scale = 1.f;
@@ -313,6 +313,9 @@ template <typename T>
 fa_status_t fwd_tiled_t(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                         int Nq, int Nk, int d, float scale, int causal, cudaStream_t s)
 {
+    if (kernel_d(d) == 256)
+        return causal ? launch_fwd<256, true, T>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, s)
+                      : launch_fwd<256, false, T>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, s);
     if (kernel_d(d) == 128)
         return causal ? launch_fwd<128, true, T>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, s)
                       : launch_fwd<128, false, T>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, s);
@@ -857,7 +860,7 @@ fa_status_t fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache
 
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d)
 {
-    if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || Hq % Hkv != 0 || d < 1)
+    if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || Hq % Hkv != 0 || d < 1 || d > 128)
         return 0;
     return bwd_plan(B, Hq, Nq, d).total;
 }
@@ -879,6 +882,10 @@ static fa_status_t bwd_entry(int dtype, const void* q, const void* k, const void
         return st;
     if ((st = check_shape(B, Hq, Hkv, Nq, Nk, d, scale, causal)) != FA_OK)
         return st;
+    if (d > 128) {
+        set_error("the backward takes d up to 128 (got %d)", d);
+        return FA_ERR_UNSUPPORTED;
+    }
     if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) {
         set_error("workspace is not 256-byte aligned");
         return FA_ERR_INVALID_ARGUMENT;

@@ -19,6 +19,10 @@
 //     one tile overlaps the MMAs of the other; warps 10-11 only complete the
 //     third warpgroup, which hands most of its registers to the softmax ones.
 //
+// At d = 256 the CTA holds one query tile (kTiles = 1): its O accumulator takes
+// 256 TMEM columns, so there is no room for a second tile's S and O; the second
+// softmax warpgroup then has no work, and the MMA order is S(0) | PV(j) S(j+1).
+//
 // Scores are kept in the log2 domain: x = s * scale * log2(e), p = 2^(x - m).
 // Rescaling is lazy: the reference max m moves (and U, l are multiplied by
 // 2^(m_old - m_new)) only when the block max exceeds it by more than
@@ -42,6 +46,7 @@ constexpr float kLn2 = 0.69314718055994530942f;
 // see fp8_vt_kernel; otherwise they are 16-bit (T).
 template <int D, bool F8 = false>
 struct FwdCfg {
+    static constexpr int kTiles = (D == 256) ? 1 : 2;    // 128-row query tiles per CTA
     static constexpr int kThreads = 384;
     // registers per thread after the split: 2 x 128 x 208 + 128 x 80 <= 384 x 168
     static constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 80;
@@ -51,14 +56,15 @@ struct FwdCfg {
     static constexpr int kPanels = D * kElt / 128;
     static constexpr int kPanelElems = 128 / kElt;
     static constexpr int kKSteps = D * kElt / 32;        // Q.K^T instructions (32 bytes of d each)
-    static constexpr int kStages = F8 ? 10 : (D == 128) ? 5 : 8;
+    static constexpr int kStages = F8 ? 10 : (D == 256) ? 2 : (D == 128) ? 5 : 8;
     static constexpr int kBarBytes = F8 ? 512 : 256;
     static constexpr int kOffQ = 0;
-    static constexpr int kOffKV = 2 * kTileBytes;
+    static constexpr int kOffKV = kTiles * kTileBytes;
     static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
     static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + barriers + alignment slack
     static constexpr uint32_t kTmemCols = 512;
     static_assert(!F8 || D == 128, "the e4m3 kernel is built for d = 128");
+    static_assert(kTiles == 2 || 128 + D <= (int)kTmemCols, "one tile: S and O must fit in TMEM");
 };
 
 __device__ __forceinline__ int fwd_blocks_for_tile(int qt, int Nq, int Nk, bool causal)
@@ -106,11 +112,11 @@ __global__ void __launch_bounds__(384, 1)
     const int bh = (int)(blockIdx.x % n_bh);
     const int b = bh / p.Hq, h = bh % p.Hq;
     const int kvh = b * p.Hkv + h / p.G;
-    const int q0 = pair * 256;
+    const int q0 = pair * 128 * C::kTiles;
     const int delta = p.Nk - p.Nq;
     int nblk[2];
     nblk[0] = fwd_blocks_for_tile(q0, p.Nq, p.Nk, CAUSAL);
-    nblk[1] = fwd_blocks_for_tile(q0 + 128, p.Nq, p.Nk, CAUSAL);
+    nblk[1] = (C::kTiles == 2) ? fwd_blocks_for_tile(q0 + 128, p.Nq, p.Nk, CAUSAL) : 0;
     const int n_iter = max(nblk[0], nblk[1]);
 
     if (threadIdx.x == 0) {
@@ -219,7 +225,8 @@ __global__ void __launch_bounds__(384, 1)
             auto issue_S = [&](int t, int j) {
                 const uint32_t ko = slot_off(2 * j);
                 const uint32_t qo = (uint32_t)(t * C::kTileBytes);
-#pragma unroll
+                constexpr int kUnrollS = C::kKSteps <= 8 ? C::kKSteps : 4;   // d = 256: fewer live descriptors
+#pragma unroll kUnrollS
                 for (int kk = 0; kk < C::kKSteps; ++kk) {
                     const uint32_t o = (uint32_t)((kk >> 2) * C::kPanelBytes + (kk & 3) * 32);
                     mma_ss_k<F8>(tS[t], dQ_k + off(qo + o), dKV_k + off(ko + o), idS, kk > 0 ? 1u : 0u);
@@ -433,7 +440,7 @@ __global__ void __launch_bounds__(384, 1)
         }
 
         // ---- epilogue: O = U / l (bf16), LSE = (m + log2 l) ln 2
-        const bool row_valid = qi < p.Nq;
+        const bool row_valid = (C::kTiles == 2 || t == 0) && qi < p.Nq;   // one-tile CTAs: warps 4-7 idle
         const size_t row = (size_t)bh * (size_t)p.Nq + (size_t)qi;
         if (nb > 0 && ok) {
             ok = mbar_wait(&bar_o[t], 0, abort_flag);

@@ -20,11 +20,12 @@
  *    hold bf16 (fp16 through the *_ex calls), lse holds fp32 (natural log of
  *    the scaled scores).
  *  - Every tensor pointer is a DEVICE pointer, non-NULL and 16-byte aligned.
- *  - d is 32, 64, 96 or 128 (page "AI infra 一层全看懂(五) Flash Attention",
- *    §五, gives 64 to 128 as the usual head dimension; 32 and 96 run on the 64
- *    and 128 kernels with the missing columns zero-filled on chip).  The
- *    split-KV and paged calls take d = 128 only.  Hq must be a multiple of Hkv.
- *    B, Hq, Hkv, Nq, Nk >= 1.
+ *  - d is a multiple of 32 up to 256 for the forward and up to 128 for the
+ *    backward (page "AI infra 一层全看懂(五) Flash Attention", §五, gives 64 to
+ *    128 as the usual head dimension; other sizes run on the 64, 128 or 256
+ *    kernels with the missing columns zero-filled on chip; d > 128 uses one
+ *    128-row query tile per CTA).  The split-KV, paged and e4m3 calls take
+ *    d = 128 only.  Hq must be a multiple of Hkv.  B, Hq, Hkv, Nq, Nk >= 1.
  *  - causal is 0 or 1.  With causal = 1, key j is visible to query i iff
  *    j <= i + (Nk - Nq) (the mask is aligned to the bottom-right corner; for
  *    Nq = Nk this is the usual lower triangle).  A query row that sees no key

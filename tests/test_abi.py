@@ -59,7 +59,8 @@ def _fwd(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, Hq=2, Hkv=1, Nq=8, Nk=8,
     (dict(scale=0.0), fa.FA_ERR_INVALID_ARGUMENT),
     (dict(d=80), fa.FA_ERR_UNSUPPORTED),
     (dict(d=48), fa.FA_ERR_UNSUPPORTED),
-    (dict(d=256), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=16), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=288), fa.FA_ERR_UNSUPPORTED),
     (dict(d=0), fa.FA_ERR_INVALID_ARGUMENT),
     (dict(B=1 << 20, Hq=1 << 10, Hkv=1 << 10), fa.FA_ERR_UNSUPPORTED),
 ])
@@ -83,6 +84,8 @@ def test_bwd_rejects_bad_arguments():
         bad[i] = None
         assert call(bad) == fa.FA_ERR_INVALID_ARGUMENT
     assert call(args, d=80) == fa.FA_ERR_UNSUPPORTED
+    assert call(args, d=256) == fa.FA_ERR_UNSUPPORTED    # forward only at d > 128
+    assert fa.fa_bwd_workspace_size(1, 2, 1, 8, 8, 256) == 0
     # a workspace that is too small is refused before any launch
     need = fa.fa_bwd_workspace_size(1, 2, 1, 8, 8, 128)
     assert call(args, ws=ctypes.c_void_p(0x100000), ws_bytes=need - 1) == fa.FA_ERR_WORKSPACE

@@ -1,6 +1,7 @@
-"""GPU parity for head dims 32 and 96 (run on the 64 and 128 kernels with the
-missing columns zero-filled by TMA) against the oracle: forward and backward,
-tails around the tiles, GQA, causal and not."""
+"""GPU parity for head dims other than 64 and 128 against the oracle: 32 and 96
+(on the 64 and 128 kernels with the missing columns zero-filled by TMA; forward
+and backward) and 160 .. 256 (the one-tile forward kernel; the backward takes
+d <= 128).  Tails around the tiles, GQA, causal and not."""
 import pytest
 import torch
 
@@ -51,3 +52,48 @@ def test_headdim_forward_backward(shape, dtype):
     G.assert_grad(G.f64(dq), rq, "dQ")
     G.assert_grad(G.f64(dk), rk, "dK")
     G.assert_grad(G.f64(dv), rv, "dV")
+
+
+FWD_ONLY = [
+    # B, Hq, Hkv, Nq, Nk, d, causal
+    (1, 2, 1, 1, 1, 256, False),
+    (1, 2, 1, 63, 63, 256, True),
+    (2, 2, 1, 129, 129, 256, True),
+    (1, 4, 2, 300, 300, 256, True),
+    (1, 2, 2, 333, 200, 256, True),     # rows that see no key
+    (1, 2, 2, 200, 333, 256, False),
+    (1, 8, 1, 70, 640, 256, False),
+    (1, 4, 1, 257, 257, 192, True),
+    (1, 2, 2, 130, 130, 160, False),
+]
+
+
+@pytest.mark.parametrize("dtype", DTYPES, ids=["bf16", "fp16"])
+@pytest.mark.parametrize("shape", FWD_ONLY, ids=[str(s) for s in FWD_ONLY])
+def test_large_headdim_forward(shape, dtype):
+    B, Hq, Hkv, Nq, Nk, d, causal = shape
+    w = synth.Workload("headdim_fwd", B, Hq, Hkv, Nq, Nk, d, causal, 6400 + FWD_ONLY.index(shape))
+    x = synth.make_inputs(w, dtype=dtype, dout=False)
+    xd = {k: v.cuda() for k, v in x.items()}
+    o = torch.full_like(xd["q"], float("nan"))
+    o, lse = fa.fa_fwd(xd["q"], xd["k"], xd["v"], o=o, causal=causal)
+    torch.cuda.synchronize()
+    fa.fa_check_device_status()
+    xr = {k: v.double() for k, v in x.items()}
+    o_ref, lse_ref = oracle.fwd(xr["q"], xr["k"], xr["v"], w.scale, causal)
+    G.assert_o(G.f64(o), o_ref)
+    G.assert_lse(G.f64(lse), lse_ref)
+
+
+def test_large_headdim_sampled_long():
+    """d = 256, N = 4096 causal GQA: sampled rows of a multi-wave launch."""
+    w = synth.Workload("headdim_long", 1, 16, 4, 4096, 4096, 256, True, 6450)
+    x = synth.make_inputs(w, dout=False)
+    xd = {k: v.cuda() for k, v in x.items()}
+    o, lse = fa.fa_fwd(xd["q"], xd["k"], xd["v"], causal=True)
+    torch.cuda.synchronize()
+    fa.fa_check_device_status()
+    rows = G.sample_rows(w, n_random=24)
+    o_ref, lse_ref = oracle.fwd(x["q"], x["k"], x["v"], w.scale, True, rows=rows)
+    G.assert_o(G.f64(o).reshape(-1, w.d)[rows], o_ref)
+    G.assert_lse(G.f64(lse).reshape(-1)[rows], lse_ref)
