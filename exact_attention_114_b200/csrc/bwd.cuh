@@ -201,14 +201,19 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* bar_kv = bars;            // K, V landed
     uint64_t* bar_full = bars + 1;      // [kSlots] step slot landed
     uint64_t* bar_sdp = bars + 7;       // S^T and dP^T of a step in TMEM
-    uint64_t* bar_ds = bars + 8;        // P^T (TMEM), dS^T (smem) of a step written (count 4)
-    // [2] gradient MMAs of step `it` done (bar_gdone[it & 1]): dQ^T(it) is in TMEM,
-    // dS^T buffer (it & 1) and step slot (it % kSlots) are free again
-    uint64_t* bar_gdone = bars + 9;
-    uint64_t* bar_dqfree = bars + 12;   // dQ^T read out of TMEM (count 4)
-    uint64_t* bar_final = bars + 13;    // all MMAs done
-    uint64_t* bar_sdp_read = bars + 14; // S^T, dP^T of a step loaded into registers (count 4)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+    // A parity wait tells phase k from phase k + 2 apart only if the waiter can never be
+    // two phases behind.  The compute warps may finish step it + 1 before the MMA warp
+    // looks at step it, and the TMA warp waits for step it - 3's gradients while steps
+    // it - 2 and it - 1 run on: so bar_ds alternates between two barriers and bar_gdone
+    // between four, and no waiter is ever two phases behind on the barrier it waits on.
+    uint64_t* bar_ds = bars + 8;        // [2] P^T (TMEM), dS^T (smem) of step it written: [it & 1] (count 4)
+    // [4] gradient MMAs of step it done ([it & 3]): dQ^T(it) is in TMEM, the dS^T
+    // buffer (it & 1) and step slot (it % kSlots) are free again
+    uint64_t* bar_gdone = bars + 10;
+    uint64_t* bar_dqfree = bars + 14;   // dQ^T read out of TMEM (count 4)
+    uint64_t* bar_final = bars + 15;    // all MMAs done
+    uint64_t* bar_sdp_read = bars + 16; // S^T, dP^T of a step loaded into registers (count 4)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = warp_id(), lane = lane_id();
@@ -230,10 +235,11 @@ __global__ void __launch_bounds__(384, 1)
         for (int s = 0; s < C::kSlots; ++s)
             mbar_init(&bar_full[s], 1);
         mbar_init(bar_sdp, 1);
-        mbar_init(bar_ds, 4);
+        mbar_init(&bar_ds[0], 4);
+        mbar_init(&bar_ds[1], 4);
         mbar_init(bar_sdp_read, 4);
-        mbar_init(&bar_gdone[0], 1);
-        mbar_init(&bar_gdone[1], 1);
+        for (int i = 0; i < 4; ++i)
+            mbar_init(&bar_gdone[i], 1);
         mbar_init(bar_dqfree, 4);
         mbar_init(bar_final, 1);
         *abort_flag = 0;
@@ -279,7 +285,7 @@ __global__ void __launch_bounds__(384, 1)
                 // the slot was last used by step it - kSlots: wait for its gradient MMAs
                 if (it >= C::kSlots) {
                     const int prev = it - C::kSlots;
-                    if (!mbar_wait(&bar_gdone[prev & 1], (uint32_t)((prev >> 1) & 1), abort_flag))
+                    if (!mbar_wait(&bar_gdone[prev & 3], (uint32_t)((prev >> 2) & 1), abort_flag))
                         break;
                 }
                 int h, qb;
@@ -323,7 +329,6 @@ __global__ void __launch_bounds__(384, 1)
             const uint64_t dK_mn = sdesc_sw128(smem_u32(smem + C::kOffK), lbo_kt, 1024);
             const uint64_t dSlot_k = sdesc_sw128(smem_u32(smem + C::kOffSlots), 16, 1024);   // Q / dO K-major
             const uint64_t dSlot_mn = sdesc_sw128(smem_u32(smem + C::kOffSlots), C::kQPanel, 1024);
-            const uint64_t dDS_k = sdesc_sw128(smem_u32(smem + C::kOffDS), 16, 1024);
             const uint64_t dDS_mn = sdesc_sw128(smem_u32(smem + C::kOffDS), C::kPTile, 1024);
             auto off = [](uint32_t bytes) { return (uint64_t)(bytes >> 4); };
 
@@ -362,7 +367,7 @@ __global__ void __launch_bounds__(384, 1)
                         break;
                     issue_sdp(in);
                 }
-                if (!(ok = mbar_wait_w(bar_ds, (uint32_t)(it & 1), abort_flag)))
+                if (!(ok = mbar_wait_w(&bar_ds[it & 1], (uint32_t)((it >> 1) & 1), abort_flag)))
                     break;
                 tc_fence_after();
                 if (it > 0) {
@@ -378,13 +383,13 @@ __global__ void __launch_bounds__(384, 1)
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
                     mma_ts_w(tDV, tP + (uint32_t)(kk * 8), dSlot_mn + off(so + C::kQTile + kk * 2048), id_grad, acc);
-                    mma_ss_w(tDK, dDS_k + off(dso + kk * 32), dSlot_mn + off(so + kk * 2048), id_grad, acc);
+                    mma_ts_w(tDK, tP + 32u + (uint32_t)(kk * 8), dSlot_mn + off(so + kk * 2048), id_grad, acc);
                 }
                 // dQ^T = K^T dS^T   (K dimension = 128 keys)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ss_w(tDQ, dK_mn + off(kk * 2048), dDS_mn + off(dso + kk * 2048), id_dq, kk > 0 ? 1u : 0u);
-                mma_commit_w(&bar_gdone[it & 1]);
+                mma_commit_w(&bar_gdone[it & 3]);
             }
             mma_commit_w(bar_final);
             if (!ok)
@@ -447,7 +452,7 @@ __global__ void __launch_bounds__(384, 1)
             tmem_st32(tSb, pp);
             // dS^T into this step's buffer, free once the gradient MMAs of step it-2 are done
             if (it >= 2) {
-                ok = mbar_wait(&bar_gdone[it & 1], (uint32_t)((it >> 1) & 1) ^ 1u, abort_flag);
+                ok = mbar_wait(&bar_gdone[(it - 2) & 3], (uint32_t)(((it - 2) >> 2) & 1), abort_flag);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok)
                     break;
@@ -458,11 +463,14 @@ __global__ void __launch_bounds__(384, 1)
                 *reinterpret_cast<uint4*>(sDS + sw128_off(r, ch)) =
                     make_uint4(dd[4 * ch], dd[4 * ch + 1], dd[4 * ch + 2], dd[4 * ch + 3]);
             fence_proxy_async_smem();
+            // dS^T also over the other 32 S^T columns: the dK MMA reads it from there
+            // (A in TMEM), which takes its 16 KB per step off the shared-memory reads
+            tmem_st32(tSb + 32u, dd);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(bar_ds);
+                mbar_arrive(&bar_ds[it & 1]);
         }
         // ---- epilogue: dK = scale * acc, dV = acc  (bf16)
         if (ok) {
@@ -516,7 +524,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int it = 0; it < n_it; ++it) {
             int h, qb;
             step_coords(it, h, qb);
-            ok = mbar_wait(&bar_gdone[it & 1], (uint32_t)((it >> 1) & 1), abort_flag);
+            ok = mbar_wait(&bar_gdone[it & 3], (uint32_t)((it >> 2) & 1), abort_flag);
             // all four drain warps decide together: the named barriers below need all of them
             ok = named_bar_and(2, 128, ok);
             if (!ok)
