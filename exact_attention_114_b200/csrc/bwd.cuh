@@ -66,7 +66,8 @@ __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // ----------------------------------------------------------------------------
-// bwd_pre: D = rowsum(dO * O), LSE in log2 units, zero the dQ accumulator
+// bwd_pre: -D = -rowsum(dO * O), -LSE in log2 units (stored negated: the main
+// kernel adds them), zero the dQ accumulator
 // ----------------------------------------------------------------------------
 template <int D, typename T = __nv_bfloat16>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdParams p)
@@ -84,8 +85,8 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdParams p)
         acc[e] = 0.f;
     if (i >= p.Nq) {
         if (lane == 0) {
-            p.delta[row] = 0.f;
-            p.lse_log2[row] = INFINITY;
+            p.neg_delta[row] = 0.f;
+            p.neg_lse_log2[row] = -INFINITY;
         }
         return;
     }
@@ -115,9 +116,9 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdParams p)
     for (int off = 16; off > 0; off >>= 1)
         s += __shfl_xor_sync(0xffffffffu, s, off);
     if (lane == 0) {
-        p.delta[row] = s;
+        p.neg_delta[row] = -s;
         const float l = p.lse[(size_t)bh * p.Nq + i];
-        p.lse_log2[row] = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+        p.neg_lse_log2[row] = (l == -INFINITY) ? -INFINITY : -l * 1.4426950408889634f;
     }
 }
 
@@ -153,7 +154,7 @@ struct BwdCfg {
     static constexpr int kKTile = (D / 64) * kKPanel;  // K or V block
     static constexpr int kQPanel = 64 * 128;           // 64 rows x 64 bf16
     static constexpr int kQTile = (D / 64) * kQPanel;  // Q or dO block
-    static constexpr int kSlot = 2 * kQTile + 1024;    // Q, dO, lse_log2[64], delta[64] (1 KB-aligned)
+    static constexpr int kSlot = 2 * kQTile + 1024;    // Q, dO, -lse_log2[64], -delta[64] (1 KB-aligned)
     static constexpr int kSlots = 3;                   // step slots in flight (TMA latency cover)
     static constexpr int kPTile = 128 * 128;           // dS^T: 128 keys x 64 q bf16
     static constexpr int kOffK = 0;
@@ -298,8 +299,8 @@ __global__ void __launch_bounds__(384, 1)
                     tma_load_3d(slot + C::kQTile + pn * C::kQPanel, &tmDO, &bar_full[s], pn * 64, qb * 64, bh);
                 }
                 const size_t vrow = (size_t)bh * p.Nq_pad + (size_t)qb * 64;
-                bulk_load(slot + 2 * C::kQTile, p.lse_log2 + vrow, 256, &bar_full[s]);
-                bulk_load(slot + 2 * C::kQTile + 256, p.delta + vrow, 256, &bar_full[s]);
+                bulk_load(slot + 2 * C::kQTile, p.neg_lse_log2 + vrow, 256, &bar_full[s]);
+                bulk_load(slot + 2 * C::kQTile + 256, p.neg_delta + vrow, 256, &bar_full[s]);
                 ++issued;
             }
             if (*abort_flag) {
@@ -414,9 +415,11 @@ __global__ void __launch_bounds__(384, 1)
             if (!ok)
                 break;
             tc_fence_after();
-            const float* lse2 =
-                reinterpret_cast<const float*>(smem + C::kOffSlots + (it % C::kSlots) * C::kSlot + 2 * C::kQTile);
-            const float* dlt = lse2 + 64;
+            // -LSE * log2(e) and -D of the step's 64 query rows, read four at a time: each
+            // load is a broadcast, and 16-byte ones take a quarter of the shared-memory cycles
+            const float4* nlse4 = reinterpret_cast<const float4*>(
+                smem + C::kOffSlots + (it % C::kSlots) * C::kSlot + 2 * C::kQTile);
+            const float4* ndlt4 = nlse4 + 16;
             const uint32_t tSb = tS + (uint32_t)(64 * (it & 1));
             uint32_t sr[64], dr[64];
             tmem_ld64x2(tSb, tDP, sr, dr);
@@ -433,20 +436,26 @@ __global__ void __launch_bounds__(384, 1)
             // rows >= min_row see the key; whole 64-row block visible in most steps
             const bool all_vis = key_ok && (q_first >= min_row);
 #pragma unroll
-            for (int c = 0; c < 64; c += 2) {
-                const float2 nl = make_float2(-lse2[c], -lse2[c + 1]);
-                const float2 x = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl22, nl);
-                float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-                if (!all_vis) {
-                    pv.x = (key_ok && q_first + c >= min_row) ? pv.x : 0.f;
-                    pv.y = (key_ok && q_first + c + 1 >= min_row) ? pv.y : 0.f;
+            for (int c4 = 0; c4 < 16; ++c4) {
+                const float4 nl4 = nlse4[c4], nd4 = ndlt4[c4];
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int c = 4 * c4 + 2 * h2;
+                    const float2 nl = h2 ? make_float2(nl4.z, nl4.w) : make_float2(nl4.x, nl4.y);
+                    const float2 nd = h2 ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
+                    const float2 x =
+                        ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl22, nl);
+                    float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                    if (!all_vis) {
+                        pv.x = (key_ok && q_first + c >= min_row) ? pv.x : 0.f;
+                        pv.y = (key_ok && q_first + c + 1 >= min_row) ? pv.y : 0.f;
+                    }
+                    // dS = P * (dP - D)
+                    const float2 dd2 = fadd2(make_float2(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])), nd);
+                    const float2 ds2 = fmul2(pv, dd2);
+                    pp[c >> 1] = Elt<T>::pack(pv.x, pv.y);
+                    dd[c >> 1] = Elt<T>::pack(ds2.x, ds2.y);
                 }
-                // dS = P * (dP - D)
-                const float2 dd2 = fadd2(make_float2(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])),
-                                         make_float2(-dlt[c], -dlt[c + 1]));
-                const float2 ds2 = fmul2(pv, dd2);
-                pp[c >> 1] = Elt<T>::pack(pv.x, pv.y);
-                dd[c >> 1] = Elt<T>::pack(ds2.x, ds2.y);
             }
             // P^T over this step's S^T columns (the dV MMA reads it from there)
             tmem_st32(tSb, pp);

@@ -915,8 +915,8 @@ static fa_status_t bwd_entry(int dtype, const void* q, const void* k, const void
     p.dk = dk;
     p.dv = dv;
     char* w = static_cast<char*>(ws);
-    p.delta = reinterpret_cast<float*>(w + pl.delta_off);
-    p.lse_log2 = reinterpret_cast<float*>(w + pl.lse_off);
+    p.neg_delta = reinterpret_cast<float*>(w + pl.delta_off);
+    p.neg_lse_log2 = reinterpret_cast<float*>(w + pl.lse_off);
     p.dq_acc = reinterpret_cast<float*>(w + pl.acc_off);
     p.B = B;
     p.Hq = Hq;

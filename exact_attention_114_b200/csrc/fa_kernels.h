@@ -53,8 +53,8 @@ struct BwdParams {
     void* dq;                   // [B, Hq, Nq, d]
     void* dk;                   // [B, Hkv, Nk, d]
     void* dv;
-    float* delta;               // [B, Hq, Nq_pad]  D_i = rowsum(dout * o)
-    float* lse_log2;            // [B, Hq, Nq_pad]  LSE_i * log2(e) (+inf for masked rows)
+    float* neg_delta;           // [B, Hq, Nq_pad]  -D_i = -rowsum(dout * o)
+    float* neg_lse_log2;        // [B, Hq, Nq_pad]  -LSE_i * log2(e) (-inf for masked and padded rows)
     float* dq_acc;              // [B, Hq, Nq_pad, d] fp32 accumulator
     int B, Hq, Hkv, Nq, Nk;
     int G;
