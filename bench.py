@@ -204,6 +204,12 @@ def run_reference(args, rank, world):
 # ----------------------------------------------------------------------------
 # GPU arm
 # ----------------------------------------------------------------------------
+# DRAM bytes (read + write) of one bwd_main launch on this workload, from a one-pass
+# ncu capture of this bench command on the current kernel (dram__bytes_read.sum +
+# dram__bytes_write.sum); to be taken again whenever the kernel changes.
+BWD_MAIN_DRAM_BYTES = 666.12e6 + 333.94e6
+
+
 def run_libfa(args, rank, world, local):
     import torch
     import exact_attention_114_b200 as fa
@@ -472,7 +478,8 @@ def run_libfa(args, rank, world, local):
         "roofline": {"kernel": "fa_bwd (bwd_main dominant; pre/post included in the time)",
                      "bound": "tensor", "achieved": bwd_tf,
                      "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                     "frac": bwd_tf / peaks["bf16_tflops_sustained"], "traffic": None,
+                     "frac": bwd_tf / peaks["bf16_tflops_sustained"],
+                     "traffic": BWD_MAIN_DRAM_BYTES, "traffic_kernel": "bwd_main (one launch, ncu)",
                      "peak_source": peaks["source"] + " (sustained bf16 cuBLAS)"},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,

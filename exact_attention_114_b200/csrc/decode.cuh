@@ -82,11 +82,14 @@ __device__ __forceinline__ uint32_t dec_tile_off(int key, int chunk)
     return (uint32_t)(panel * DecCfg::kPanelBytes + key * 128 + ((c ^ (key & 7)) << 4));
 }
 
-template <bool PAGED, typename T = __nv_bfloat16>
-__global__ void __launch_bounds__(160)
+// NARROW: the head has fewer than 128 columns (p.d_io); the full-width kernel
+// compiles without the column checks.
+template <bool PAGED, typename T = __nv_bfloat16, bool NARROW = false>
+__global__ void __launch_bounds__(160, 2)   // two CTAs per SM (shared memory allows exactly two)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         DecodeParams p)
 {
+    const int d_io = NARROW ? p.d_io : 128;
     using C = DecCfg;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -126,7 +129,9 @@ __global__ void __launch_bounds__(160)
                     break;
                 uint8_t* dk = smem + C::kOffRing + slot * 2 * C::kTileBytes;
                 uint8_t* dv = dk + C::kTileBytes;
-                mbar_arrive_expect_tx(&bar_full[slot], 2 * C::kTileBytes);
+                // the second 64-column panel only when the head has columns there
+                const bool two = d_io > 64;
+                mbar_arrive_expect_tx(&bar_full[slot], (two ? 4 : 2) * C::kPanelBytes);
                 const int key0 = k_begin + t * C::kKeys;
                 if (PAGED) {
                     // a 64-key tile never straddles a page (page_size is a multiple of 64);
@@ -134,14 +139,18 @@ __global__ void __launch_bounds__(160)
                     const int page = __ldg(p.block_table + (size_t)b * p.max_pages + key0 / p.page_size);
                     const int off = key0 % p.page_size;
                     tma_load_4d(dk, &tmK, &bar_full[slot], 0, hk, off, page);
-                    tma_load_4d(dk + C::kPanelBytes, &tmK, &bar_full[slot], 64, hk, off, page);
                     tma_load_4d(dv, &tmV, &bar_full[slot], 0, hk, off, page);
-                    tma_load_4d(dv + C::kPanelBytes, &tmV, &bar_full[slot], 64, hk, off, page);
+                    if (two) {
+                        tma_load_4d(dk + C::kPanelBytes, &tmK, &bar_full[slot], 64, hk, off, page);
+                        tma_load_4d(dv + C::kPanelBytes, &tmV, &bar_full[slot], 64, hk, off, page);
+                    }
                 } else {
                     tma_load_3d(dk, &tmK, &bar_full[slot], 0, key0, kvh);
-                    tma_load_3d(dk + C::kPanelBytes, &tmK, &bar_full[slot], 64, key0, kvh);
                     tma_load_3d(dv, &tmV, &bar_full[slot], 0, key0, kvh);
-                    tma_load_3d(dv + C::kPanelBytes, &tmV, &bar_full[slot], 64, key0, kvh);
+                    if (two) {
+                        tma_load_3d(dk + C::kPanelBytes, &tmK, &bar_full[slot], 64, key0, kvh);
+                        tma_load_3d(dv + C::kPanelBytes, &tmV, &bar_full[slot], 64, key0, kvh);
+                    }
                 }
             }
             if (*abort_flag) {
@@ -169,8 +178,10 @@ __global__ void __launch_bounds__(160)
                 continue;
             const int h = hk * p.G + r / p.Nq, i = r % p.Nq;
             const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-                static_cast<const T*>(p.q) + (((size_t)b * p.Hq + h) * p.Nq + i) * 128);
+                static_cast<const T*>(p.q) + (((size_t)b * p.Hq + h) * p.Nq + i) * d_io);
             for (int ks = 0; ks < 8; ++ks) {
+                if (ks * 16 >= d_io)
+                    break;
                 qa[ks][hr] = __ldg(qrow + ks * 8 + tq);          // cols 16ks + 2tq, +1
                 qa[ks][hr + 2] = __ldg(qrow + ks * 8 + 4 + tq);  // cols 16ks + 8 + 2tq, +1
             }
@@ -208,6 +219,8 @@ __global__ void __launch_bounds__(160)
             const int key = key_w + (mi >> 1) * 8 + rr;
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
+                if (ks * 16 >= d_io)   // columns past the head: not loaded
+                    break;
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4(kbase + dec_tile_off(key, 2 * ks + (mi & 1)), b0, b1, b2, b3);
                 mma_16816<T>(s[0], qa[ks], b0, b1);
@@ -254,6 +267,8 @@ __global__ void __launch_bounds__(160)
             const int key = key_w + (mi & 1) * 8 + rr;
 #pragma unroll
             for (int nd = 0; nd < 16; nd += 2) {
+                if (nd * 8 >= d_io)   // output columns past the head stay zero
+                    break;
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4_t(vbase + dec_tile_off(key, nd + (mi >> 1)), b0, b1, b2, b3);
                 mma_16816<T>(o[nd], pa, b0, b1);
@@ -310,7 +325,8 @@ __global__ void __launch_bounds__(160)
         if (p.splits == 1) {
             const int h = hk * p.G + r / p.Nq, i = r % p.Nq;
             const size_t row = ((size_t)b * p.Hq + h) * p.Nq + i;
-            static_cast<T*>(p.o)[row * 128 + dcol] = Elt<T>::from_float(on);
+            if (dcol < d_io)
+                static_cast<T*>(p.o)[row * d_io + dcol] = Elt<T>::from_float(on);
             if (dcol == 0 && p.lse)
                 p.lse[row] = lse;
         } else {
@@ -362,7 +378,8 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(DecodeParams p)
     uint2 w2;
     w2.x = Elt<T>::pack(acc[0] * inv, acc[1] * inv);
     w2.y = Elt<T>::pack(acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<uint2*>(static_cast<T*>(p.o) + row * 128 + lane * 4) = w2;
+    if (lane * 4 < p.d_io)
+        *reinterpret_cast<uint2*>(static_cast<T*>(p.o) + row * p.d_io + lane * 4) = w2;
     if (lane == 0 && p.lse)
         p.lse[row] = (L > 0.f) ? M + __logf(L) : -INFINITY;
 }

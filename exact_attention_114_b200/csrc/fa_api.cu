@@ -336,7 +336,13 @@ fa_status_t fwd_tiled(int dtype, const void* q, const void* k, const void* v, vo
 constexpr int kDecodeMaxRows = 16;
 constexpr int kDecodeCtasPerSm = 2;
 
-bool decode_shape(int Hq, int Hkv, int Nq, int d) { return d == 128 && (long long)Nq * (Hq / Hkv) <= kDecodeMaxRows; }
+// The split-KV kernels work at width 128; narrower heads (32, 64, 96) leave the
+// rest of the tiles as TMA zero fill and skip it in the MMAs.
+constexpr int kDecodeWidth = 128;
+bool decode_shape(int Hq, int Hkv, int Nq, int d)
+{
+    return d <= kDecodeWidth && (long long)Nq * (Hq / Hkv) <= kDecodeMaxRows;
+}
 
 // Number of key chunks: the first count whose CTAs fill whole waves of the GPU
 // to 95% (at least 256 keys per chunk), else the best fill found.
@@ -378,7 +384,8 @@ DecodePlan decode_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, int reques
     pl.chunk = ((Nk + s - 1) / s + kt - 1) / kt * kt;
     pl.splits = (Nk + pl.chunk - 1) / pl.chunk;
     const size_t R = (size_t)Nq * (Hq / Hkv);
-    pl.o_bytes = (size_t)B * Hkv * pl.splits * R * d * sizeof(float);
+    pl.o_bytes = (size_t)B * Hkv * pl.splits * R * kDecodeWidth * sizeof(float);
+    (void)d;
     pl.lse_bytes = (size_t)B * Hkv * pl.splits * R * sizeof(float);
     return pl;
 }
@@ -404,7 +411,8 @@ fa_status_t launch_decode_t(const void* q, const void* k, const void* v, void* o
         if ((st = make_map(&mk, k, d, Nk, (uint64_t)B * Hkv, 64, tma_type<T>())) != FA_OK) return st;
         if ((st = make_map(&mv, v, d, Nk, (uint64_t)B * Hkv, 64, tma_type<T>())) != FA_OK) return st;
     }
-    auto kern = pg ? fa::decode_split_kernel<true, T> : fa::decode_split_kernel<false, T>;
+    auto kern = d < 128 ? (pg ? fa::decode_split_kernel<true, T, true> : fa::decode_split_kernel<false, T, true>)
+                        : (pg ? fa::decode_split_kernel<true, T, false> : fa::decode_split_kernel<false, T, false>);
     if ((st = ensure_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes)) != FA_OK) return st;
     fa::DecodeParams p;
     p.q = q;
@@ -424,6 +432,7 @@ fa_status_t launch_decode_t(const void* q, const void* k, const void* v, void* o
     p.splits = pl.splits;
     p.chunk = pl.chunk;
     p.causal = causal;
+    p.d_io = d;
     p.scale_log2 = scale * kLog2e;
     p.block_table = pg ? pg->block_table : nullptr;
     p.seq_lens = pg ? pg->seq_lens : nullptr;
@@ -715,7 +724,7 @@ fa_status_t fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o,
         return FA_ERR_INVALID_ARGUMENT;
     }
     if (!decode_shape(Hq, Hkv, Nq, d)) {
-        set_error("split-KV needs d = 128 and Nq * Hq / Hkv <= %d", kDecodeMaxRows);
+        set_error("split-KV needs d <= 128 and Nq * Hq / Hkv <= %d", kDecodeMaxRows);
         return FA_ERR_UNSUPPORTED;
     }
     if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) {
@@ -766,7 +775,7 @@ fa_status_t fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, 
         return FA_ERR_INVALID_ARGUMENT;
     }
     if (!decode_shape(Hq, Hkv, Nq, d)) {
-        set_error("split-KV needs d = 128 and Nq * Hq / Hkv <= %d", kDecodeMaxRows);
+        set_error("split-KV needs d <= 128 and Nq * Hq / Hkv <= %d", kDecodeMaxRows);
         return FA_ERR_UNSUPPORTED;
     }
     const DecodePlan pl = decode_plan(B, Hq, Hkv, Nq, Nk, d, num_splits);
@@ -826,7 +835,7 @@ fa_status_t fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache
         return FA_ERR_INVALID_ARGUMENT;
     }
     if (!decode_shape(Hq, Hkv, Nq, d)) {
-        set_error("paged decode needs d = 128 and Nq * Hq / Hkv <= %d", kDecodeMaxRows);
+        set_error("paged decode needs d <= 128 and Nq * Hq / Hkv <= %d", kDecodeMaxRows);
         return FA_ERR_UNSUPPORTED;
     }
     if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) {

@@ -33,6 +33,8 @@ struct DecodeParams {
     int splits;              // key chunks per (b, kv head)
     int chunk;               // keys per chunk (multiple of the key tile)
     int causal;
+    int d_io;                // head dim in memory (<= 128, multiple of 32): columns d_io..127 are zero
+                             // fill of the K/V tiles, zero in Q, skipped in the MMAs and never stored
     float scale_log2;
     // paged KV cache (decode_split_kernel<true>): K/V are [num_pages, page_size, Hkv, d];
     // the keys of sequence b are block_table[b][key / page_size] * page_size + key % page_size,

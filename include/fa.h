@@ -24,8 +24,9 @@
  *    backward (page "AI infra 一层全看懂(五) Flash Attention", §五, gives 64 to
  *    128 as the usual head dimension; other sizes run on the 64, 128 or 256
  *    kernels with the missing columns zero-filled on chip; d > 128 uses one
- *    128-row query tile per CTA).  The split-KV, paged and e4m3 calls take
- *    d = 128 only.  Hq must be a multiple of Hkv.  B, Hq, Hkv, Nq, Nk >= 1.
+ *    128-row query tile per CTA).  The split-KV and paged calls take d up to
+ *    128, the e4m3 call d = 128 only.  Hq must be a multiple of Hkv.
+ *    B, Hq, Hkv, Nq, Nk >= 1.
  *  - causal is 0 or 1.  With causal = 1, key j is visible to query i iff
  *    j <= i + (Nk - Nq) (the mask is aligned to the bottom-right corner; for
  *    Nq = Nk this is the usual lower triangle).  A query row that sees no key
@@ -137,7 +138,7 @@ fa_status_t fa_fwd_fp8(const void* q, const void* k, const void* v, float descal
  * Hq / Hkv query heads of the group, and a combine kernel merges them with the
  * rescale-and-add rule of §04 in log form:
  *     lse = ln sum_s exp(lse_s),   O = sum_s exp(lse_s - lse) O_s.
- *   Requires Nq * (Hq / Hkv) <= 16.
+ *   Requires Nq * (Hq / Hkv) <= 16 and d <= 128.
  *   num_splits: 0 picks a value from the shape; otherwise 1..256.
  *   workspace: device scratch of at least fa_fwd_splitkv_workspace_size(...)
  *   bytes, 256-byte aligned; NULL makes the call allocate it stream-ordered.
@@ -162,7 +163,7 @@ fa_status_t fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o,
  *   q, o: [B, Hq, Nq, d] bf16; lse [B, Hq, Nq] fp32 or NULL.  With causal = 1 the
  *     Nq query rows of sequence b are its last Nq positions (bottom-right mask
  *     against seq_lens[b]).
- *   page_size: a multiple of 64.  d = 128, Nq * Hq / Hkv <= 16.
+ *   page_size: a multiple of 64.  d <= 128, Nq * Hq / Hkv <= 16.
  *   num_splits / workspace as for fa_fwd_splitkv, sized with
  *   fa_fwd_paged_workspace_size().
  */

@@ -102,7 +102,7 @@ def test_splitkv_rejects_bad_arguments():
     assert call(splits=-1) == fa.FA_ERR_INVALID_ARGUMENT
     assert call(splits=257) == fa.FA_ERR_INVALID_ARGUMENT
     assert call(Nq=8) == fa.FA_ERR_UNSUPPORTED       # 8 * 4 rows per kv head > 16
-    assert call(d=64) == fa.FA_ERR_UNSUPPORTED
+    assert call(d=160) == fa.FA_ERR_UNSUPPORTED
     need = fa.fa_fwd_splitkv_workspace_size(2, 32, 8, 1, 4096, 128, 4)
     assert need > 0
     assert call(splits=4, ws=ctypes.c_void_p(0x100000), ws_bytes=need - 16) == fa.FA_ERR_WORKSPACE
@@ -145,7 +145,7 @@ def test_paged_rejects_bad_arguments():
     assert call(page_size=0) == fa.FA_ERR_INVALID_ARGUMENT
     assert call(num_pages=0) == fa.FA_ERR_INVALID_ARGUMENT
     assert call(max_pages=0) == fa.FA_ERR_INVALID_ARGUMENT
-    assert call(d=64) == fa.FA_ERR_UNSUPPORTED
+    assert call(d=160) == fa.FA_ERR_UNSUPPORTED
     assert call(Nq=5) == fa.FA_ERR_UNSUPPORTED      # 5 * 4 rows per kv head > 16
     assert call(splits=300) == fa.FA_ERR_INVALID_ARGUMENT
     assert fa.fa_fwd_paged_workspace_size(2, 8, 2, 1, 64, 4, 128, 2) > 0

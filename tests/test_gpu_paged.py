@@ -46,14 +46,14 @@ def gather(pool, table_row, L, page_size):
     return torch.stack(rows, 0).permute(1, 0, 2).unsqueeze(0).contiguous()
 
 
-def run_case(B, Hq, Hkv, Nq, page_size, seq_lens, causal, splits, seed):
-    q, kp, vp, table, lens = make_paged(B, Hq, Hkv, Nq, page_size, seq_lens, seed)
+def run_case(B, Hq, Hkv, Nq, page_size, seq_lens, causal, splits, seed, d=128):
+    q, kp, vp, table, lens = make_paged(B, Hq, Hkv, Nq, page_size, seq_lens, seed, d=d)
     dq, dk, dv = q.cuda(), kp.cuda(), vp.cuda()
     dt, dl = torch.from_numpy(table).cuda(), torch.from_numpy(lens).cuda()
     o, lse = fa.fa_fwd_paged(dq, dk, dv, dt, dl, causal=causal, num_splits=splits)
     torch.cuda.synchronize()
     fa.fa_check_device_status()
-    scale = 1.0 / np.sqrt(128)
+    scale = 1.0 / np.sqrt(d)
     for b, L in enumerate(seq_lens):
         og, lg = G.f64(o[b:b + 1]), G.f64(lse[b:b + 1])
         if L == 0:
@@ -100,3 +100,8 @@ def test_paged_matches_contiguous_cache():
                              num_splits=4)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("d", [32, 64, 96])
+def test_paged_decode_narrow_heads(d):
+    run_case(3, 8, 2, 2, 64, [1, 700, 2049], True, 0, 8300 + d, d=d)
