@@ -117,7 +117,8 @@ class ClockSampler:
                     sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
                     mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
                     rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
-                    self.samples.append((sm, mx, rs))
+                    mem = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_MEM)
+                    self.samples.append((sm, mx, rs, mem))
                 except Exception:
                     pass
                 self._stop.wait(self.period)
@@ -137,12 +138,13 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         import pynvml
         reasons = set()
-        for _, _, rs in self.samples:
+        for s_ in self.samples:
             for name, const in self.REASONS:
-                if rs & getattr(pynvml, const, 0):
+                if s_[2] & getattr(pynvml, const, 0):
                     reasons.add(name)
         return {"sm_mhz": statistics.median(x[0] for x in self.samples),
                 "sm_max_mhz": max(x[1] for x in self.samples), "reasons": sorted(reasons),
+                "mem_mhz": statistics.median(x[3] for x in self.samples),
                 "samples": len(self.samples)}
 
 
@@ -156,24 +158,34 @@ def oracle_sample_workload():
     return w.with_(B=1, Hq=w.G, Hkv=1, Nq=2048, Nk=2048)
 
 
-def time_oracle_step(w):
+def time_oracle_step(w, nthreads=0):
+    """Wall-clock seconds of the oracle's forward and backward on ``w``."""
     import oracle
     x = synth.make_inputs(w)
     t0 = time.perf_counter()
-    oracle.fwd(x["q"], x["k"], x["v"], w.scale, w.causal)
-    oracle.bwd(x["q"], x["k"], x["v"], x["dout"], w.scale, w.causal)
-    return time.perf_counter() - t0
+    oracle.fwd(x["q"], x["k"], x["v"], w.scale, w.causal, nthreads=nthreads)
+    t1 = time.perf_counter()
+    oracle.bwd(x["q"], x["k"], x["v"], x["dout"], w.scale, w.causal, nthreads=nthreads)
+    return t1 - t0, time.perf_counter() - t1
 
 
 def cpu_baseline_leg(reps=10):
     w = oracle_sample_workload()
-    dt = sum(time_oracle_step(w) for _ in range(reps)) / reps
+    times = [time_oracle_step(w) for _ in range(reps)]
+    t_fwd = sum(t[0] for t in times) / reps
+    t_bwd = sum(t[1] for t in times) / reps
     flops = w.fwd_flops() + w.bwd_flops()
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
+    # one thread on one (b, h) of the d = 64 MHA workload, for scaling context
+    w1 = synth.WORKLOADS["mha_1k"].with_(B=1, Hq=1, Hkv=1)
+    f1, b1 = time_oracle_step(w1, nthreads=1)
+    return {"value": flops / (t_fwd + t_bwd) / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
             "kind": "oracle",
             "sample": (f"fwd+bwd of one kv group (B=1, Hq=4, Hkv=1, N=2048, d=128, causal) "
                        f"of the {STEP_WORKLOAD} workload, {flops / 1e9:.1f} GFLOP by the FLOP "
-                       f"rule, mean of {reps} runs of {dt:.1f} s, fp64 oracle on all host cores")}
+                       f"rule, mean of {reps} runs of {t_fwd + t_bwd:.1f} s, fp64 oracle on all host cores"),
+            "fwd_gflops": w.fwd_flops() / t_fwd / 1e9, "bwd_gflops": w.bwd_flops() / t_bwd / 1e9,
+            "one_thread": {"sample": "one (b, h) of mha_1k (N=1024, d=64, causal)",
+                           "fwd_gflops": w1.fwd_flops() / f1 / 1e9, "bwd_gflops": w1.bwd_flops() / b1 / 1e9}}
 
 
 def run_reference(args, rank, world):
@@ -361,6 +373,39 @@ def run_libfa(args, rank, world, local):
     e2e_value = world * flops_step / (e2e_ms * 1e-3) / 1e12
     del bufs[1]
 
+    # ---- the other training-shape workloads, reported beside the step workload: the
+    # long MHA one (B=2, H=32, N=4096, d=128, causal, every 64th query row x8) held
+    # to the same bar, and the d = 64 MHA one (B=4, H=16, N=1024), causal and not
+    other = {}
+    for name in ("mha_4k_long", "mha_1k", "mha_1k_noncausal"):
+        wo = synth.WORKLOADS[name].with_(seed=rank_seed(synth.WORKLOADS[name].seed, rank))
+        xo = {k_: v_.to(dev) for k_, v_ in synth.make_inputs(wo).items()}
+        oo = torch.empty_like(xo["q"])
+        lo = torch.empty((wo.B, wo.Hq, wo.Nq), dtype=torch.float32, device=dev)
+        go = [torch.empty_like(xo[k_]) for k_ in ("q", "k", "v")]
+        wso = torch.empty(fa.fa_bwd_workspace_size(wo.B, wo.Hq, wo.Hkv, wo.Nq, wo.Nk, wo.d),
+                          dtype=torch.uint8, device=dev)
+
+        def fo():
+            fa.fa_fwd(xo["q"], xo["k"], xo["v"], oo, lo, causal=wo.causal, scale=wo.scale)
+
+        def bo():
+            fa.fa_bwd(xo["q"], xo["k"], xo["v"], oo, xo["dout"], lo, *go, causal=wo.causal,
+                      scale=wo.scale, workspace=wso)
+
+        for _ in range(3):
+            fo()
+            bo()
+        torch.cuda.synchronize()
+        f_ms = statistics.median(timed(fo, max(10, args.steps)))
+        b_ms = statistics.median(timed(bo, max(10, args.steps)))
+        other[name] = {"workload": f"B={wo.B}, H={wo.Hq}, N={wo.Nq}, d={wo.d}, "
+                                   f"{'causal' if wo.causal else 'non-causal'}",
+                       "fwd_ms": f_ms, "fwd_tflops": wo.fwd_flops() / (f_ms * 1e-3) / 1e12,
+                       "bwd_ms": b_ms, "bwd_tflops": wo.bwd_flops() / (b_ms * 1e-3) / 1e12}
+        del xo, oo, lo, go, wso
+    fa.fa_check_device_status()
+
     # ---- the same workload with fp16 inputs, and the e4m3 forward (kind::f8f6f4)
     x16 = {k: v.to(dev) for k, v in synth.make_inputs(w, dtype=torch.float16).items()}
     o16, dq16 = torch.empty_like(x16["q"]), torch.empty_like(x16["q"])
@@ -468,6 +513,7 @@ def run_libfa(args, rank, world, local):
                         "frac_of_peak": f8_tf / (2 * peaks["bf16_tflops"]),
                         "peak_source": "measured burst bf16 x 2 (nominal e4m3 / bf16 dense ratio)",
                         "includes": "V transpose kernel + forward kernel"},
+            **other,
             "decode": {"workload": f"{DECODE_WORKLOAD}: B=64, Hq=32, Hkv=8, Nq=1, Nk=8192, d=128",
                        "ms": dec_ms, "gbs": dec_gbs, "frac_of_hbm": dec_gbs / peaks["hbm_gbs"],
                        "algorithmic_bytes": dec_bytes},
@@ -488,6 +534,7 @@ def run_libfa(args, rank, world, local):
                 "serial_ms_per_step": e2e_serial_ms,
                 "serial_value": world * flops_step / (e2e_serial_ms * 1e-3) / 1e12},
         "gpu_launches": args.steps * 4,  # timed region: fwd (1) + bwd (pre, main, post) per step
+        "gpu_name": torch.cuda.get_device_name(dev),
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
