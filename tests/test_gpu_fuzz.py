@@ -16,7 +16,7 @@ from tests import gpu_parity as G
 pytestmark = pytest.mark.gpu
 
 
-def draw_cases(n=40, seed=20261202):
+def draw_cases(n=64, seed=20261202):
     rng = np.random.default_rng(seed)
     cases = []
     for i in range(n):
