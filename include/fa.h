@@ -43,8 +43,9 @@
  *    FA_ERR_TIMEOUT in a per-device status word and the kernel returns early;
  *    fa_check_device_status() reads and clears it.
  *  - Results are equal to the definition up to floating-point ordering, not
- *    bit for bit (§04: "equivalent results" are not bitwise identical); the
- *    dq accumulation uses atomics and is not run-to-run deterministic.
+ *    bit for bit (§04 calls the tiled result equivalent, not identical).  Every
+ *    output is bitwise repeatable from run to run except dq, which is added up
+ *    across key blocks by reductions in L2 whose order varies.
  */
 #ifndef LIBFA_FA_H
 #define LIBFA_FA_H
@@ -58,7 +59,7 @@ extern "C" {
 typedef enum {
     FA_OK = 0,
     FA_ERR_INVALID_ARGUMENT = 1, /* NULL / misaligned pointer, bad size or flag */
-    FA_ERR_UNSUPPORTED = 2,      /* valid but not implemented (e.g. d = 96) */
+    FA_ERR_UNSUPPORTED = 2,      /* valid but not implemented (e.g. d = 80, or d > 128 in the backward) */
     FA_ERR_WORKSPACE = 3,        /* workspace given but smaller than required */
     FA_ERR_CUDA = 4,             /* a CUDA runtime / driver call failed */
     FA_ERR_TIMEOUT = 5           /* a bounded device wait ran out */
@@ -151,7 +152,7 @@ fa_status_t fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o,
                            void* stream);
 
 /*
- * Decode over a paged KV cache (§09: paged KV management "orthogonal" to the
+ * Decode over a paged KV cache (§09: paged KV management is independent of the
  * attention computation -- it only decides where K and V are stored).
  *   k_cache, v_cache: [num_pages, page_size, Hkv, d] bf16, one pool shared by
  *     all sequences (heads innermost).
