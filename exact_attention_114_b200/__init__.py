@@ -81,6 +81,8 @@ def lib() -> ctypes.CDLL:
             L.fa_fwd_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, ip, ip, fl,
                                        ip, ip, vp, sz, vp]
             L.fa_fwd_paged.restype = ip
+            L.fa_fwd_paged_ex.argtypes = [ip] + list(L.fa_fwd_paged.argtypes)
+            L.fa_fwd_paged_ex.restype = ip
             L.fa_bwd_workspace_size.argtypes = [ip, ip, ip, ip, ip, ip]
             L.fa_bwd_workspace_size.restype = sz
             L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, fl, ip,
@@ -234,8 +236,9 @@ def fa_fwd_paged_workspace_size(B, Hq, Hkv, Nq, page_size, max_pages_per_seq, d,
 
 def fa_fwd_paged(q, k_cache, v_cache, block_table, seq_lens, o=None, lse=None, *, causal=False,
                  scale=None, num_splits=0, workspace=None, stream=None):
-    """Decode over a paged KV cache.  k_cache/v_cache [num_pages, page_size, Hkv, d] bf16,
-    block_table int32 [B, max_pages_per_seq], seq_lens int32 [B], q [B, Hq, Nq, d]."""
+    """Decode over a paged KV cache.  k_cache/v_cache [num_pages, page_size, Hkv, d] bf16 or
+    fp16 (the type of q), block_table int32 [B, max_pages_per_seq], seq_lens int32 [B],
+    q [B, Hq, Nq, d]."""
     import torch
     B, Hq, Nq, d = q.shape
     num_pages, page_size, Hkv, dk = k_cache.shape
@@ -251,10 +254,13 @@ def fa_fwd_paged(q, k_cache, v_cache, block_table, seq_lens, o=None, lse=None, *
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib().fa_fwd_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
-                              _ptr(seq_lens), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, d, page_size,
-                              num_pages, max_pages, scale, int(bool(causal)), int(num_splits),
-                              _ptr(workspace), ws_bytes, _stream(stream)))
+    dt = _dtype_code(q)
+    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache"), (o, "o")):
+        _require(t, n, q.dtype)
+    _check(lib().fa_fwd_paged_ex(dt, _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                 _ptr(seq_lens), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, d, page_size,
+                                 num_pages, max_pages, scale, int(bool(causal)), int(num_splits),
+                                 _ptr(workspace), ws_bytes, _stream(stream)))
     return o, lse
 
 

@@ -161,7 +161,7 @@ fa_status_t make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t 
 // 4-D map over a paged KV pool [pages][page_size][Hkv][d] (bf16), box {64, 1, 64, 1}
 // (one kv head, 64 keys of one page), 128-byte swizzle.
 fa_status_t make_map_paged(CUtensorMap* m, const void* base, uint64_t d, uint64_t Hkv, uint64_t page_size,
-                           uint64_t pages)
+                           uint64_t pages, CUtensorMapDataType dt)
 {
     EncodeTiledFn enc = get_encode();
     if (!enc) {
@@ -172,7 +172,7 @@ fa_status_t make_map_paged(CUtensorMap* m, const void* base, uint64_t d, uint64_
     cuuint64_t strides[3] = {d * 2, Hkv * d * 2, page_size * Hkv * d * 2};
     cuuint32_t box[4] = {64, 1, 64, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+    CUresult r = enc(m, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
@@ -405,8 +405,8 @@ fa_status_t launch_decode_t(const void* q, const void* k, const void* v, void* o
     CUtensorMap mk, mv;
     fa_status_t st;
     if (pg) {
-        if ((st = make_map_paged(&mk, k, d, Hkv, pg->page_size, pg->num_pages)) != FA_OK) return st;
-        if ((st = make_map_paged(&mv, v, d, Hkv, pg->page_size, pg->num_pages)) != FA_OK) return st;
+        if ((st = make_map_paged(&mk, k, d, Hkv, pg->page_size, pg->num_pages, tma_type<T>())) != FA_OK) return st;
+        if ((st = make_map_paged(&mv, v, d, Hkv, pg->page_size, pg->num_pages, tma_type<T>())) != FA_OK) return st;
     } else {
         if ((st = make_map(&mk, k, d, Nk, (uint64_t)B * Hkv, 64, tma_type<T>())) != FA_OK) return st;
         if ((st = make_map(&mv, v, d, Nk, (uint64_t)B * Hkv, 64, tma_type<T>())) != FA_OK) return st;
@@ -803,13 +803,18 @@ size_t fa_fwd_paged_workspace_size(int B, int Hq, int Hkv, int Nq, int page_size
     return decode_plan(B, Hq, Hkv, Nq, page_size * max_pages_per_seq, d, num_splits).total();
 }
 
-fa_status_t fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
-                         const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int d,
-                         int page_size, int num_pages, int max_pages_per_seq, float scale, int causal,
-                         int num_splits, void* workspace, size_t workspace_bytes, void* stream)
+static fa_status_t paged_entry(int dtype, const void* q, const void* k_cache, const void* v_cache,
+                               const int* block_table, const int* seq_lens, void* o, float* lse, int B, int Hq,
+                               int Hkv, int Nq, int d, int page_size, int num_pages, int max_pages_per_seq,
+                               float scale, int causal, int num_splits, void* workspace, size_t workspace_bytes,
+                               void* stream)
 {
     t_error.clear();
     fa_status_t st;
+    if (dtype != FA_DTYPE_BF16 && dtype != FA_DTYPE_FP16) {
+        set_error("dtype=%d is not FA_DTYPE_BF16 or FA_DTYPE_FP16", dtype);
+        return FA_ERR_INVALID_ARGUMENT;
+    }
     if ((st = check_ptr(q, "q")) || (st = check_ptr(k_cache, "k_cache")) || (st = check_ptr(v_cache, "v_cache")) ||
         (st = check_ptr(o, "o")))
         return st;
@@ -858,13 +863,35 @@ fa_status_t fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache
         }
     }
     PagedDesc pg{block_table, seq_lens, page_size, num_pages, max_pages_per_seq};
-    st = launch_decode(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Nq, max_len, d, scale, causal, pl, ws, s, &pg);
+    st = launch_decode(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Nq, max_len, d, scale, causal, pl, ws, s, &pg,
+                       dtype);
     if (owned) {
         cudaError_t e = cudaFreeAsync(ws, s);
         if (e != cudaSuccess && st == FA_OK)
             st = cuda_fail(e, "cudaFreeAsync");
     }
     return st;
+}
+
+fa_status_t fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                         const int* seq_lens, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int d,
+                         int page_size, int num_pages, int max_pages_per_seq, float scale, int causal,
+                         int num_splits, void* workspace, size_t workspace_bytes, void* stream)
+{
+    return paged_entry(FA_DTYPE_BF16, q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, Nq, d,
+                       page_size, num_pages, max_pages_per_seq, scale, causal, num_splits, workspace,
+                       workspace_bytes, stream);
+}
+
+fa_status_t fa_fwd_paged_ex(fa_dtype_t dtype, const void* q, const void* k_cache, const void* v_cache,
+                            const int* block_table, const int* seq_lens, void* o, float* lse, int B, int Hq,
+                            int Hkv, int Nq, int d, int page_size, int num_pages, int max_pages_per_seq,
+                            float scale, int causal, int num_splits, void* workspace, size_t workspace_bytes,
+                            void* stream)
+{
+    return paged_entry((int)dtype, q, k_cache, v_cache, block_table, seq_lens, o, lse, B, Hq, Hkv, Nq, d,
+                       page_size, num_pages, max_pages_per_seq, scale, causal, num_splits, workspace,
+                       workspace_bytes, stream);
 }
 
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d)

@@ -154,7 +154,8 @@ fa_status_t fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o,
 /*
  * Decode over a paged KV cache (§09: paged KV management is independent of the
  * attention computation -- it only decides where K and V are stored).
- *   k_cache, v_cache: [num_pages, page_size, Hkv, d] bf16, one pool shared by
+ *   k_cache, v_cache: [num_pages, page_size, Hkv, d] bf16 (fp16 through
+ *     fa_fwd_paged_ex), one pool shared by
  *     all sequences (heads innermost).
  *   block_table: int32 [B, max_pages_per_seq] (device); logical page n of
  *     sequence b is physical page block_table[b * max_pages_per_seq + n].
@@ -175,6 +176,17 @@ fa_status_t fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache
                          int B, int Hq, int Hkv, int Nq, int d, int page_size, int num_pages,
                          int max_pages_per_seq, float scale, int causal, int num_splits,
                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_fwd_paged for either 16-bit element type: q, o, k_cache and v_cache hold
+ * `dtype` elements (FA_DTYPE_BF16 is exactly fa_fwd_paged).  An unknown dtype
+ * returns FA_ERR_INVALID_ARGUMENT.
+ */
+fa_status_t fa_fwd_paged_ex(fa_dtype_t dtype, const void* q, const void* k_cache, const void* v_cache,
+                            const int* block_table, const int* seq_lens, void* o, float* lse,
+                            int B, int Hq, int Hkv, int Nq, int d, int page_size, int num_pages,
+                            int max_pages_per_seq, float scale, int causal, int num_splits,
+                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Split-KV forward that allocates nothing (the paper has no counterpart; this

@@ -15,7 +15,7 @@ from tests import gpu_parity as G
 pytestmark = pytest.mark.gpu
 
 
-def make_paged(B, Hq, Hkv, Nq, page_size, seq_lens, seed, extra_pages=3, d=128):
+def make_paged(B, Hq, Hkv, Nq, page_size, seq_lens, seed, extra_pages=3, d=128, fp16=False):
     rng = np.random.default_rng(seed)
     pages_per_seq = [max(1, -(-L // page_size)) for L in seq_lens]
     max_pages = max(pages_per_seq)
@@ -29,14 +29,15 @@ def make_paged(B, Hq, Hkv, Nq, page_size, seq_lens, seed, extra_pages=3, d=128):
         pos += n
     n_pool = num_pages * page_size * Hkv * d
 
-    def pool(tid):
-        bits = synth.normal_bf16_bits(seed, tid, n_pool)
-        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).reshape(
-            num_pages, page_size, Hkv, d)
+    def draw(tid, n, shape):
+        if fp16:
+            return torch.from_numpy(synth.normal_f32(seed, tid, n).astype(np.float16)).reshape(shape)
+        bits = synth.normal_bf16_bits(seed, tid, n)
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).reshape(shape)
 
-    k_pool, v_pool = pool(synth.TENSOR_K), pool(synth.TENSOR_V)
-    qbits = synth.normal_bf16_bits(seed, synth.TENSOR_Q, B * Hq * Nq * d)
-    q = torch.from_numpy(qbits.view(np.int16)).view(torch.bfloat16).reshape(B, Hq, Nq, d)
+    k_pool = draw(synth.TENSOR_K, n_pool, (num_pages, page_size, Hkv, d))
+    v_pool = draw(synth.TENSOR_V, n_pool, (num_pages, page_size, Hkv, d))
+    q = draw(synth.TENSOR_Q, B * Hq * Nq * d, (B, Hq, Nq, d))
     return q, k_pool, v_pool, table, np.array(seq_lens, np.int32)
 
 
@@ -46,8 +47,8 @@ def gather(pool, table_row, L, page_size):
     return torch.stack(rows, 0).permute(1, 0, 2).unsqueeze(0).contiguous()
 
 
-def run_case(B, Hq, Hkv, Nq, page_size, seq_lens, causal, splits, seed, d=128):
-    q, kp, vp, table, lens = make_paged(B, Hq, Hkv, Nq, page_size, seq_lens, seed, d=d)
+def run_case(B, Hq, Hkv, Nq, page_size, seq_lens, causal, splits, seed, d=128, fp16=False):
+    q, kp, vp, table, lens = make_paged(B, Hq, Hkv, Nq, page_size, seq_lens, seed, d=d, fp16=fp16)
     dq, dk, dv = q.cuda(), kp.cuda(), vp.cuda()
     dt, dl = torch.from_numpy(table).cuda(), torch.from_numpy(lens).cuda()
     o, lse = fa.fa_fwd_paged(dq, dk, dv, dt, dl, causal=causal, num_splits=splits)
@@ -105,3 +106,8 @@ def test_paged_matches_contiguous_cache():
 @pytest.mark.parametrize("d", [32, 64, 96])
 def test_paged_decode_narrow_heads(d):
     run_case(3, 8, 2, 2, 64, [1, 700, 2049], True, 0, 8300 + d, d=d)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_paged_decode_fp16(d):
+    run_case(2, 16, 4, 2, 128, [300, 4099], True, 0, 8400 + d, d=d, fp16=True)
