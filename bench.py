@@ -3,8 +3,16 @@
 
 One step = one training pass of attention over one batch of the GQA workload
 (B=1, Hq=32, Hkv=8, N=8192, d=128, causal): fa_fwd then fa_bwd, through the C
-ABI, inputs resident in HBM.  The decode workload (B=64, Hq=32, Hkv=8, Nq=1,
-Nk=8192) is timed in the same run and reported under "parts".
+ABI, inputs resident in HBM, L2 flushed before every timed call.  "value" is
+that step's TFLOP/s; "roofline" is fa_bwd (its bwd_main kernel is about 69% of
+the step) against the measured sustained bf16 peak; "e2e" is the same step
+with every step's inputs copied in from pinned host memory and its gradients
+copied out, double-buffered on three streams (the serial figure too).  Timed in
+the same run and reported under "parts": the step's forward and backward, the
+same workload in fp16 and (forward) in e4m3, the long-MHA and d = 64
+workloads, the decode workload (B=64, Hq=32, Hkv=8, Nq=1, Nk=8192) and the
+same decode over a paged cache.  "cpu_baseline" (rank 0, one GPU) times the
+fp64 oracle on a bounded sample on all host cores.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl libfa|reference]
 
