@@ -8,6 +8,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -232,6 +233,28 @@ int sm_count()
 // columns add nothing to Q K^T, and P V gives zero there, never stored).
 int kernel_d(int d) { return d <= 64 ? 64 : d <= 128 ? 128 : 256; }
 
+// The forward is persistent: one block per SM (its shared memory allows no
+// second), together working through the n_pairs * B * Hq tiles.
+unsigned fwd_grid(const fa::FwdParams& p)
+{
+    const long long tiles = (long long)p.n_pairs * p.B * p.Hq;
+    return (unsigned)std::max<long long>(1, std::min<long long>(tiles, sm_count()));
+}
+
+// The launch's tile counter: the next slot of fa::g_fwd_tile_ctr (zero between
+// launches: the kernel's last block resets it).  Slots rotate, so concurrent
+// launches on different streams get different ones.
+fa_status_t fwd_tile_counter(unsigned** ctr)
+{
+    static std::atomic<unsigned> seq{0};
+    void* base = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&base, fa::g_fwd_tile_ctr);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "tile counter address");
+    *ctr = static_cast<unsigned*>(base) + 2 * (seq.fetch_add(1u, std::memory_order_relaxed) % fa::kFwdCtrSlots);
+    return FA_OK;
+}
+
 template <int D, bool CAUSAL, typename T>
 fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                        int Nq, int Nk, int d, float scale, cudaStream_t stream)
@@ -257,8 +280,9 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     p.d_io = d;
     p.scale_log2 = scale * kLog2e;
     p.o_scale = 1.f;
-    const long long grid = (long long)p.n_pairs * B * Hq;
-    kern<<<(unsigned)grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
+    if ((st = fwd_tile_counter(&p.tile_ctr)) != FA_OK)
+        return st;
+    kern<<<fwd_grid(p), C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
     return check_launch("fwd_kernel launch");
 }
 
@@ -304,8 +328,9 @@ fa_status_t launch_fwd_fp8(const void* q, const void* k, const void* v, void* vt
     p.d_io = kF8D;
     p.scale_log2 = scale_log2;
     p.o_scale = o_scale;
-    const long long grid = (long long)p.n_pairs * B * Hq;
-    kern<<<(unsigned)grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
+    if ((st = fwd_tile_counter(&p.tile_ctr)) != FA_OK)
+        return st;
+    kern<<<fwd_grid(p), C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
     return check_launch("fwd_kernel (e4m3) launch");
 }
 

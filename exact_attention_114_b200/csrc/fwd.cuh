@@ -19,6 +19,16 @@
 //     one tile overlaps the MMAs of the other; warps 10-11 only complete the
 //     third warpgroup, which hands most of its registers to the softmax ones.
 //
+// The launch is persistent: one CTA per SM works through the (query tile pair,
+// batch, head) tiles, heaviest causal tiles first, each CTA claiming its next
+// tile from an atomic counter (fwd_tile).  The TMA warp claims it and hands it
+// to the other roles through a two-entry ring in shared memory.  TMEM,
+// barriers and the K/V ring carry over from tile to tile.  The producer reloads a
+// Q slot as soon as the tile's last Q.K^T has read it, and the MMA warp starts
+// the next tile's S while the softmax warps still write this tile's O.  The
+// start-up of a tile (Q load, first S) and its epilogue therefore overlap the
+// neighbouring tiles' work instead of leaving the tensor core idle.
+//
 // At d = 256 the CTA holds one query tile (kTiles = 1): its O accumulator takes
 // 256 TMEM columns, so there is no room for a second tile's S and O; the second
 // softmax warpgroup then has no work, and the MMA order is S(0) | PV(j) S(j+1).
@@ -48,8 +58,8 @@ template <int D, bool F8 = false>
 struct FwdCfg {
     static constexpr int kTiles = (D == 256) ? 1 : 2;    // 128-row query tiles per CTA
     static constexpr int kThreads = 384;
-    // registers per thread after the split: 2 x 128 x 208 + 128 x 80 <= 384 x 168
-    static constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 80;
+    // registers per thread after the split: 2 x 128 x 208 + 128 x 88 = 384 x 168
+    static constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 88;
     static constexpr int kElt = F8 ? 1 : 2;              // bytes per Q/K/V element
     static constexpr int kTileBytes = 128 * D * kElt;    // a 128-row Q or K tile, a V tile
     static constexpr int kPanelBytes = 128 * 128;        // 128 rows x 128 bytes (one swizzle span)
@@ -57,7 +67,7 @@ struct FwdCfg {
     static constexpr int kPanelElems = 128 / kElt;
     static constexpr int kKSteps = D * kElt / 32;        // Q.K^T instructions (32 bytes of d each)
     static constexpr int kStages = F8 ? 10 : (D == 256) ? 2 : (D == 128) ? 5 : 8;
-    static constexpr int kBarBytes = F8 ? 512 : 256;
+    static constexpr int kBarBytes = 512;
     static constexpr int kOffQ = 0;
     static constexpr int kOffKV = kTiles * kTileBytes;
     static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
@@ -81,6 +91,58 @@ __device__ __forceinline__ int fwd_blocks_for_tile(int qt, int Nq, int Nk, bool 
     return min(nkb, last_key / 128 + 1);
 }
 
+// Tile counters of the forward launches, two words per slot: tiles claimed
+// beyond each block's first, and blocks that have stopped claiming.  Each
+// launch takes the next slot (launches in flight on different streams do not
+// share one); the last block to stop claiming sets both words back to zero for
+// the slot's next launch, so a slot is zero whenever no launch is using it.
+constexpr int kFwdCtrSlots = 256;
+__device__ unsigned g_fwd_tile_ctr[kFwdCtrSlots][2];
+
+// One work tile: a pair of 128-row query tiles (one at d = 256) of one
+// (batch, head).  Tile i of the launch: pair n_pairs-1 - i / (B*Hq) (heaviest
+// causal pairs first), (batch, head) i % (B*Hq).
+struct FwdTile {
+    int bh;        // batch * Hq + head
+    int kvh;       // batch * Hkv + kv head
+    int q0;        // first query row
+    int nb0, nb1;  // 128-key blocks seen by query tile 0 / 1
+    int n_iter;    // max of the two
+};
+
+// The launch has at most one block per SM.  Block c starts with tile c; each
+// further tile is the next unclaimed one (the launch's tile counter), so like a
+// hardware block scheduler the blocks take the heavy causal tiles first and
+// whichever block is free takes the next.
+template <int kTiles, bool CAUSAL>
+__device__ __forceinline__ void fwd_tile(const FwdParams& p, int i, FwdTile& w)
+{
+    const int n_bh = p.B * p.Hq;
+    const int pair = p.n_pairs - 1 - i / n_bh;
+    w.bh = i % n_bh;
+    const int b = w.bh / p.Hq, h = w.bh % p.Hq;
+    w.kvh = b * p.Hkv + h / p.G;
+    w.q0 = pair * 128 * kTiles;
+    w.nb0 = fwd_blocks_for_tile(w.q0, p.Nq, p.Nk, CAUSAL);
+    w.nb1 = (kTiles == 2) ? fwd_blocks_for_tile(w.q0 + 128, p.Nq, p.Nk, CAUSAL) : 0;
+    w.n_iter = max(w.nb0, w.nb1);
+}
+
+// A consumer warp's read of the u-th tile index: wait until the producer has
+// published it, read it, and give the ring entry back (one arrival per warp).
+__device__ __forceinline__ int fwd_take_tile(uint64_t* bar_tfull, uint64_t* bar_tfree, volatile int* tile_ring,
+                                             int u, int lane, volatile int* abort_flag, bool& ok)
+{
+    ok = __all_sync(0xffffffffu, mbar_wait(&bar_tfull[u & 1], (uint32_t)(u >> 1) & 1u, abort_flag));
+    if (!ok)
+        return 0;
+    const int tile = tile_ring[u & 1];
+    __syncwarp();
+    if (lane == 0)
+        mbar_arrive(&bar_tfree[u & 1]);
+    return tile;
+}
+
 template <int D, bool CAUSAL, typename T = __nv_bfloat16, bool F8 = false>
 __global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -94,34 +156,32 @@ __global__ void __launch_bounds__(384, 1)
     uint8_t* sQ = smem + C::kOffQ;
     uint8_t* sKV = smem + C::kOffKV;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+    // Barrier phases run on across the tiles of the block: every role counts
+    // the completions it has waited for (Q loads per tile slot, K/V ring loads,
+    // blocks per tile slot, tiles per tile slot) and waits on their parity.
     uint64_t* bar_q = bars;                            // [2]  Q tile landed
-    uint64_t* bar_full = bar_q + 2;                    // [S]  ring slot landed
+    uint64_t* bar_qfree = bar_q + 2;                   // [2]  last Q.K^T of a tile done: Q slot reusable
+    uint64_t* bar_full = bar_qfree + 2;                // [S]  ring slot landed
     uint64_t* bar_empty = bar_full + C::kStages;       // [S]  ring slot released
     uint64_t* bar_s = bar_empty + C::kStages;          // [2]  S tile ready in TMEM
     uint64_t* bar_p = bar_s + 2;                       // [2][2] P half h (and O rescale) written
     uint64_t* bar_o = bar_p + 4;                       // [2]  last P.V of a tile done
     uint64_t* bar_drain = bar_o + 2;                   // [1]  MMA drain on abort
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
+    uint64_t* bar_tfull = bar_drain + 1;               // [2]  tile index published in tile_ring[u & 1]
+    uint64_t* bar_tfree = bar_tfull + 2;               // [2]  tile index read by the MMA and softmax warps
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tfree + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* tile_ring = abort_flag + 1;          // [2]  tile indices (>= n_tiles: no more)
+    static_assert((17 + 2 * C::kStages) * 8 + 16 <= C::kBarBytes, "barrier area too small");
+    const int n_tiles = p.n_pairs * p.B * p.Hq;
 
     const int warp = warp_id(), lane = lane_id();
-
-    // ---- work item: (query tile pair, batch, head); heaviest causal pairs first
-    const int n_bh = p.B * p.Hq;
-    const int pair = p.n_pairs - 1 - (int)(blockIdx.x / n_bh);
-    const int bh = (int)(blockIdx.x % n_bh);
-    const int b = bh / p.Hq, h = bh % p.Hq;
-    const int kvh = b * p.Hkv + h / p.G;
-    const int q0 = pair * 128 * C::kTiles;
     const int delta = p.Nk - p.Nq;
-    int nblk[2];
-    nblk[0] = fwd_blocks_for_tile(q0, p.Nq, p.Nk, CAUSAL);
-    nblk[1] = (C::kTiles == 2) ? fwd_blocks_for_tile(q0 + 128, p.Nq, p.Nk, CAUSAL) : 0;
-    const int n_iter = max(nblk[0], nblk[1]);
 
     if (threadIdx.x == 0) {
         for (int t = 0; t < 2; ++t) {
             mbar_init(&bar_q[t], 1);
+            mbar_init(&bar_qfree[t], 1);
             mbar_init(&bar_s[t], 1);
             mbar_init(&bar_p[2 * t], 4);
             mbar_init(&bar_p[2 * t + 1], 4);
@@ -132,6 +192,10 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(&bar_empty[s], 1);
         }
         mbar_init(bar_drain, 1);
+        for (int u = 0; u < 2; ++u) {
+            mbar_init(&bar_tfull[u], 1);
+            mbar_init(&bar_tfree[u], 9);   // the MMA warp and the eight softmax warps
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -148,6 +212,7 @@ __global__ void __launch_bounds__(384, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    FwdTile w;
 
     // Each role runs inside the branch that sets its register budget.
     if (warp >= 8) {
@@ -155,46 +220,76 @@ __global__ void __launch_bounds__(384, 1)
       if (warp == 8) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            for (int t = 0; t < 2; ++t) {
-                if (nblk[t] == 0)
-                    continue;
-                mbar_arrive_expect_tx(&bar_q[t], C::kTileBytes);
-                for (int pn = 0; pn < C::kPanels; ++pn)
-                    tma_load_3d(sQ + t * C::kTileBytes + pn * C::kPanelBytes, &tmQ, &bar_q[t],
-                                pn * C::kPanelElems, q0 + 128 * t, bh);
-            }
-            int slot = 0;
-            uint32_t round = 0;
-            int issued = 0;
-            for (int j = 0; j < n_iter; ++j) {
-                bool ok = true;
-                for (int kv = 0; kv < 2; ++kv) {
-                    if (!mbar_wait(&bar_empty[slot], (round & 1u) ^ 1u, abort_flag)) {
-                        ok = false;
+            int nq0 = 0, nq1 = 0;   // Q loads so far into tile slot 0 / 1
+            int kvi = 0;            // K/V ring loads so far
+            bool ok = true;
+            int tile = (int)blockIdx.x;
+            for (int u = 0; ok; ++u) {
+                // publish the tile to the other roles (a ring of two entries)
+                if (!(ok = mbar_wait(&bar_tfree[u & 1], ((uint32_t)(u >> 1) & 1u) ^ 1u, abort_flag)))
+                    break;
+                tile_ring[u & 1] = tile;
+                mbar_arrive(&bar_tfull[u & 1]);
+                if (tile >= n_tiles)
+                    break;
+                fwd_tile<C::kTiles, CAUSAL>(p, tile, w);
+                for (int t = 0; t < 2 && ok; ++t) {
+                    if ((t ? w.nb1 : w.nb0) == 0)
+                        continue;
+                    const int nq = t ? nq1 : nq0;
+                    // the slot still holds the previous tile's Q until its last Q.K^T is done
+                    if (nq > 0 && !(ok = mbar_wait(&bar_qfree[t], (uint32_t)((nq - 1) & 1), abort_flag)))
                         break;
-                    }
-                    uint8_t* dst = sKV + slot * C::kTileBytes;
-                    mbar_arrive_expect_tx(&bar_full[slot], C::kTileBytes);
-                    if (F8 && kv)   // V^T: d rows of keys j*128 .. j*128+127
-                        tma_load_3d(dst, &tmV, &bar_full[slot], j * 128, 0, kvh);
+                    mbar_arrive_expect_tx(&bar_q[t], C::kTileBytes);
+                    for (int pn = 0; pn < C::kPanels; ++pn)
+                        tma_load_3d(sQ + t * C::kTileBytes + pn * C::kPanelBytes, &tmQ, &bar_q[t],
+                                    pn * C::kPanelElems, w.q0 + 128 * t, w.bh);
+                    if (t)
+                        ++nq1;
                     else
-                        for (int pn = 0; pn < C::kPanels; ++pn)
-                            tma_load_3d(dst + pn * C::kPanelBytes, kv ? &tmV : &tmK, &bar_full[slot],
-                                        pn * C::kPanelElems, j * 128, kvh);
-                    ++issued;
-                    if (++slot == C::kStages) {
-                        slot = 0;
-                        ++round;
+                        ++nq0;
+                }
+                for (int j = 0; ok && j < w.n_iter; ++j) {
+                    for (int kv = 0; kv < 2; ++kv) {
+                        const int slot = kvi % C::kStages;
+                        const uint32_t round = (uint32_t)(kvi / C::kStages);
+                        if (!(ok = mbar_wait(&bar_empty[slot], (round & 1u) ^ 1u, abort_flag)))
+                            break;
+                        uint8_t* dst = sKV + slot * C::kTileBytes;
+                        mbar_arrive_expect_tx(&bar_full[slot], C::kTileBytes);
+                        if (F8 && kv)   // V^T: d rows of keys j*128 .. j*128+127
+                            tma_load_3d(dst, &tmV, &bar_full[slot], j * 128, 0, w.kvh);
+                        else
+                            for (int pn = 0; pn < C::kPanels; ++pn)
+                                tma_load_3d(dst + pn * C::kPanelBytes, kv ? &tmV : &tmK, &bar_full[slot],
+                                            pn * C::kPanelElems, j * 128, w.kvh);
+                        ++kvi;
                     }
                 }
-                if (!ok)
-                    break;
+                // Claim the next tile once this one's loads are all issued, a couple of
+                // key blocks before its end: blocks claim in the order they run out of
+                // work (a block that claimed at its start would take a second tile
+                // before knowing whether its first is long), and the claim's latency
+                // hides behind the rest of the tile.
+                tile = (int)gridDim.x + (int)atomicAdd(p.tile_ctr, 1u);
+            }
+            // this block claims no more tiles; the last one to get here (finished or
+            // aborted) resets the launch's counter slot
+            __threadfence();
+            if (atomicAdd(p.tile_ctr + 1, 1u) == gridDim.x - 1) {
+                __threadfence();
+                atomicExch(p.tile_ctr, 0u);
+                atomicExch(p.tile_ctr + 1, 0u);
             }
             if (*abort_flag) {
-                // let the last load of every slot land before the block exits
-                for (int i = max(0, issued - C::kStages); i < issued; ++i)
+                // let the last load of every slot and of both Q slots land before the block exits
+                for (int i = max(0, kvi - C::kStages); i < kvi; ++i)
                     mbar_wait_limited(&bar_full[i % C::kStages], (uint32_t)(i / C::kStages) & 1u,
                                       FA_WAIT_LIMIT_CYCLES);
+                if (nq0 > 0)
+                    mbar_wait_limited(&bar_q[0], (uint32_t)((nq0 - 1) & 1), FA_WAIT_LIMIT_CYCLES);
+                if (nq1 > 0)
+                    mbar_wait_limited(&bar_q[1], (uint32_t)((nq1 - 1) & 1), FA_WAIT_LIMIT_CYCLES);
             }
         }
       } else if (warp == 9) {
@@ -206,13 +301,8 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t idS = idesc_f16kind(fmt, 128, 128, false, false);
             const uint32_t idPV = idesc_f16kind(fmt, 128, D, false, !F8);
             const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
-            const uint32_t tS[2] = {tmem, tmem + 128u};
-            const uint32_t tO[2] = {tmem + 256u, tmem + 256u + (uint32_t)D};
-            bool ok = true;
-            for (int t = 0; t < 2 && ok; ++t)
-                if (nblk[t] > 0)
-                    ok = mbar_wait_w(&bar_q[t], 0, abort_flag);
-            tc_fence_after();
+            auto tS = [&](int t) { return tmem + 128u * (uint32_t)t; };
+            auto tO = [&](int t) { return tmem + 256u + (uint32_t)(D * t); };
 
             // base descriptors; a byte offset `o` inside an operand is added as o >> 4
             // to the start-address field (addresses stay below 256 KB, no carry)
@@ -222,82 +312,112 @@ __global__ void __launch_bounds__(384, 1)
             auto off = [](uint32_t bytes) { return (uint64_t)(bytes >> 4); };
             auto slot_off = [&](int idx) { return (uint32_t)((idx % C::kStages) * C::kTileBytes); };
             auto phase = [&](int idx) { return (uint32_t)((idx / C::kStages) & 1); };
-            auto issue_S = [&](int t, int j) {
-                const uint32_t ko = slot_off(2 * j);
+            // S(t) = Q(t) K^T for the K block at ring index ik
+            auto issue_S = [&](int t, int ik) {
+                const uint32_t ko = slot_off(ik);
                 const uint32_t qo = (uint32_t)(t * C::kTileBytes);
-                constexpr int kUnrollS = C::kKSteps <= 8 ? C::kKSteps : 4;   // d = 256: fewer live descriptors
+                constexpr int kUnrollS = C::kKSteps <= 4 ? C::kKSteps : 4;   // fewer live descriptors
 #pragma unroll kUnrollS
                 for (int kk = 0; kk < C::kKSteps; ++kk) {
                     const uint32_t o = (uint32_t)((kk >> 2) * C::kPanelBytes + (kk & 3) * 32);
-                    mma_ss_k<F8>(tS[t], dQ_k + off(qo + o), dKV_k + off(ko + o), idS, kk > 0 ? 1u : 0u);
+                    mma_ss_k<F8>(tS(t), dQ_k + off(qo + o), dKV_k + off(ko + o), idS, kk > 0 ? 1u : 0u);
                 }
                 mma_commit_w(&bar_s[t]);
             };
-            // keys 64*half .. 64*half+63 of block j (P columns 32*half .. 32*half+31)
-            auto issue_PV = [&](int t, int j, int half) {
-                const uint32_t vo = slot_off(2 * j + 1);
+            // O(t) += P V for keys 64*half .. 64*half+63 of block j (P columns 32*half ..
+            // 32*half+31), V at ring index iv; block 0 of a tile overwrites O
+            auto issue_PV = [&](int t, int j, int iv, int half) {
+                const uint32_t vo = slot_off(iv);
                 if constexpr (F8) {
                     // P: four e4m3 per column, 8 columns per 32 keys; V^T rows are 128 keys
 #pragma unroll
                     for (int k2 = 0; k2 < 2; ++k2) {
                         const int kk = 2 * half + k2;
-                        mma_ts_f8_w(tO[t], tS[t] + (uint32_t)(kk * 8), dKV_k + off(vo + (uint32_t)(kk * 32)),
+                        mma_ts_f8_w(tO(t), tS(t) + (uint32_t)(kk * 8), dKV_k + off(vo + (uint32_t)(kk * 32)),
                                     idPV, (j > 0 || kk > 0) ? 1u : 0u);
                     }
                 } else {
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
                         const int kk = 4 * half + k4;
-                        mma_ts_w(tO[t], tS[t] + (uint32_t)(kk * 8), dKV_mn + off(vo + (uint32_t)(kk * 2048)),
+                        mma_ts_w(tO(t), tS(t) + (uint32_t)(kk * 8), dKV_mn + off(vo + (uint32_t)(kk * 2048)),
                                  idPV, (j > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
             };
 
-            if (ok && n_iter > 0) {
-                ok = mbar_wait_w(&bar_full[0], 0, abort_flag);
-                tc_fence_after();
-                if (ok) {
-                    for (int t = 0; t < 2; ++t)
-                        if (nblk[t] > 0)
-                            issue_S(t, 0);
-                    mma_commit_w(&bar_empty[0]);
-                }
-            }
-            for (int j = 0; ok && j < n_iter; ++j) {
-                const int iv = 2 * j + 1, ik = 2 * j + 2;
-                if (!(ok = mbar_wait_w(&bar_full[iv % C::kStages], phase(iv), abort_flag)))
+            bool ok = true;
+            // phase bits: 1 << t = parity of the Q loads of tile slot t waited for so far,
+            // 4 << t = parity of the blocks of slot t in earlier tiles (bar_p phases)
+            uint32_t ph = 0;
+            int kvi = 0;            // ring index of the tile's first K block
+            for (int u = 0; ok; ++u) {
+                const int tile = fwd_take_tile(bar_tfull, bar_tfree, tile_ring, u, lane, abort_flag, ok);
+                if (!ok || tile >= n_tiles)
                     break;
-                tc_fence_after();
-                bool k_ready = false;
+                fwd_tile<C::kTiles, CAUSAL>(p, tile, w);
                 for (int t = 0; t < 2 && ok; ++t) {
-                    if (j < nblk[t]) {
-                        for (int hf = 0; hf < 2 && ok; ++hf) {
-                            if (!(ok = mbar_wait_w(&bar_p[2 * t + hf], (uint32_t)(j & 1), abort_flag)))
-                                break;
-                            tc_fence_after();
-                            issue_PV(t, j, hf);
-                        }
-                        if (!ok)
-                            break;
-                        if (j == nblk[t] - 1)
-                            mma_commit_w(&bar_o[t]);
-                    }
-                    if (j + 1 < nblk[t]) {
-                        if (!k_ready) {
-                            if (!(ok = mbar_wait_w(&bar_full[ik % C::kStages], phase(ik), abort_flag)))
-                                break;
-                            tc_fence_after();
-                            k_ready = true;
-                        }
-                        issue_S(t, j + 1);
+                    if ((t ? w.nb1 : w.nb0) == 0)
+                        continue;
+                    ok = mbar_wait_w(&bar_q[t], (ph >> t) & 1u, abort_flag);
+                    ph ^= 1u << t;
+                }
+                tc_fence_after();
+                const int k0 = kvi;
+                if (ok && w.n_iter > 0) {
+                    ok = mbar_wait_w(&bar_full[k0 % C::kStages], phase(k0), abort_flag);
+                    tc_fence_after();
+                    if (ok) {
+                        for (int t = 0; t < 2; ++t)
+                            if ((t ? w.nb1 : w.nb0) > 0) {
+                                issue_S(t, k0);
+                                if ((t ? w.nb1 : w.nb0) == 1)
+                                    mma_commit_w(&bar_qfree[t]);
+                            }
+                        mma_commit_w(&bar_empty[k0 % C::kStages]);
                     }
                 }
-                if (!ok)
-                    break;
-                mma_commit_w(&bar_empty[iv % C::kStages]);
-                if (k_ready)
-                    mma_commit_w(&bar_empty[ik % C::kStages]);
+                for (int j = 0; ok && j < w.n_iter; ++j) {
+                    const int iv = k0 + 2 * j + 1, ik = k0 + 2 * j + 2;
+                    if (!(ok = mbar_wait_w(&bar_full[iv % C::kStages], phase(iv), abort_flag)))
+                        break;
+                    tc_fence_after();
+                    bool k_ready = false;
+                    for (int t = 0; t < 2 && ok; ++t) {
+                        const int nbt = t ? w.nb1 : w.nb0;
+                        if (j < nbt) {
+                            const uint32_t pp = ((ph >> (2 + t)) ^ (uint32_t)j) & 1u;
+                            for (int hf = 0; hf < 2 && ok; ++hf) {
+                                if (!(ok = mbar_wait_w(&bar_p[2 * t + hf], pp, abort_flag)))
+                                    break;
+                                tc_fence_after();
+                                issue_PV(t, j, iv, hf);
+                            }
+                            if (!ok)
+                                break;
+                            if (j == nbt - 1)
+                                mma_commit_w(&bar_o[t]);
+                        }
+                        if (j + 1 < nbt) {
+                            if (!k_ready) {
+                                if (!(ok = mbar_wait_w(&bar_full[ik % C::kStages], phase(ik), abort_flag)))
+                                    break;
+                                tc_fence_after();
+                                k_ready = true;
+                            }
+                            issue_S(t, ik);
+                            if (j + 2 == nbt)   // that was the tile's last Q(t).K^T
+                                mma_commit_w(&bar_qfree[t]);
+                        }
+                    }
+                    if (!ok)
+                        break;
+                    mma_commit_w(&bar_empty[iv % C::kStages]);
+                    if (k_ready)
+                        mma_commit_w(&bar_empty[ik % C::kStages]);
+                }
+                kvi = k0 + 2 * w.n_iter;
+                ph ^= (((uint32_t)w.nb0 & 1u) << 2) | (((uint32_t)w.nb1 & 1u) << 3);
             }
             if (!ok) {
                 mma_commit_w(bar_drain);
@@ -310,142 +430,155 @@ __global__ void __launch_bounds__(384, 1)
         // ------------------------------------------------------------ softmax
         const int t = warp >> 2;
         const int r = ((warp & 3) << 5) + lane;
-        const int qi = q0 + 128 * t + r;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_off + 128u * (uint32_t)t;
         const uint32_t tO = tmem + lane_off + 256u + (uint32_t)(D * t);
-        const int nb = t ? nblk[1] : nblk[0];
-        const int qlim = qi + delta;
         const float sl2 = p.scale_log2;
-        float m_ref = -INFINITY, l = 0.f;
+        int bt = 0;   // blocks of earlier tiles (bar_s phases)
+        int no = 0;   // earlier tiles with at least one block (bar_o phases)
         bool ok = true;
 
-        for (int j = 0; j < nb; ++j) {
-            ok = mbar_wait(&bar_s[t], (uint32_t)(j & 1), abort_flag);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok)
+        for (int u = 0; ok; ++u) {
+            const int tile = fwd_take_tile(bar_tfull, bar_tfree, tile_ring, u, lane, abort_flag, ok);
+            if (!ok || tile >= n_tiles)
                 break;
-            tc_fence_after();
-            uint32_t sr[128];
-            tmem_ld128(tS, sr);
-            float s[128];
-#pragma unroll
-            for (int c = 0; c < 128; ++c)
-                s[c] = __uint_as_float(sr[c]);
+            fwd_tile<C::kTiles, CAUSAL>(p, tile, w);
+            const int qi = w.q0 + 128 * t + r;
+            const int nb = t ? w.nb1 : w.nb0;
+            const int qlim = qi + delta;
+            float m_ref = -INFINITY, l = 0.f;
 
-            const int kb = j * 128;
-            const bool need_mask = (kb + 128 > p.Nk) || (CAUSAL && kb + 127 > qlim);
-            if (need_mask) {
-                const int lim = CAUSAL ? min(p.Nk - 1, qlim) : p.Nk - 1;
+            for (int j = 0; j < nb; ++j) {
+                ok = mbar_wait(&bar_s[t], (uint32_t)((bt + j) & 1), abort_flag);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok)
+                    break;
+                tc_fence_after();
+                uint32_t sr[128];
+                tmem_ld128(tS, sr);
+                float s[128];
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
-                    if (kb + c > lim)
-                        s[c] = -INFINITY;
-            }
-            // row max: two independent chains of three-input max
-            float mxa = fmaxf(s[0], s[1]), mxb = fmaxf(s[2], s[3]);
-#pragma unroll
-            for (int c = 4; c < 128; c += 4) {
-                mxa = fmax3(mxa, s[c], s[c + 1]);
-                mxb = fmax3(mxb, s[c + 2], s[c + 3]);
-            }
-            const float m_blk = fmaxf(mxa, mxb) * sl2;
-            float a = 1.f;
-            bool resc = false;
-            if (m_blk > m_ref + kRescaleLog2) {
-                a = ex2_approx(m_ref - m_blk);
-                resc = (j > 0);
-                m_ref = m_blk;
-                l *= a;
-            }
-            if (__any_sync(0xffffffffu, resc)) {
-#pragma unroll 1
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    uint32_t o[32];
-                    tmem_ld32(tO + (uint32_t)c0, o);
-#pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        o[c] = __float_as_uint(__uint_as_float(o[c]) * a);
-                    tmem_st32(tO + (uint32_t)c0, o);
-                }
-            }
-            const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-            const float2 sl22 = make_float2(sl2, sl2), nm2 = make_float2(neg_m, neg_m);
-            float2 acc = make_float2(0.f, 0.f);
-            // One exp2 per score: the MUFU unit would be as busy as the tensor
-            // core at d = 128, so in blocks without masked scores one pair in
-            // four goes to the FMA-pipe exp2 instead (masked -inf scores always
-            // take ex2.approx, which returns exactly 0 for them).
-            const bool soft = !__any_sync(0xffffffffu, need_mask);
-            auto half_block_f8 = [&](int hf, auto use_poly) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const int e = 64 * hf + 4 * c;
-                    const float2 x0 = ffma2(make_float2(s[e], s[e + 1]), sl22, nm2);
-                    const float2 x1 = ffma2(make_float2(s[e + 2], s[e + 3]), sl22, nm2);
-                    const float2 p0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
-                    float2 p1;
-                    if (decltype(use_poly)::value && (c & 1) == 1)
-                        p1 = exp2_poly2(x1);
-                    else
-                        p1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
-                    acc = fadd2(acc, fadd2(p0, p1));
-                    pk[c] = pack_e4m3x4(p0.x, p0.y, p1.x, p1.y);
-                }
-                tmem_st16(tS + (uint32_t)(16 * hf), pk);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&bar_p[2 * t + hf]);
-            };
-            auto half_block_16 = [&](int hf, auto use_poly) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const int e = 64 * hf + 2 * c;
-                    const float2 x = ffma2(make_float2(s[e], s[e + 1]), sl22, nm2);
-                    float2 pv;
-                    if (decltype(use_poly)::value && (c & 3) == 3)
-                        pv = exp2_poly2(x);
-                    else
-                        pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-                    acc = fadd2(acc, pv);
-                    pk[c] = Elt<T>::pack(pv.x, pv.y);
-                }
-                tmem_st32(tS + (uint32_t)(32 * hf), pk);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&bar_p[2 * t + hf]);
-            };
-            auto half_block = [&](int hf, auto use_poly) {
-                if constexpr (F8)
-                    half_block_f8(hf, use_poly);
-                else
-                    half_block_16(hf, use_poly);
-            };
-            // P in two halves of 64 keys: the MMA warp starts P.V on the first
-            // half while the second is still being exponentiated
-            if (soft) {
-                half_block(0, std::true_type{});
-                half_block(1, std::true_type{});
-            } else {
-                half_block(0, std::false_type{});
-                half_block(1, std::false_type{});
-            }
-            l += acc.x + acc.y;
-        }
+                    s[c] = __uint_as_float(sr[c]);
 
-        // ---- epilogue: O = U / l (bf16), LSE = (m + log2 l) ln 2
-        const bool row_valid = (C::kTiles == 2 || t == 0) && qi < p.Nq;   // one-tile CTAs: warps 4-7 idle
-        const size_t row = (size_t)bh * (size_t)p.Nq + (size_t)qi;
-        if (nb > 0 && ok) {
-            ok = mbar_wait(&bar_o[t], 0, abort_flag);
-            ok = __all_sync(0xffffffffu, ok);
-            if (ok) {
+                const int kb = j * 128;
+                const bool need_mask = (kb + 128 > p.Nk) || (CAUSAL && kb + 127 > qlim);
+                if (need_mask) {
+                    const int lim = CAUSAL ? min(p.Nk - 1, qlim) : p.Nk - 1;
+#pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if (kb + c > lim)
+                            s[c] = -INFINITY;
+                }
+                // row max: two independent chains of three-input max
+                float mxa = fmaxf(s[0], s[1]), mxb = fmaxf(s[2], s[3]);
+#pragma unroll
+                for (int c = 4; c < 128; c += 4) {
+                    mxa = fmax3(mxa, s[c], s[c + 1]);
+                    mxb = fmax3(mxb, s[c + 2], s[c + 3]);
+                }
+                const float m_blk = fmaxf(mxa, mxb) * sl2;
+                float a = 1.f;
+                bool resc = false;
+                if (m_blk > m_ref + kRescaleLog2) {
+                    a = ex2_approx(m_ref - m_blk);
+                    resc = (j > 0);
+                    m_ref = m_blk;
+                    l *= a;
+                }
+                if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + (uint32_t)c0, o);
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            o[c] = __float_as_uint(__uint_as_float(o[c]) * a);
+                        tmem_st32(tO + (uint32_t)c0, o);
+                    }
+                }
+                const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+                const float2 sl22 = make_float2(sl2, sl2), nm2 = make_float2(neg_m, neg_m);
+                float2 acc = make_float2(0.f, 0.f);
+                // One exp2 per score: the MUFU unit would be as busy as the tensor
+                // core at d = 128, so in blocks without masked scores one pair in
+                // four goes to the FMA-pipe exp2 instead (masked -inf scores always
+                // take ex2.approx, which returns exactly 0 for them).
+                const bool soft = !__any_sync(0xffffffffu, need_mask);
+                auto half_block_f8 = [&](int hf, auto use_poly) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const int e = 64 * hf + 4 * c;
+                        const float2 x0 = ffma2(make_float2(s[e], s[e + 1]), sl22, nm2);
+                        const float2 x1 = ffma2(make_float2(s[e + 2], s[e + 3]), sl22, nm2);
+                        const float2 p0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
+                        float2 p1;
+                        if (decltype(use_poly)::value && (c & 1) == 1)
+                            p1 = exp2_poly2(x1);
+                        else
+                            p1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+                        acc = fadd2(acc, fadd2(p0, p1));
+                        pk[c] = pack_e4m3x4(p0.x, p0.y, p1.x, p1.y);
+                    }
+                    tmem_st16(tS + (uint32_t)(16 * hf), pk);
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&bar_p[2 * t + hf]);
+                };
+                auto half_block_16 = [&](int hf, auto use_poly) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const int e = 64 * hf + 2 * c;
+                        const float2 x = ffma2(make_float2(s[e], s[e + 1]), sl22, nm2);
+                        float2 pv;
+                        if (decltype(use_poly)::value && (c & 3) == 3)
+                            pv = exp2_poly2(x);
+                        else
+                            pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                        acc = fadd2(acc, pv);
+                        pk[c] = Elt<T>::pack(pv.x, pv.y);
+                    }
+                    tmem_st32(tS + (uint32_t)(32 * hf), pk);
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&bar_p[2 * t + hf]);
+                };
+                auto half_block = [&](int hf, auto use_poly) {
+                    if constexpr (F8)
+                        half_block_f8(hf, use_poly);
+                    else
+                        half_block_16(hf, use_poly);
+                };
+                // P in two halves of 64 keys: the MMA warp starts P.V on the first
+                // half while the second is still being exponentiated
+                if (soft) {
+                    half_block(0, std::true_type{});
+                    half_block(1, std::true_type{});
+                } else {
+                    half_block(0, std::false_type{});
+                    half_block(1, std::false_type{});
+                }
+                l += acc.x + acc.y;
+            }
+
+            if (!ok)
+                break;
+
+            // ---- epilogue: O = U / l (bf16), LSE = (m + log2 l) ln 2
+            const bool row_valid = (C::kTiles == 2 || t == 0) && qi < p.Nq;   // one-tile blocks: warps 4-7 idle
+            const size_t row = (size_t)w.bh * (size_t)p.Nq + (size_t)qi;
+            if (nb > 0) {
+                ok = mbar_wait(&bar_o[t], (uint32_t)(no & 1), abort_flag);
+                ok = __all_sync(0xffffffffu, ok);
+                ++no;
+                if (!ok)
+                    break;
                 tc_fence_after();
                 const float inv_l = (l > 0.f) ? p.o_scale / l : 0.f;
 #pragma unroll 1
@@ -453,28 +586,32 @@ __global__ void __launch_bounds__(384, 1)
                     uint32_t o[32];
                     tmem_ld32(tO + (uint32_t)c0, o);
                     if (row_valid) {
-                        uint32_t w[16];
+                        uint32_t wv[16];
 #pragma unroll
                         for (int c = 0; c < 16; ++c)
-                            w[c] = Elt<T>::pack(__uint_as_float(o[2 * c]) * inv_l,
-                                               __uint_as_float(o[2 * c + 1]) * inv_l);
+                            wv[c] = Elt<T>::pack(__uint_as_float(o[2 * c]) * inv_l,
+                                                 __uint_as_float(o[2 * c + 1]) * inv_l);
                         uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(p.o) + row * p.d_io + c0);
 #pragma unroll
                         for (int c = 0; c < 4; ++c)
-                            dst[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                            dst[c] = make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
                     }
                 }
+                // O(t) is read out: the next tile's first P.V may overwrite it once this
+                // warpgroup's P of that tile is signalled (after the fence in the P write)
+                tc_fence_before();
                 if (row_valid && p.lse)
                     p.lse[row] = (l > 0.f) ? (m_ref + __log2f(l)) * kLn2 : -INFINITY;
-            }
-        } else if (nb == 0 && row_valid) {
-            // no visible key for any row of this tile
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(p.o) + row * p.d_io);
+            } else if (row_valid) {
+                // no visible key for any row of this tile
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(p.o) + row * p.d_io);
 #pragma unroll 1
-            for (int c = 0; c < p.d_io / 8; ++c)
-                dst[c] = make_uint4(0u, 0u, 0u, 0u);
-            if (p.lse)
-                p.lse[row] = -INFINITY;
+                for (int c = 0; c < p.d_io / 8; ++c)
+                    dst[c] = make_uint4(0u, 0u, 0u, 0u);
+                if (p.lse)
+                    p.lse[row] = -INFINITY;
+            }
+            bt += nb;
         }
     }
 
