@@ -72,73 +72,100 @@ __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_
 template <int D, typename T = __nv_bfloat16>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdParams p)
 {
-    const int row = (int)(blockIdx.x * 8 + (threadIdx.x >> 5));   // over B * Hq * Nq_pad
+    // one warp per two rows of B * Hq * Nq_pad (both rows' loads issued before
+    // either is reduced); lane l owns columns E*l .. E*l+E-1
+    constexpr int E = D / 32;   // elements per lane
     const int lane = threadIdx.x & 31;
     const int total = p.B * p.Hq * p.Nq_pad;
-    if (row >= total)
-        return;
-    const int bh = row / p.Nq_pad, i = row % p.Nq_pad;
-    constexpr int E = D / 32;   // elements per lane
-    float* acc = p.dq_acc + (size_t)row * D + lane * E;
-#pragma unroll
-    for (int e = 0; e < E; ++e)
-        acc[e] = 0.f;
-    if (i >= p.Nq) {
-        if (lane == 0) {
-            p.neg_delta[row] = 0.f;
-            p.neg_lse_log2[row] = -INFINITY;
-        }
-        return;
-    }
-    const size_t src = ((size_t)bh * p.Nq + i) * p.d_io + lane * E;
-    float s = 0.f;
+    const int row0 = (int)(blockIdx.x * 16 + (threadIdx.x >> 5) * 2);
     const T* po = static_cast<const T*>(p.o);
     const T* pd = static_cast<const T*>(p.dout);
-    if (lane * E >= p.d_io) {
-        // padded columns of a narrower head: nothing to read
-    } else if constexpr (E == 4) {
-        const uint2 a = *reinterpret_cast<const uint2*>(po + src);
-        const uint2 c = *reinterpret_cast<const uint2*>(pd + src);
-        const uint32_t aw[2] = {a.x, a.y}, cw[2] = {c.x, c.y};
+    float s[2] = {0.f, 0.f};
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const float2 x = Elt<T>::unpack(aw[e]), y = Elt<T>::unpack(cw[e]);
-            s = fmaf(x.x, y.x, s);
-            s = fmaf(x.y, y.y, s);
+    for (int r = 0; r < 2; ++r) {
+        const int row = row0 + r;
+        if (row >= total)
+            continue;
+        float* acc = p.dq_acc + (size_t)row * D + lane * E;
+        if constexpr (E == 4)
+            *reinterpret_cast<float4*>(acc) = make_float4(0.f, 0.f, 0.f, 0.f);
+        else
+            *reinterpret_cast<float2*>(acc) = make_float2(0.f, 0.f);
+        const int bh = row / p.Nq_pad, i = row - bh * p.Nq_pad;
+        if (i >= p.Nq || lane * E >= p.d_io)   // padded row, or padded columns of a narrower head
+            continue;
+        const size_t src = ((size_t)bh * p.Nq + i) * p.d_io + lane * E;
+        if constexpr (E == 4) {
+            const uint2 a = *reinterpret_cast<const uint2*>(po + src);
+            const uint2 c = *reinterpret_cast<const uint2*>(pd + src);
+            const float2 x0 = Elt<T>::unpack(a.x), y0 = Elt<T>::unpack(c.x);
+            const float2 x1 = Elt<T>::unpack(a.y), y1 = Elt<T>::unpack(c.y);
+            s[r] = fmaf(x0.x, y0.x, s[r]);
+            s[r] = fmaf(x0.y, y0.y, s[r]);
+            s[r] = fmaf(x1.x, y1.x, s[r]);
+            s[r] = fmaf(x1.y, y1.y, s[r]);
+        } else {
+            const float2 x = Elt<T>::unpack(*reinterpret_cast<const uint32_t*>(po + src));
+            const float2 y = Elt<T>::unpack(*reinterpret_cast<const uint32_t*>(pd + src));
+            s[r] = fmaf(x.x, y.x, s[r]);
+            s[r] = fmaf(x.y, y.y, s[r]);
         }
-    } else {
-        const float2 x = Elt<T>::unpack(*reinterpret_cast<const uint32_t*>(po + src));
-        const float2 y = Elt<T>::unpack(*reinterpret_cast<const uint32_t*>(pd + src));
-        s = fmaf(x.x, y.x, s);
-        s = fmaf(x.y, y.y, s);
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-        s += __shfl_xor_sync(0xffffffffu, s, off);
-    if (lane == 0) {
-        p.neg_delta[row] = -s;
-        const float l = p.lse[(size_t)bh * p.Nq + i];
-        p.neg_lse_log2[row] = (l == -INFINITY) ? -INFINITY : -l * 1.4426950408889634f;
+    for (int r = 0; r < 2; ++r) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            s[r] += __shfl_xor_sync(0xffffffffu, s[r], off);
+    }
+    if (lane < 2) {
+        const int row = row0 + lane;
+        if (row < total) {
+            const float sr = lane ? s[1] : s[0];
+            const int bh = row / p.Nq_pad, i = row - bh * p.Nq_pad;
+            if (i >= p.Nq) {
+                p.neg_delta[row] = 0.f;
+                p.neg_lse_log2[row] = -INFINITY;
+            } else {
+                p.neg_delta[row] = -sr;
+                const float l = p.lse[(size_t)bh * p.Nq + i];
+                p.neg_lse_log2[row] = (l == -INFINITY) ? -INFINITY : -l * 1.4426950408889634f;
+            }
+        }
     }
 }
 
 // ----------------------------------------------------------------------------
-// bwd_post: dQ = bf16(scale * accumulator)
+// bwd_post: dQ = 16-bit(scale * accumulator).  Grid (row chunks, batch * head):
+// one warp per two rows, lane l converting columns 4l .. 4l+3 (d <= 128), no
+// per-element index division.
 // ----------------------------------------------------------------------------
 template <int D, typename T = __nv_bfloat16>
 __global__ void __launch_bounds__(256) bwd_post_kernel(BwdParams p)
 {
-    const size_t n4 = (size_t)p.B * p.Hq * p.Nq * p.d_io / 4;
-    for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n4;
-         idx += (size_t)gridDim.x * blockDim.x) {
-        const size_t e = idx * 4;
-        const size_t row = e / p.d_io, c = e % p.d_io;
-        const size_t bh = row / p.Nq, i = row % p.Nq;
-        const float4 a = *reinterpret_cast<const float4*>(p.dq_acc + (bh * p.Nq_pad + i) * D + c);
-        uint2 w;
-        w.x = Elt<T>::pack(a.x * p.scale, a.y * p.scale);
-        w.y = Elt<T>::pack(a.z * p.scale, a.w * p.scale);
-        *reinterpret_cast<uint2*>(static_cast<T*>(p.dq) + e) = w;
+    const int lane = threadIdx.x & 31, c = lane * 4;
+    if (c >= p.d_io)
+        return;
+    const long long BH = (long long)p.B * p.Hq;
+    const int i_step = (int)gridDim.x * 16;
+    for (long long bh = blockIdx.y; bh < BH; bh += gridDim.y) {
+        const float* acc = p.dq_acc + bh * p.Nq_pad * D + c;
+        T* dq = static_cast<T*>(p.dq) + bh * p.Nq * p.d_io + c;
+        for (int i0 = (int)(blockIdx.x * 16 + (threadIdx.x >> 5) * 2); i0 < p.Nq; i0 += i_step) {
+            const bool two = i0 + 1 < p.Nq;
+            const float4 a0 = *reinterpret_cast<const float4*>(acc + (size_t)i0 * D);
+            float4 a1 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (two)
+                a1 = *reinterpret_cast<const float4*>(acc + (size_t)(i0 + 1) * D);
+            uint2 w;
+            w.x = Elt<T>::pack(a0.x * p.scale, a0.y * p.scale);
+            w.y = Elt<T>::pack(a0.z * p.scale, a0.w * p.scale);
+            *reinterpret_cast<uint2*>(dq + (size_t)i0 * p.d_io) = w;
+            if (two) {
+                w.x = Elt<T>::pack(a1.x * p.scale, a1.y * p.scale);
+                w.y = Elt<T>::pack(a1.z * p.scale, a1.w * p.scale);
+                *reinterpret_cast<uint2*>(dq + (size_t)(i0 + 1) * p.d_io) = w;
+            }
+        }
     }
 }
 

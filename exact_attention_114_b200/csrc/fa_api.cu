@@ -543,7 +543,7 @@ fa_status_t launch_bwd(const fa::BwdParams& p, const void* q, const void* k, con
     using C = fa::BwdCfg<D>;
     fa_status_t st;
     const long long rows = (long long)p.B * p.Hq * p.Nq_pad;
-    fa::bwd_pre_kernel<D, T><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p);
+    fa::bwd_pre_kernel<D, T><<<(unsigned)((rows + 15) / 16), 256, 0, stream>>>(p);
     if ((st = check_launch("bwd_pre_kernel launch")) != FA_OK) return st;
 
     CUtensorMap mq, mk, mv, mdo;
@@ -558,9 +558,10 @@ fa_status_t launch_bwd(const fa::BwdParams& p, const void* q, const void* k, con
     kern<<<(unsigned)grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mdo, p);
     if ((st = check_launch("bwd_main_kernel launch")) != FA_OK) return st;
 
-    const long long n4 = (long long)p.B * p.Hq * p.Nq * p.d_io / 4;
-    const long long blocks = std::min<long long>((n4 + 255) / 256, (long long)sm_count() * 8);
-    fa::bwd_post_kernel<D, T><<<(unsigned)std::max<long long>(blocks, 1), 256, 0, stream>>>(p);
+    // 16 rows per block; the y dimension walks batch * head (looping past 65535)
+    const dim3 pgrid((unsigned)std::max(1, std::min((p.Nq + 15) / 16, 4096)),
+                     (unsigned)std::max<long long>(1, std::min<long long>((long long)p.B * p.Hq, 65535)));
+    fa::bwd_post_kernel<D, T><<<pgrid, 256, 0, stream>>>(p);
     return check_launch("bwd_post_kernel launch");
 }
 
