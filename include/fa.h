@@ -90,6 +90,12 @@ const char* fa_last_error_message(void);
  * of §09) run the split-KV kernels; their partial results need scratch, which
  * this call allocates stream-ordered with cudaMallocAsync and frees with
  * cudaFreeAsync on `stream`.  Use fa_fwd_splitkv() to pass the scratch instead.
+ * Other shapes run one persistent block per SM.  The blocks share a tile
+ * counter, one of 256 slots in the library's device memory that launches take
+ * in turn; the launch's last block resets it.  So at most 256 tiled forward
+ * launches (this call, fa_fwd_ex, fa_fwd_fp8) may be in flight on one device
+ * at once; more, on concurrent streams, could share a slot and skip tiles.
+ * A launch captured in a CUDA graph keeps its slot on every replay.
  */
 fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                    int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
