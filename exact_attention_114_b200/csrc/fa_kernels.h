@@ -12,7 +12,7 @@ struct FwdParams {
     float* lse;         // [B, Hq, Nq] or nullptr
     int B, Hq, Hkv, Nq, Nk;
     int G;              // Hq / Hkv
-    int n_pairs;        // ceil(Nq / 256): 256-row query tile pairs per head
+    int n_pairs;        // query tile pairs per head: ceil(Nq / 256) (ceil(Nq / 128) at d = 256)
     int d_io;           // head dim of the tensors in memory (<= kernel D, multiple of 32); the
                         // columns d_io..D-1 of the tiles are TMA zero fill and are never stored
     float scale_log2;   // scale * log2(e) (times the Q and K descales for e4m3 inputs)

@@ -5,8 +5,8 @@
 // numerator and denominator together by exp(m_old - m_new), add the block).
 //
 // Layout of one CTA (384 threads = 3 warpgroups, one CTA per SM):
-//   * two 128-row query tiles of one (batch, head), Q0 and Q1, staged once in
-//     shared memory by TMA (128-byte swizzle, 64-column panels);
+//   * per work tile, two 128-row query tiles of one (batch, head), Q0 and Q1,
+//     staged in shared memory by TMA (128-byte swizzle, 64-column panels);
 //   * K and V blocks of 128 keys stream through one ring of NSTAGE tile slots
 //     (order K0, V0, K1, V1, ...), each slot guarded by a full / empty mbarrier;
 //   * tensor memory (512 columns): S0 | S1 (128 fp32 columns each) | O0 | O1
@@ -14,7 +14,8 @@
 //     packed bf16 pairs and is read from there by the P.V MMA;
 //   * warps 0-3 run the softmax of tile 0, warps 4-7 that of tile 1: thread r of
 //     a warpgroup owns query row r, which is TMEM lane r;
-//   * warp 8 issues the TMA loads, warp 9 (one thread) the tcgen05.mma ops in the
+//   * warp 8 claims the work tiles and issues the TMA loads, warp 9 (one
+//     elected thread) the tcgen05.mma ops in the
 //     order S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ..., so the softmax of
 //     one tile overlaps the MMAs of the other; warps 10-11 only complete the
 //     third warpgroup, which hands most of its registers to the softmax ones.
