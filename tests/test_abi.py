@@ -109,6 +109,33 @@ def test_splitkv_rejects_bad_arguments():
     assert call(splits=4, ws=ctypes.c_void_p(0x100080), ws_bytes=need) == fa.FA_ERR_INVALID_ARGUMENT
 
 
+def test_splitkv_noalloc_rejects_before_touching_cuda():
+    # explicit split counts keep the plan off the device query, so every
+    # refusal below happens before the first CUDA call
+    L = fa.lib()
+
+    def call(B=2, Hq=32, Hkv=8, Nq=1, Nk=4096, d=128, splits=4, q=FAKE):
+        return L.fa_fwd_splitkv_noalloc(q, FAKE, FAKE, FAKE, None, B, Hq, Hkv, Nq, Nk, d, 0.1, 0,
+                                        splits, None)
+
+    assert call(q=None) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(q=MISALIGNED) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(splits=-1) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(splits=257) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(Nq=8) == fa.FA_ERR_UNSUPPORTED
+    assert call(d=160) == fa.FA_ERR_UNSUPPORTED
+    # partials larger than the fixed scratch are refused, naming the sizes
+    need = fa.fa_fwd_splitkv_workspace_size(64, 32, 8, 4, 8192, 128, 64)
+    assert need > fa.NOALLOC_SCRATCH_BYTES
+    assert call(B=64, Nq=4, Nk=8192, splits=64) == fa.FA_ERR_WORKSPACE
+    msg = fa.last_error_message()
+    assert str(need) in msg and str(fa.NOALLOC_SCRATCH_BYTES) in msg
+    # the limit is the header's
+    text = open(HEADER, encoding="utf-8").read()
+    m = re.search(r"FA_SPLITKV_NOALLOC_SCRATCH_BYTES \((\d+)u \* (\d+)u \* (\d+)u\)", text)
+    assert m and int(m[1]) * int(m[2]) * int(m[3]) == fa.NOALLOC_SCRATCH_BYTES
+
+
 def test_workspace_sizes():
     # backward: D and LSE rows (fp32) + fp32 dQ accumulator, rows padded to 64
     n = fa.fa_bwd_workspace_size(1, 32, 8, 8192, 8192, 128)
