@@ -202,9 +202,9 @@ def run_reference(args, rank, world):
     w = oracle_sample_workload()
     flops = w.fwd_flops() + w.bwd_flops()
     for _ in range(args.warmup):
-        pass  # the oracle has no warm-up state; its first step is timed like the rest
+        time_oracle_step(w)      # untimed: loads the oracle library and pages in its buffers
     times = [time_oracle_step(w) for _ in range(args.steps)]
-    dt = sum(times) / len(times)
+    dt = sum(sum(t) for t in times) / len(times)
     value = flops / dt / 1e12
     line = {
         "impl": "reference", "metric": "attention fwd+bwd TFLOP/s (causal GQA, N=8192, d=128)",
