@@ -40,6 +40,7 @@ if ROOT not in sys.path:
 import synth  # noqa: E402
 
 STEP_WORKLOAD = "gqa_8k"
+METRIC = "attention fwd+bwd TFLOP/s (causal GQA, N=8192, d=128)"
 DECODE_WORKLOAD = "gqa_decode"
 L2_BYTES = 126 * 1024 * 1024
 
@@ -57,6 +58,15 @@ def dist_env():
 def rank_seed(base_seed: int, rank: int) -> int:
     """Each rank draws its own batch: a distinct seed per rank."""
     return base_seed + 1000 * rank
+
+
+def step_config(world: int) -> dict:
+    """The step workload as both arms report it."""
+    w = synth.WORKLOADS[STEP_WORKLOAD]
+    return {"workload": f"{STEP_WORKLOAD}: B={w.B}, Hq={w.Hq}, Hkv={w.Hkv}, N={w.Nq}, d={w.d}, causal, "
+                        f"bf16 N(0,1) inputs (seed {w.seed})",
+            "global_batch": world * w.B, "seq_len": w.Nq, "parallelism": f"replicas x{world}",
+            "l2": "flushed before every timed call (2 x 126 MiB write)"}
 
 
 def max_over_ranks(value: float, world: int, device=None) -> float:
@@ -207,14 +217,16 @@ def run_reference(args, rank, world):
     dt = sum(sum(t) for t in times) / len(times)
     value = flops / dt / 1e12
     line = {
-        "impl": "reference", "metric": "attention fwd+bwd TFLOP/s (causal GQA, N=8192, d=128)",
-        "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "impl": "reference", "metric": METRIC,
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{STEP_WORKLOAD} (oracle sample: one kv group at N=2048)",
-                   "B": 1, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.Nq, "d": w.d, "causal": True},
+        "config": step_config(world),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
-                         "sample": "fwd+bwd of one kv group (Hq=4, Hkv=1) at N=2048, per step"},
+                         "sample": (f"each step: fp64 oracle fwd+bwd of one kv group (B=1, Hq={w.Hq}, "
+                                    f"Hkv=1, N={w.Nq}, d={w.d}, causal) of the step workload, "
+                                    f"{flops / 1e9:.1f} GFLOP by the FLOP rule, on all host cores, "
+                                    f"rank 0 only")},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -503,14 +515,11 @@ def run_libfa(args, rank, world, local):
 
     clocks = clk.summary()
     line = {
-        "metric": "attention fwd+bwd TFLOP/s (causal GQA, N=8192, d=128)",
+        "metric": METRIC,
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{STEP_WORKLOAD}: B=1, Hq=32, Hkv=8, N=8192, d=128, causal, "
-                               f"bf16 N(0,1) inputs (seed {w.seed})",
-                   "global_batch": world * w.B, "seq_len": w.Nq, "parallelism": f"replicas x{world}",
-                   "l2": "flushed before every timed call (2 x 126 MiB write)"},
+        "config": step_config(world),
         "parts": {
             "fwd": {"ms": fwd_med, "tflops": fwd_tf, "frac_of_peak": fwd_tf / peaks["bf16_tflops_sustained"]},
             "bwd": {"ms": bwd_med, "tflops": bwd_tf, "frac_of_peak": bwd_tf / peaks["bf16_tflops_sustained"]},

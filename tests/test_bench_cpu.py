@@ -6,6 +6,8 @@ import os
 import subprocess
 import sys
 
+import bench
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
@@ -28,10 +30,12 @@ def test_reference_arm_prints_one_contract_line():
     assert d["steps"] == 2 and d["warmup"] == 3 and d["n_gpus"] == 1
     assert d["unit"] == "TFLOP/s" and d["higher_is_better"] is True
     assert d["value"] > 0 and d["ms_per_step"] > 0
+    # the GPU arm's metric and workload; the oracle times a bounded sample of it
+    assert d["metric"] == bench.METRIC and d["config"] == bench.step_config(1)
     # value is the FLOP rule's fwd + bwd FLOPs of the sample over the mean step time
-    c = d["config"]
-    fwd = 4 * c["B"] * c["Hq"] * c["N"] * c["N"] * c["d"] / 2   # causal halves the forward
-    flops = fwd * 3.5                                             # bwd = 2.5 x fwd
+    w = bench.oracle_sample_workload()
+    fwd = 4 * w.B * w.Hq * w.Nq * w.Nk * w.d / 2   # causal halves the forward
+    flops = fwd * 3.5                               # bwd = 2.5 x fwd
     assert abs(flops / (d["ms_per_step"] * 1e-3) / 1e12 - d["value"]) <= 1e-9 * d["value"]
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
