@@ -24,6 +24,7 @@ FA_ERR_UNSUPPORTED = 2
 FA_ERR_WORKSPACE = 3
 FA_ERR_CUDA = 4
 FA_ERR_TIMEOUT = 5
+FA_ERR_SLOT_CONFLICT = 6
 
 FA_DTYPE_BF16 = 0
 FA_DTYPE_FP16 = 1
@@ -92,6 +93,8 @@ def lib() -> ctypes.CDLL:
             L.fa_check_device_status.restype = ip
             L.fa_selftest_wait_timeout.argtypes = [uip, vp]
             L.fa_selftest_wait_timeout.restype = ip
+            L.fa_testhook_tile_slot.argtypes = [ip, uip]
+            L.fa_testhook_tile_slot.restype = ip
             _lib = L
         return _lib
 
@@ -131,9 +134,38 @@ def _dims(q, k):
     return B, Hq, Hkv, Nq, Nk, d
 
 
-def _require(t, name, dtype):
+def _require(t, name, dtype, shape=None):
+    """t must be a contiguous CUDA tensor of `dtype` (and of `shape`, if given):
+    the C ABI only sees a pointer, so a wrong type is read as garbage and a
+    short buffer is written past its end."""
     if not t.is_cuda or not t.is_contiguous() or t.dtype != dtype:
         raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _require_lse(lse, B, Hq, Nq):
+    import torch
+    if lse is not None:
+        _require(lse, "lse", torch.float32, (B, Hq, Nq))
+
+
+def _ws_bytes(workspace):
+    """Size in bytes of a workspace tensor (contiguous, on the device), or 0 for None."""
+    if workspace is None:
+        return 0
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return workspace.numel() * workspace.element_size()
+
+
+def _check_io(q, k, v, o, dtype):
+    """q, k, v, o of one 16-bit dtype; v shaped like k, o like q."""
+    _require(q, "q", dtype)
+    _require(k, "k", dtype)
+    _require(v, "v", dtype, k.shape)
+    if o is not None:
+        _require(o, "o", dtype, q.shape)
 
 
 def _dtype_code(t):
@@ -156,8 +188,8 @@ def fa_fwd(q, k, v, o=None, lse=None, *, causal=False, scale=None, stream=None, 
     import torch
     B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
     dt = _dtype_code(q)
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _require(t, n, q.dtype)
+    _check_io(q, k, v, o, q.dtype)
+    _require_lse(lse, B, Hq, Nq)
     if o is None:
         o = torch.empty_like(q)
     if lse is None and want_lse:
@@ -185,13 +217,16 @@ def fa_fwd_fp8(q, k, v, descale_q, descale_k, descale_v, o=None, lse=None, *, ca
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         if not t.is_cuda or not t.is_contiguous() or t.element_size() != 1:
             raise ValueError(f"{n} must be a contiguous CUDA tensor of e4m3 bytes")
+    if tuple(v.shape) != tuple(k.shape):
+        raise ValueError(f"v has shape {tuple(v.shape)}, expected {tuple(k.shape)}")
     if o is None:
         o = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
-    _require(o, "o", torch.bfloat16)
+    _require(o, "o", torch.bfloat16, q.shape)
+    _require_lse(lse, B, Hq, Nq)
     if lse is None and want_lse:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    ws_bytes = _ws_bytes(workspace)
     _check(lib().fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), float(descale_q), float(descale_k),
                             float(descale_v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d, scale,
                             int(bool(causal)), _ptr(workspace), ws_bytes, _stream(stream)))
@@ -213,16 +248,18 @@ def fa_fwd_splitkv_workspace_size(B, Hq, Hkv, Nq, Nk, d, num_splits=0) -> int:
 
 def fa_fwd_splitkv(q, k, v, o=None, lse=None, *, causal=False, scale=None, num_splits=0,
                    workspace=None, stream=None):
-    """Split-KV (decode-shape) forward.  ``workspace`` is an optional device
-    tensor of at least ``fa_fwd_splitkv_workspace_size`` bytes."""
+    """Split-KV (decode-shape) forward on bf16 tensors.  ``workspace`` is an
+    optional device tensor of at least ``fa_fwd_splitkv_workspace_size`` bytes."""
     import torch
     B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
+    _check_io(q, k, v, o, torch.bfloat16)
+    _require_lse(lse, B, Hq, Nq)
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    ws_bytes = _ws_bytes(workspace)
     _check(lib().fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq,
                                 Nk, d, scale, int(bool(causal)), int(num_splits), _ptr(workspace),
                                 ws_bytes, _stream(stream)))
@@ -247,16 +284,22 @@ def fa_fwd_paged(q, k_cache, v_cache, block_table, seq_lens, o=None, lse=None, *
     for t, n in ((block_table, "block_table"), (seq_lens, "seq_lens")):
         if not t.is_cuda or t.dtype != torch.int32 or not t.is_contiguous():
             raise ValueError(f"{n} must be a contiguous CUDA int32 tensor")
+    if block_table.dim() != 2 or block_table.shape[0] != B or tuple(seq_lens.shape) != (B,):
+        raise ValueError("block_table must be [B, max_pages_per_seq] and seq_lens [B]")
     max_pages = block_table.shape[1]
+    dt = _dtype_code(q)
+    _require(q, "q", q.dtype)
+    _require(k_cache, "k_cache", q.dtype)
+    _require(v_cache, "v_cache", q.dtype)
+    if o is not None:
+        _require(o, "o", q.dtype, q.shape)
+    _require_lse(lse, B, Hq, Nq)
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    dt = _dtype_code(q)
-    for t, n in ((k_cache, "k_cache"), (v_cache, "v_cache"), (o, "o")):
-        _require(t, n, q.dtype)
+    ws_bytes = _ws_bytes(workspace)
     _check(lib().fa_fwd_paged_ex(dt, _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
                                  _ptr(seq_lens), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, d, page_size,
                                  num_pages, max_pages, scale, int(bool(causal)), int(num_splits),
@@ -269,11 +312,16 @@ NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024  # FA_SPLITKV_NOALLOC_SCRATCH_BYTES in f
 
 def fa_fwd_splitkv_noalloc(q, k, v, o, lse, *, causal=False, scale=None, num_splits=0,
                            stream=None):
-    """Split-KV forward that allocates nothing on the device: its partials use
-    a fixed array inside the library.  ``o`` and ``lse`` must be given (this
-    wrapper allocates nothing either).  Calls that overlap on the GPU race on
-    the shared array."""
+    """Split-KV forward on bf16 tensors that allocates nothing on the device:
+    its partials use a fixed array inside the library.  ``o`` [B, Hq, Nq, d]
+    bf16 and ``lse`` [B, Hq, Nq] fp32 must be given (this wrapper allocates
+    nothing either).  Calls that overlap on the GPU race on the shared array."""
+    import torch
     B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
+    if o is None or lse is None:
+        raise ValueError("fa_fwd_splitkv_noalloc needs o and lse (it allocates nothing)")
+    _check_io(q, k, v, o, torch.bfloat16)
+    _require_lse(lse, B, Hq, Nq)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     _check(lib().fa_fwd_splitkv_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv,
                                         Nq, Nk, d, scale, int(bool(causal)), int(num_splits),
@@ -290,12 +338,18 @@ def fa_bwd(q, k, v, o, dout, lse, dq=None, dk=None, dv=None, *, causal=False, sc
     """Backward: returns (dq, dk, dv).  Allocates the gradients when not given."""
     import torch
     B, Hq, Hkv, Nq, Nk, d = _dims(q, k)
+    dt = _dtype_code(q)
+    _check_io(q, k, v, o, q.dtype)
+    _require(dout, "dout", q.dtype, q.shape)
+    _require(lse, "lse", torch.float32, (B, Hq, Nq))
+    for t, n, ref in ((dq, "dq", q), (dk, "dk", k), (dv, "dv", v)):
+        if t is not None:
+            _require(t, n, q.dtype, ref.shape)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    dt = _dtype_code(q)
+    ws_bytes = _ws_bytes(workspace)
     if dt == FA_DTYPE_BF16:
         _check(lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
                             _ptr(dk), _ptr(dv), B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)),
@@ -314,3 +368,9 @@ def fa_check_device_status(stream=None):
 def fa_selftest_wait_timeout(timeout_us: int = 2000, stream=None) -> int:
     """Runs the bounded-wait self-test; returns the raw status (5 = timeout seen)."""
     return int(lib().fa_selftest_wait_timeout(int(timeout_us), _stream(stream)))
+
+
+def fa_testhook_tile_slot(slot: int, preset_owner: int = 0):
+    """Test hook: pin later tiled forward launches to counter slot ``slot``
+    (-1 restores the rotation), optionally presetting the slot's owner tag."""
+    _check(lib().fa_testhook_tile_slot(int(slot), int(preset_owner)))

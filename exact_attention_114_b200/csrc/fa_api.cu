@@ -241,17 +241,26 @@ unsigned fwd_grid(const fa::FwdParams& p)
     return (unsigned)std::max<long long>(1, std::min<long long>(tiles, sm_count()));
 }
 
+// Test hook state: a slot every tiled forward launch is pinned to (-1: rotate).
+std::atomic<int> g_pinned_slot{-1};
+
 // The launch's tile counter: the next slot of fa::g_fwd_tile_ctr (zero between
-// launches: the kernel's last block resets it).  Slots rotate, so concurrent
-// launches on different streams get different ones.
-fa_status_t fwd_tile_counter(unsigned** ctr)
+// launches: the kernel's last block resets it) and the launch's owner tag, a
+// nonzero number unique among the last 2^32 - 1 launches of the process.
+// Slots rotate, so concurrent launches on different streams get different ones;
+// a launch that still finds its slot held by another reports kStatusSlotShared.
+fa_status_t fwd_tile_counter(unsigned** ctr, unsigned* tag)
 {
     static std::atomic<unsigned> seq{0};
     void* base = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&base, fa::g_fwd_tile_ctr);
     if (e != cudaSuccess)
         return cuda_fail(e, "tile counter address");
-    *ctr = static_cast<unsigned*>(base) + 2 * (seq.fetch_add(1u, std::memory_order_relaxed) % fa::kFwdCtrSlots);
+    const unsigned n = seq.fetch_add(1u, std::memory_order_relaxed);
+    const int pinned = g_pinned_slot.load(std::memory_order_relaxed);
+    const unsigned slot = pinned >= 0 ? (unsigned)pinned : n % fa::kFwdCtrSlots;
+    *ctr = static_cast<unsigned*>(base) + fa::kFwdCtrWords * slot;
+    *tag = n % 0xFFFFFFFFu + 1u;
     return FA_OK;
 }
 
@@ -280,7 +289,7 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     p.d_io = d;
     p.scale_log2 = scale * kLog2e;
     p.o_scale = 1.f;
-    if ((st = fwd_tile_counter(&p.tile_ctr)) != FA_OK)
+    if ((st = fwd_tile_counter(&p.tile_ctr, &p.tile_tag)) != FA_OK)
         return st;
     kern<<<fwd_grid(p), C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
     return check_launch("fwd_kernel launch");
@@ -328,7 +337,7 @@ fa_status_t launch_fwd_fp8(const void* q, const void* k, const void* v, void* vt
     p.d_io = kF8D;
     p.scale_log2 = scale_log2;
     p.o_scale = o_scale;
-    if ((st = fwd_tile_counter(&p.tile_ctr)) != FA_OK)
+    if ((st = fwd_tile_counter(&p.tile_ctr, &p.tile_tag)) != FA_OK)
         return st;
     kern<<<fwd_grid(p), C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
     return check_launch("fwd_kernel (e4m3) launch");
@@ -489,13 +498,33 @@ fa_status_t launch_decode(const void* q, const void* k, const void* v, void* o, 
 // Every GPU that loads the library holds this array until the process exits.
 static __device__ __align__(256) unsigned char g_splitkv_scratch[FA_SPLITKV_NOALLOC_SCRATCH_BYTES];
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn get_ctx_current()
+{
+    static std::once_flag once;
+    static CtxGetCurrentFn fn = nullptr;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+    });
+    return fn;
+}
+
 // Device address of g_splitkv_scratch on the current device.  In host code the
-// symbol is only a host-side stand-in, so the address is looked up once per
-// device (with that device current) and cached.
+// symbol is only a host-side stand-in, so the address is looked up with the
+// device current, once per device and context, and cached.  The cache is keyed
+// on the current CUDA context as well as the device: after cudaDeviceReset the
+// runtime makes a new context, the module (and the array) is loaded again, and
+// the address is looked up again instead of reusing the old one.
 fa_status_t noalloc_scratch(void** out)
 {
     static std::mutex mu;
     static void* addr[64] = {};
+    static CUcontext ctx_of[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
@@ -504,13 +533,26 @@ fa_status_t noalloc_scratch(void** out)
         set_error("device ordinal %d out of range", dev);
         return FA_ERR_UNSUPPORTED;
     }
+    CtxGetCurrentFn get_ctx = get_ctx_current();
+    CUcontext ctx = nullptr;
+    if (!get_ctx || get_ctx(&ctx) != CUDA_SUCCESS) {
+        set_error("cuCtxGetCurrent is unavailable");
+        return FA_ERR_CUDA;
+    }
     std::lock_guard<std::mutex> lk(mu);
-    if (addr[dev] == nullptr) {
+    if (ctx == nullptr || addr[dev] == nullptr || ctx_of[dev] != ctx) {
+        // the lookup also sets up the runtime's context on this device if this
+        // thread had none yet; the context is read again after it
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_splitkv_scratch);
         if (e != cudaSuccess)
             return cuda_fail(e, "cudaGetSymbolAddress (split-KV scratch)");
+        if (get_ctx(&ctx) != CUDA_SUCCESS) {
+            set_error("cuCtxGetCurrent failed");
+            return FA_ERR_CUDA;
+        }
         addr[dev] = p;
+        ctx_of[dev] = ctx;
     }
     *out = addr[dev];
     return FA_OK;
@@ -601,6 +643,7 @@ const char* fa_status_string(fa_status_t s)
     case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
     case FA_ERR_CUDA: return "FA_ERR_CUDA";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    case FA_ERR_SLOT_CONFLICT: return "FA_ERR_SLOT_CONFLICT";
     }
     return "FA_ERR_UNKNOWN";
 }
@@ -804,7 +847,11 @@ fa_status_t fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, 
         set_error("split-KV needs d <= 128 and Nq * Hq / Hkv <= %d", kDecodeMaxRows);
         return FA_ERR_UNSUPPORTED;
     }
-    const DecodePlan pl = decode_plan(B, Hq, Hkv, Nq, Nk, d, num_splits);
+    DecodePlan pl = decode_plan(B, Hq, Hkv, Nq, Nk, d, num_splits);
+    // an automatic split count is lowered until the partials fit (one split
+    // needs no scratch at all); an explicit count that does not fit is refused
+    while (num_splits == 0 && pl.splits > 1 && pl.total() > (size_t)FA_SPLITKV_NOALLOC_SCRATCH_BYTES)
+        pl = decode_plan(B, Hq, Hkv, Nq, Nk, d, pl.splits - 1);
     if (pl.total() > (size_t)FA_SPLITKV_NOALLOC_SCRATCH_BYTES) {
         set_error("this shape needs %zu bytes of split-KV scratch but the fixed scratch holds %zu; "
                   "use fewer splits or fa_fwd_splitkv with a caller workspace",
@@ -1043,10 +1090,47 @@ fa_status_t fa_check_device_status(void* stream)
         e = cudaStreamSynchronize(s);
     if (e != cudaSuccess)
         return cuda_fail(e, "reading the device status word");
+    if (h & fa::kStatusSlotShared) {
+        // A slot may have been left marked by the launch that lost it: once every
+        // launch on the device has finished, all slots are cleared.
+        void* base = nullptr;
+        e = cudaDeviceSynchronize();
+        if (e == cudaSuccess)
+            e = cudaGetSymbolAddress(&base, fa::g_fwd_tile_ctr);
+        if (e == cudaSuccess)
+            e = cudaMemset(base, 0, sizeof(fa::g_fwd_tile_ctr));
+        if (e == cudaSuccess)
+            e = cudaDeviceSynchronize();
+        if (e != cudaSuccess)
+            return cuda_fail(e, "clearing the forward tile-counter slots");
+        set_error("a tiled forward launch found its tile-counter slot held by another launch in flight "
+                  "(more than 256 tiled forwards at once); its output is incomplete");
+        return FA_ERR_SLOT_CONFLICT;
+    }
     if (h & fa::kStatusTimeout) {
         set_error("a bounded device wait ran out");
         return FA_ERR_TIMEOUT;
     }
+    return FA_OK;
+}
+
+fa_status_t fa_testhook_tile_slot(int slot, unsigned preset_owner)
+{
+    t_error.clear();
+    if (slot < -1 || slot >= fa::kFwdCtrSlots) {
+        set_error("slot=%d must be -1 or in [0, %d)", slot, fa::kFwdCtrSlots);
+        return FA_ERR_INVALID_ARGUMENT;
+    }
+    if (slot >= 0 && preset_owner != 0u) {
+        void* base = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&base, fa::g_fwd_tile_ctr);
+        if (e == cudaSuccess)
+            e = cudaMemcpy(static_cast<unsigned*>(base) + fa::kFwdCtrWords * slot + 2, &preset_owner,
+                           sizeof preset_owner, cudaMemcpyHostToDevice);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "presetting a tile-counter slot owner");
+    }
+    g_pinned_slot.store(slot, std::memory_order_relaxed);
     return FA_OK;
 }
 

@@ -17,8 +17,9 @@ struct FwdParams {
                         // columns d_io..D-1 of the tiles are TMA zero fill and are never stored
     float scale_log2;   // scale * log2(e) (times the Q and K descales for e4m3 inputs)
     float o_scale;      // O = o_scale * U / l: 1, or the V descale for e4m3 inputs
-    unsigned* tile_ctr; // [2]: tiles claimed beyond each block's first, blocks done claiming
-                        // (zero at launch; the last block resets them)
+    unsigned* tile_ctr; // [4]: tiles claimed beyond each block's first, blocks done claiming,
+                        // owner tag (zero when free; the last block resets all three), padding
+    unsigned tile_tag;  // this launch's owner tag (nonzero)
 };
 
 struct DecodeParams {

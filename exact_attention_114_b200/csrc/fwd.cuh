@@ -92,13 +92,19 @@ __device__ __forceinline__ int fwd_blocks_for_tile(int qt, int Nq, int Nk, bool 
     return min(nkb, last_key / 128 + 1);
 }
 
-// Tile counters of the forward launches, two words per slot: tiles claimed
-// beyond each block's first, and blocks that have stopped claiming.  Each
-// launch takes the next slot (launches in flight on different streams do not
-// share one); the last block to stop claiming sets both words back to zero for
-// the slot's next launch, so a slot is zero whenever no launch is using it.
+// Tile counters of the forward launches, four words per slot: tiles claimed
+// beyond each block's first, blocks that have stopped claiming, the owner tag
+// of the launch using the slot (0 = free), and padding.  Each launch takes the
+// next slot (launches in flight on different streams do not share one) and a
+// nonzero tag of its own.  Every block first swaps the free owner word for its
+// launch's tag; a block that finds another launch's tag there records
+// kStatusSlotShared, runs its own first tile only and leaves the slot alone, so
+// the other launch's tiles are never taken.  The last block to stop claiming
+// sets the counters and then the owner back to zero, so a slot is all zero
+// whenever no launch is using it.
 constexpr int kFwdCtrSlots = 256;
-__device__ unsigned g_fwd_tile_ctr[kFwdCtrSlots][2];
+constexpr int kFwdCtrWords = 4;
+__device__ unsigned g_fwd_tile_ctr[kFwdCtrSlots][kFwdCtrWords];
 
 // One work tile: a pair of 128-row query tiles (one at d = 256) of one
 // (batch, head).  Tile i of the launch: pair n_pairs-1 - i / (B*Hq) (heaviest
@@ -225,6 +231,11 @@ __global__ void __launch_bounds__(384, 1)
             int kvi = 0;            // K/V ring loads so far
             bool ok = true;
             int tile = (int)blockIdx.x;
+            // take the counter slot for this launch, or find it held by another one
+            const unsigned owner = atomicCAS(p.tile_ctr + 2, 0u, p.tile_tag);
+            const bool own_slot = (owner == 0u || owner == p.tile_tag);
+            if (!own_slot)
+                atomicOr(&g_status, kStatusSlotShared);
             for (int u = 0; ok; ++u) {
                 // publish the tile to the other roles (a ring of two entries)
                 if (!(ok = mbar_wait(&bar_tfree[u & 1], ((uint32_t)(u >> 1) & 1u) ^ 1u, abort_flag)))
@@ -272,15 +283,22 @@ __global__ void __launch_bounds__(384, 1)
                 // work (a block that claimed at its start would take a second tile
                 // before knowing whether its first is long), and the claim's latency
                 // hides behind the rest of the tile.
-                tile = (int)gridDim.x + (int)atomicAdd(p.tile_ctr, 1u);
+                tile = own_slot ? (int)gridDim.x + (int)atomicAdd(p.tile_ctr, 1u) : n_tiles;
             }
             // this block claims no more tiles; the last one to get here (finished or
-            // aborted) resets the launch's counter slot
-            __threadfence();
-            if (atomicAdd(p.tile_ctr + 1, 1u) == gridDim.x - 1) {
+            // aborted) resets the launch's counter slot, the owner word last.  A block
+            // that found the slot held by another launch touches nothing: its launch
+            // never counts all its blocks, so the slot stays marked until
+            // fa_check_device_status() clears every slot after reporting the conflict.
+            if (own_slot) {
                 __threadfence();
-                atomicExch(p.tile_ctr, 0u);
-                atomicExch(p.tile_ctr + 1, 0u);
+                if (atomicAdd(p.tile_ctr + 1, 1u) == gridDim.x - 1) {
+                    __threadfence();
+                    atomicExch(p.tile_ctr, 0u);
+                    atomicExch(p.tile_ctr + 1, 0u);
+                    __threadfence();
+                    atomicExch(p.tile_ctr + 2, 0u);
+                }
             }
             if (*abort_flag) {
                 // let the last load of every slot and of both Q slots land before the block exits

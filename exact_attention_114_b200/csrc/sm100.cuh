@@ -19,6 +19,8 @@ namespace fa {
 // device status word: bounded waits that run out record an error code here
 // ---------------------------------------------------------------------------
 constexpr unsigned kStatusTimeout = 1u;
+// a tiled forward launch found its tile-counter slot held by another launch
+constexpr unsigned kStatusSlotShared = 2u;
 
 // One word per device and per module (libfa is a single translation unit).
 static __device__ unsigned int g_status = 0;

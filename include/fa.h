@@ -62,7 +62,8 @@ typedef enum {
     FA_ERR_UNSUPPORTED = 2,      /* valid but not implemented (e.g. d = 80, or d > 128 in the backward) */
     FA_ERR_WORKSPACE = 3,        /* workspace given but smaller than required */
     FA_ERR_CUDA = 4,             /* a CUDA runtime / driver call failed */
-    FA_ERR_TIMEOUT = 5           /* a bounded device wait ran out */
+    FA_ERR_TIMEOUT = 5,          /* a bounded device wait ran out */
+    FA_ERR_SLOT_CONFLICT = 6     /* a tiled forward found its tile-counter slot in use (see fa_fwd) */
 } fa_status_t;
 
 /* Element type of the 16-bit tensors (q, k, v, o, dout, dq, dk, dv). */
@@ -94,8 +95,12 @@ const char* fa_last_error_message(void);
  * counter, one of 256 slots in the library's device memory that launches take
  * in turn; the launch's last block resets it.  So at most 256 tiled forward
  * launches (this call, fa_fwd_ex, fa_fwd_fp8) may be in flight on one device
- * at once; more, on concurrent streams, could share a slot and skip tiles.
- * A launch captured in a CUDA graph keeps its slot on every replay.
+ * at once.  Each launch marks its slot with a tag of its own; a launch whose
+ * blocks find the slot held by another launch takes no tile from it, leaves
+ * its own output incomplete and records FA_ERR_SLOT_CONFLICT in the device
+ * status word, which the next fa_check_device_status() reports (so an overrun
+ * is reported, never a silently wrong O).  A launch captured in a CUDA graph
+ * keeps its slot and tag on every replay.
  */
 fa_status_t fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                    int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
@@ -207,12 +212,19 @@ fa_status_t fa_fwd_paged_ex(fa_dtype_t dtype, const void* q, const void* k_cache
  * array of FA_SPLITKV_NOALLOC_SCRATCH_BYTES inside the library, which every GPU
  * that loads the library holds until the process exits.
  *   - No cudaMalloc, cudaFree or other allocating call is made.
- *   - A shape whose partials need more than FA_SPLITKV_NOALLOC_SCRATCH_BYTES
- *     (fa_fwd_splitkv_workspace_size() with the same arguments) is rejected
- *     with FA_ERR_WORKSPACE before anything is launched; fewer splits need less.
+ *   - With num_splits = 0 the split count is chosen as for fa_fwd_splitkv and
+ *     then lowered until the partials fit the array (a single split needs no
+ *     scratch), so the automatic choice never fails for lack of scratch.  An
+ *     explicit num_splits whose partials need more than
+ *     FA_SPLITKV_NOALLOC_SCRATCH_BYTES (fa_fwd_splitkv_workspace_size() with
+ *     the same arguments) is rejected with FA_ERR_WORKSPACE before anything is
+ *     launched; fewer splits need less.
  *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current and caches it; make that
- *     first call before any stream capture.
+ *     (cudaGetSymbolAddress) with that device current and caches it, keyed on
+ *     the device and its current CUDA context, so a call after cudaDeviceReset
+ *     (a new context, the array loaded again) looks the address up again; make
+ *     the first call on a device, and the first after a reset, before any
+ *     stream capture.
  *   - All calls share the one array and it keeps the previous call's contents.
  *     Nothing in it needs clearing (each call writes every partial it reads),
  *     but calls that can overlap on the GPU -- on different streams, or on
@@ -251,10 +263,26 @@ fa_status_t fa_bwd_ex(fa_dtype_t dtype, const void* q, const void* k, const void
 
 /*
  * Reads and clears the device status word of the current device.  Synchronises
- * `stream` (the only call that does).  Returns FA_OK, or FA_ERR_TIMEOUT if a
- * bounded wait in a kernel ran out since the last check, or FA_ERR_CUDA.
+ * `stream` (the only call that does).  Returns FA_OK; FA_ERR_SLOT_CONFLICT if a
+ * tiled forward found its tile-counter slot held by another launch since the
+ * last check (the call then waits for the whole device, cudaDeviceSynchronize,
+ * and clears every slot, so call it when no forward of the results you still
+ * trust is in flight); FA_ERR_TIMEOUT if a bounded wait in a kernel ran out; or
+ * FA_ERR_CUDA.
  */
 fa_status_t fa_check_device_status(void* stream);
+
+/*
+ * Test hook (not for production use; the pages have no counterpart): pins
+ * every later tiled forward launch of the process to tile-counter slot `slot`
+ * (0..255), or restores the rotation with slot = -1.  With a slot given and
+ * preset_owner != 0, first writes preset_owner into that slot's owner word
+ * (synchronous copy), as if a launch with that tag held the slot: the next
+ * launch pinned there must then report FA_ERR_SLOT_CONFLICT.  Returns
+ * FA_ERR_INVALID_ARGUMENT for a slot outside -1..255, FA_ERR_CUDA if the copy
+ * fails.
+ */
+fa_status_t fa_testhook_tile_slot(int slot, unsigned preset_owner);
 
 /*
  * Self-test of the bounded-wait machinery: launches one block that waits on a

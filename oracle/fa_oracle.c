@@ -498,11 +498,19 @@ int oracle_bwd_dq_rows(const void* q, const void* k, const void* v, const void* 
 /* dK and dV for a list of keys (b, g, j) given as flattened key rows
  * kr = (b * Hkv + g) * Nk + j.  Every query row of the group that sees key j
  * contributes, and each such row needs its own full P and dP rows for D_i.
- * dk, dv: [nkeys, d]. */
+ * dk, dv: [nkeys, d].
+ *
+ * The work unit is (kv group, chunk of the group's query rows): each row's P
+ * and dP are computed once and then added into every requested key of that
+ * group the row sees.  For each key the rows are still added in the same order
+ * (row order inside a chunk, then the chunks in order), so the result does not
+ * depend on which other keys are requested with it. */
 typedef struct {
     const problem_t* pb;
     const int64_t* keys;
     int64_t nkeys;
+    const int64_t* groups;   /* distinct b * Hkv + g among the keys */
+    int64_t ngroups;
     double* dk_part; /* [nchunks, nkeys, d] */
     double* dv_part;
     int64_t nchunks;
@@ -522,26 +530,32 @@ static void dkrow_range(void* vctx, int64_t begin, int64_t end, int tid)
     double* oi = (double*)malloc(sizeof(double) * d);
     double* kvec = (double*)malloc(sizeof(double) * d);
     double* dp = (double*)malloc(sizeof(double) * Nk);
-    /* unit = (key index, chunk) */
+    /* unit = (group, chunk) */
     for (int64_t u = begin; u < end; ++u) {
-        int64_t kk = u / c->nchunks;
-        int64_t chunk = u % c->nchunks;
-        int64_t flat = c->keys[kk];
-        int64_t j = flat % Nk;
-        int64_t g = (flat / Nk) % pb->Hkv;
-        int64_t b = flat / (Nk * pb->Hkv);
-        double* dkj = c->dk_part + (chunk * c->nkeys + kk) * d;
-        double* dvj = c->dv_part + (chunk * c->nkeys + kk) * d;
-        for (int64_t t = 0; t < d; ++t) {
-            dkj[t] = 0.0;
-            dvj[t] = 0.0;
+        const int64_t gi = u / c->nchunks;
+        const int64_t chunk = u % c->nchunks;
+        const int64_t grp = c->groups[gi];
+        const int64_t g = grp % pb->Hkv, b = grp / pb->Hkv;
+        int64_t jmin = Nk;   /* smallest requested key of the group: rows that miss it miss all */
+        for (int64_t kk = 0; kk < c->nkeys; ++kk) {
+            if (c->keys[kk] / Nk != grp)
+                continue;
+            const int64_t j = c->keys[kk] % Nk;
+            if (j < jmin)
+                jmin = j;
+            double* dkj = c->dk_part + (chunk * c->nkeys + kk) * d;
+            double* dvj = c->dv_part + (chunk * c->nkeys + kk) * d;
+            for (int64_t t = 0; t < d; ++t) {
+                dkj[t] = 0.0;
+                dvj[t] = 0.0;
+            }
         }
         int64_t rows = G * Nq;
         int64_t r0 = rows * chunk / c->nchunks, r1 = rows * (chunk + 1) / c->nchunks;
         for (int64_t r = r0; r < r1; ++r) {
             int64_t h = g * G + r / Nq;
             int64_t i = r % Nq;
-            if (!visible(pb, i, j))
+            if (!visible(pb, i, jmin))
                 continue;
             load_vec(pb->q, pb->dtype, q_off(pb, b, h, i), d, qi);
             load_vec(pb->dout, pb->dtype, q_off(pb, b, h, i), d, doi);
@@ -559,10 +573,19 @@ static void dkrow_range(void* vctx, int64_t begin, int64_t end, int tid)
                 dp[jj] = acc;
                 D += p[jj] * acc;
             }
-            double ds = p[j] * (dp[j] - D);
-            for (int64_t t = 0; t < d; ++t) {
-                dkj[t] += pb->scale * ds * qi[t];
-                dvj[t] += p[j] * doi[t];
+            for (int64_t kk = 0; kk < c->nkeys; ++kk) {
+                if (c->keys[kk] / Nk != grp)
+                    continue;
+                const int64_t j = c->keys[kk] % Nk;
+                if (!visible(pb, i, j))
+                    continue;
+                double* dkj = c->dk_part + (chunk * c->nkeys + kk) * d;
+                double* dvj = c->dv_part + (chunk * c->nkeys + kk) * d;
+                double ds = p[j] * (dp[j] - D);
+                for (int64_t t = 0; t < d; ++t) {
+                    dkj[t] += pb->scale * ds * qi[t];
+                    dvj[t] += p[j] * doi[t];
+                }
             }
         }
     }
@@ -595,8 +618,24 @@ int oracle_bwd_dkv_rows(const void* q, const void* k, const void* v, const void*
         free(dv_part);
         return 2;
     }
-    dkrow_ctx_t c = {&pb, keys, nkeys, dk_part, dv_part, nchunks};
-    parallel_for(nkeys * nchunks, nthreads, dkrow_range, &c);
+    int64_t* groups = (int64_t*)malloc(sizeof(int64_t) * (nkeys > 0 ? nkeys : 1));
+    if (!groups) {
+        free(dk_part);
+        free(dv_part);
+        return 2;
+    }
+    int64_t ngroups = 0;
+    for (int64_t kk = 0; kk < nkeys; ++kk) {
+        const int64_t grp = keys[kk] / Nk;
+        int64_t seen = 0;
+        for (int64_t x = 0; x < ngroups; ++x)
+            seen |= (groups[x] == grp);
+        if (!seen)
+            groups[ngroups++] = grp;
+    }
+    dkrow_ctx_t c = {&pb, keys, nkeys, groups, ngroups, dk_part, dv_part, nchunks};
+    parallel_for(ngroups * nchunks, nthreads, dkrow_range, &c);
+    free(groups);
     for (int64_t kk = 0; kk < nkeys; ++kk) {
         for (int64_t t = 0; t < d; ++t) {
             double a = 0.0, bsum = 0.0;

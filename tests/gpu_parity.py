@@ -6,9 +6,9 @@ accumulation): |O - O_ref| <= 1e-2, max |LSE - LSE_ref| <= 1e-3 (rows that
 see no key must give -inf on both sides), and for each gradient
 max |dX - dX_ref| <= 2e-2 * max |dX_ref|.
 
-O is stored in bf16, whose spacing is 2^-6 for |O| in [4, 8): half of it
-exceeds 1e-2 there, so even the correctly rounded exact result can miss the
-bar.  The O bound is therefore taken per element as
+O is stored in bf16, whose values are 2^-5 apart for |O| in [4, 8): half a
+spacing (2^-6) exceeds 1e-2 there, so even the correctly rounded exact result
+can miss the bar.  The O bound is therefore taken per element as
 max(1e-2, half a bf16 ulp of O_ref + 2e-3), which is 1e-2 wherever |O_ref| < 4,
 and a failure message reports the error against the bf16-rounded reference.
 """
@@ -131,3 +131,16 @@ def sample_keys_cheap(w: synth.Workload, kv_heads=(0,), seed=0):
     js = sorted({w.Nk - 1, w.Nk - 2, w.Nk - 64, w.Nk - 127, w.Nk - 128, w.Nk - 129})
     js = [j for j in js if 0 <= j < w.Nk]
     return np.array([(0 * w.Hkv + g) * w.Nk + j for g in kv_heads for j in js], dtype=np.int64)
+
+
+def sample_keys_heavy(w: synth.Workload, kv_heads=(0,)):
+    """Flattened keys whose dK/dV collect the most query rows: the first keys of
+    the first key blocks (under a causal mask every row of the group sees key
+    0, and the CTA of key block 0 accumulates dK/dV over every query block of
+    every head of the group), the edges of blocks 0 and 1, and the two keys
+    around the middle of the sequence, in the first and the last batch."""
+    js = sorted({0, 63, 64, 127, 128, w.Nk // 2 - 1, w.Nk // 2})
+    js = [j for j in js if 0 <= j < w.Nk]
+    bs = sorted({0, w.B - 1})
+    return np.array([(b * w.Hkv + g) * w.Nk + j for b in bs for g in kv_heads for j in js],
+                    dtype=np.int64)

@@ -34,7 +34,8 @@ def test_every_declared_symbol_is_exported():
 def test_abi_version_and_status_strings():
     assert fa.abi_version() == 1
     for code, name in [(0, "FA_OK"), (1, "FA_ERR_INVALID_ARGUMENT"), (2, "FA_ERR_UNSUPPORTED"),
-                       (3, "FA_ERR_WORKSPACE"), (4, "FA_ERR_CUDA"), (5, "FA_ERR_TIMEOUT")]:
+                       (3, "FA_ERR_WORKSPACE"), (4, "FA_ERR_CUDA"), (5, "FA_ERR_TIMEOUT"),
+                       (6, "FA_ERR_SLOT_CONFLICT")]:
         assert fa.status_string(code) == name
         # the enum values in the header match
         assert re.search(rf"\b{name}\s*=\s*{code}\b", open(HEADER, encoding="utf-8").read())
@@ -222,3 +223,14 @@ def test_fp8_rejects_bad_arguments():
     assert call(ws=ctypes.c_void_p(0x100000), ws_bytes=need - 1) == fa.FA_ERR_WORKSPACE
     assert call(ws=ctypes.c_void_p(0x100010), ws_bytes=need) == fa.FA_ERR_INVALID_ARGUMENT
     assert fa.fa_fwd_fp8_workspace_size(2, 8, 8192, 128) == 2 * 8 * 128 * 8192
+
+
+def test_tile_slot_hook_checks_its_slot_before_any_cuda_call():
+    """The test hook refuses a slot outside -1..255; pinning and releasing
+    without a preset owner makes no CUDA call at all."""
+    L = fa.lib()
+    for bad in (-2, 256, 10_000):
+        assert L.fa_testhook_tile_slot(bad, 0) == fa.FA_ERR_INVALID_ARGUMENT
+        assert "slot" in fa.last_error_message()
+    assert L.fa_testhook_tile_slot(3, 0) == fa.FA_OK
+    assert L.fa_testhook_tile_slot(-1, 0) == fa.FA_OK

@@ -30,10 +30,13 @@ def test_reference_arm_prints_one_contract_line():
     assert d["steps"] == 2 and d["warmup"] == 3 and d["n_gpus"] == 1
     assert d["unit"] == "TFLOP/s" and d["higher_is_better"] is True
     assert d["value"] > 0 and d["ms_per_step"] > 0
-    # the GPU arm's metric and workload; the oracle times a bounded sample of it
-    assert d["metric"] == bench.METRIC and d["config"] == bench.step_config(1)
-    # value is the FLOP rule's fwd + bwd FLOPs of the sample over the mean step time
+    # the GPU arm's metric; the config names the bounded sample of its workload
+    # that the oracle actually times
     w = bench.oracle_sample_workload()
+    assert d["metric"] == bench.METRIC and d["config"] == bench.reference_config(w)
+    assert f"B={w.B}, Hq={w.Hq}, Hkv={w.Hkv}, N={w.Nq}" in d["config"]["workload"]
+    assert d["config"]["sample_of"] == bench.STEP_WORKLOAD
+    # value is the FLOP rule's fwd + bwd FLOPs of the sample over the mean step time
     fwd = 4 * w.B * w.Hq * w.Nq * w.Nk * w.d / 2   # causal halves the forward
     flops = fwd * 3.5                               # bwd = 2.5 x fwd
     assert abs(flops / (d["ms_per_step"] * 1e-3) / 1e12 - d["value"]) <= 1e-9 * d["value"]

@@ -55,9 +55,12 @@ def test_backward_config_one_group_full(name):
 
 @pytest.mark.parametrize("name", ["mha_4k_long", "gqa_8k"])
 def test_backward_config_sampled(name):
-    """Full-size inputs and launch; dQ on sampled rows, dK/dV on keys near the
-    end (cheap for the oracle under the causal mask), plus the dV column-sum
-    identity sum_j dV_j = sum of dO over the group's rows."""
+    """Full-size inputs and launch; dQ on sampled rows; dK/dV element by element
+    on keys near the end (seen by few rows) and on the heaviest keys (seen by
+    every row of the group: at gqa_8k the CTA of key block 0 accumulates dK/dV
+    in tensor memory over 4 heads x 128 query blocks = 512 steps), on the first
+    and last kv heads; plus the dV column-sum identity sum_j dV_j = sum of dO
+    over the group's rows."""
     w = synth.WORKLOADS[name]
     x = synth.make_inputs(w)
     xd = G.to_gpu(x)
@@ -69,10 +72,11 @@ def test_backward_config_sampled(name):
     dq_s = G.f64(dq).reshape(-1, d)[rows]
     # relative to the largest reference entry over the sampled rows
     G.assert_grad(dq_s, rq, "dQ (sampled rows)")
-    keys = G.sample_keys_cheap(w, kv_heads=(0, w.Hkv - 1))
-    rk, rv = oracle.bwd_dkv_rows(x["q"], x["k"], x["v"], x["dout"], w.scale, w.causal, keys)
-    G.assert_grad(G.f64(dk).reshape(-1, d)[keys], rk, "dK (sampled keys)")
-    G.assert_grad(G.f64(dv).reshape(-1, d)[keys], rv, "dV (sampled keys)")
+    for what, keys in (("keys near the end", G.sample_keys_cheap(w, kv_heads=(0, w.Hkv - 1))),
+                       ("heaviest keys", G.sample_keys_heavy(w, kv_heads=(0, w.Hkv - 1)))):
+        rk, rv = oracle.bwd_dkv_rows(x["q"], x["k"], x["v"], x["dout"], w.scale, w.causal, keys)
+        G.assert_grad(G.f64(dk).reshape(-1, d)[keys], rk, f"dK ({what})")
+        G.assert_grad(G.f64(dv).reshape(-1, d)[keys], rv, f"dV ({what})")
     for t in (dq, dk, dv):
         assert torch.isfinite(t).all()
     # dV column sums: every P row sums to one

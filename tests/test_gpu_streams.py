@@ -71,3 +71,36 @@ def test_many_launches_keep_counter_slots_consistent():
     torch.cuda.synchronize()
     fa.fa_check_device_status()
     assert torch.equal(o1, r1) and torch.equal(o2, r2)
+
+
+def test_slot_held_by_another_launch_is_reported_not_silent():
+    """A launch whose counter slot is held by another launch (simulated by
+    presetting the slot's owner tag through the test hook) must end in
+    FA_ERR_SLOT_CONFLICT from fa_check_device_status, never FA_OK with skipped
+    tiles; the check clears every slot, after which the same call, pinned to
+    the same slot, again matches the result of a normal launch bit for bit."""
+    # 16 tile pairs x 16 heads = 256 tiles > 148 SMs: blocks must claim tiles
+    w = synth.Workload("slot", 1, 16, 4, 4096, 4096, 128, True, 7400, backward=False)
+    x = {k: v.cuda() for k, v in synth.make_inputs(w, dout=False).items()}
+    o_ref, l_ref = fa.fa_fwd(x["q"], x["k"], x["v"], causal=True)
+    torch.cuda.synchronize()
+    fa.fa_check_device_status()
+    slot = 7
+    try:
+        fa.fa_testhook_tile_slot(slot, preset_owner=0xDEADBEEF)
+        fa.fa_fwd(x["q"], x["k"], x["v"], causal=True)
+        torch.cuda.synchronize()
+        with pytest.raises(fa.FaError) as err:
+            fa.fa_check_device_status()
+        assert err.value.status == fa.FA_ERR_SLOT_CONFLICT
+        # the check cleared the slots: a launch pinned to the same slot runs whole
+        o, lse = fa.fa_fwd(x["q"], x["k"], x["v"], causal=True)
+        torch.cuda.synchronize()
+        fa.fa_check_device_status()
+    finally:
+        fa.fa_testhook_tile_slot(-1)
+    assert torch.equal(o, o_ref) and torch.equal(lse, l_ref)
+    o2, l2 = fa.fa_fwd(x["q"], x["k"], x["v"], causal=True)
+    torch.cuda.synchronize()
+    fa.fa_check_device_status()
+    assert torch.equal(o2, o_ref) and torch.equal(l2, l_ref)

@@ -52,3 +52,33 @@ def test_two_ranks_gloo():
 def test_single_rank_helpers():
     assert bench.max_over_ranks(3.5, 1) == 3.5
     assert bench.rank_seed(1004, 0) == 1004 and bench.rank_seed(1004, 1) != 1004
+
+
+def test_gpus_flag_starts_the_ranks_itself(tmp_path):
+    """Without torchrun's environment, bench.py --gpus 2 starts two ranks
+    through its replica launcher; each joins the process group (gloo here, in
+    place of the GPU arm) and sees world == 2 on 127.0.0.1."""
+    env_keys = ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")
+    saved = {k: os.environ.pop(k) for k in env_keys if k in os.environ}
+    try:
+        probe = os.path.join(os.path.dirname(os.path.abspath(__file__)), "rank_probe.py")
+        assert bench.spawn_replicas(2, [str(tmp_path)], script=probe) == 0
+    finally:
+        os.environ.update(saved)
+    import json
+    seen = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(2)]
+    for r, s in enumerate(seen):
+        assert (s["rank"], s["world"], s["local"], s["group_world"]) == (r, 2, r, 2)
+        assert s["rank_sum"] == 1.0 and s["master"] == "127.0.0.1" and s["max_over_ranks"] == 11.0
+
+
+def test_main_spawns_only_outside_torchrun(monkeypatch):
+    calls = []
+    monkeypatch.setattr(bench, "spawn_replicas", lambda n, argv, script=None: calls.append((n, argv)) or 0)
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    assert bench.main(["--gpus", "2", "--steps", "5"]) == 0
+    assert calls == [(2, ["--gpus", "2", "--steps", "5"])]
+    cmd = bench.replica_command(4, ["--steps", "5"], port=29555)
+    assert cmd[1:3] == ["-m", "torch.distributed.run"] and "--nproc-per-node=4" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1" and cmd[-2:] == ["--steps", "5"]

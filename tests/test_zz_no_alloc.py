@@ -2,12 +2,16 @@
 device memory (for callers that may not allocate on their call path, such as
 an inference runtime's plugin whose enqueue step must not allocate).
 
-It must give the same result as fa_fwd_splitkv with a caller workspace, within
-the parity tolerances of the other tests (|O| <= 1e-2, |LSE| <= 1e-3), on two
-calls in a row with different shapes (the fixed scratch keeps the previous
-call's contents, which must not leak into the next result), and it must refuse
-a shape whose partials do not fit the fixed scratch.  This file is collected
-last so that a stop at the first failure has run every other test already.
+On two calls in a row with different shapes (the fixed scratch keeps the
+previous call's contents, which must not leak into the next result) its
+output must match the fp64 oracle on the same inputs within the parity
+tolerances of the other tests (|O - O_ref| <= 1e-2, |LSE - LSE_ref| <= 1e-3)
+and agree with fa_fwd_splitkv given a caller workspace.  The call must leave
+the device's stream-ordered memory pool untouched (the allocating entry point
+is the positive control), the automatic split count must fit the fixed
+scratch, and an explicit split count that does not fit must be refused.
+This file is collected last so that a stop at the first failure has run
+every other test already.
 """
 import ctypes
 
@@ -15,6 +19,7 @@ import pytest
 import torch
 
 import exact_attention_114_b200 as fa
+import oracle
 import synth
 from tests import gpu_parity as G
 
@@ -34,25 +39,88 @@ def _with_workspace(xd, w, splits):
                              num_splits=splits, workspace=ws if n else None)
 
 
-def test_noalloc_matches_workspace_entry_point_two_calls():
+class DefaultPool:
+    """High-water mark of used bytes in the current device's default
+    stream-ordered memory pool (the pool cudaMallocAsync draws from), read and
+    reset through the driver API."""
+    USED_MEM_CURRENT, USED_MEM_HIGH = 7, 8   # CUmemPool_attribute
+
+    def __init__(self):
+        self.cu = ctypes.CDLL("libcuda.so.1")
+        dev = ctypes.c_int()
+        assert self.cu.cuCtxGetDevice(ctypes.byref(dev)) == 0
+        self.pool = ctypes.c_void_p()
+        assert self.cu.cuDeviceGetDefaultMemPool(ctypes.byref(self.pool), dev) == 0
+
+    def _get(self, attr):
+        v = ctypes.c_uint64()
+        assert self.cu.cuMemPoolGetAttribute(self.pool, attr, ctypes.byref(v)) == 0
+        return v.value
+
+    def reset_high(self):
+        zero = ctypes.c_uint64(0)   # the only value the high-water mark can be set to
+        assert self.cu.cuMemPoolSetAttribute(self.pool, self.USED_MEM_HIGH, ctypes.byref(zero)) == 0
+
+    def used_high(self):
+        return self._get(self.USED_MEM_HIGH)
+
+    def used_current(self):
+        return self._get(self.USED_MEM_CURRENT)
+
+
+def test_noalloc_matches_oracle_and_workspace_entry_point_two_calls():
     for w, splits in CASES:
         assert 0 < fa.fa_fwd_splitkv_workspace_size(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, splits) \
             <= fa.NOALLOC_SCRATCH_BYTES
-    inputs = [G.to_gpu(synth.make_inputs(w)) for w, _ in CASES]
-    outs = []
-    for (w, splits), xd in zip(CASES, inputs):   # two calls in a row
-        o = torch.empty_like(xd["q"])
-        lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device="cuda")
+    hosts = [synth.make_inputs(w) for w, _ in CASES]
+    inputs = [G.to_gpu(x) for x in hosts]
+    outs = [(torch.empty_like(xd["q"]), torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device="cuda"))
+            for (w, _), xd in zip(CASES, inputs)]
+    torch.cuda.synchronize()
+    pool = DefaultPool()
+    base = pool.used_current()
+    pool.reset_high()
+    for (w, splits), xd, (o, lse) in zip(CASES, inputs, outs):   # two calls in a row
         fa.fa_fwd_splitkv_noalloc(xd["q"], xd["k"], xd["v"], o, lse, causal=w.causal,
                                   scale=w.scale, num_splits=splits)
-        outs.append((o, lse))
+    torch.cuda.synchronize()
+    assert pool.used_high() <= base, "the no-allocation call drew memory from the default pool"
+    fa.fa_check_device_status()
+    for (w, splits), x, xd, (o, lse) in zip(CASES, hosts, inputs, outs):
+        o_ref, lse_ref = oracle.fwd(x["q"], x["k"], x["v"], w.scale, w.causal)
+        G.assert_o(G.f64(o), o_ref, what="O (no-alloc vs oracle)")
+        G.assert_lse(G.f64(lse), lse_ref)
+        o_ws, lse_ws = _with_workspace(xd, w, splits)
+        torch.cuda.synchronize()
+        G.assert_o(G.f64(o), G.f64(o_ws), what="O (no-alloc vs workspace call)")
+        G.assert_lse(G.f64(lse), G.f64(lse_ws))
+    # positive control: the same call without a workspace allocates from the pool
+    w, splits = CASES[0]
+    xd = inputs[0]
+    pool.reset_high()
+    fa.fa_fwd_splitkv(xd["q"], xd["k"], xd["v"], causal=w.causal, scale=w.scale, num_splits=splits)
+    torch.cuda.synchronize()
+    assert pool.used_high() > base, "the pool's high-water mark did not see an allocating call"
+
+
+def test_noalloc_automatic_split_count_fits_the_fixed_scratch():
+    """A shape whose automatic split count would overflow the fixed scratch
+    runs with fewer splits and still matches the oracle on sampled rows."""
+    # on 148 SMs the automatic choice for this shape is 19 splits, 8.8 MB of partials
+    w = synth.Workload("decode_big", 7, 32, 8, 4, 8192, 128, True, 4343, backward=False)
+    assert fa.fa_fwd_splitkv_workspace_size(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, 0) \
+        > fa.NOALLOC_SCRATCH_BYTES
+    x = synth.make_inputs(w)
+    xd = G.to_gpu(x)
+    o = torch.empty_like(xd["q"])
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device="cuda")
+    fa.fa_fwd_splitkv_noalloc(xd["q"], xd["k"], xd["v"], o, lse, causal=True, scale=w.scale)
     torch.cuda.synchronize()
     fa.fa_check_device_status()
-    for (w, splits), xd, (o, lse) in zip(CASES, inputs, outs):
-        o_ref, lse_ref = _with_workspace(xd, w, splits)
-        torch.cuda.synchronize()
-        G.assert_o(G.f64(o), G.f64(o_ref), what="O (no-alloc vs workspace)")
-        G.assert_lse(G.f64(lse), G.f64(lse_ref))
+    rows = G.sample_rows(w, n_random=24)
+    o_ref, lse_ref = oracle.fwd(x["q"], x["k"], x["v"], w.scale, True, rows=rows)
+    G.assert_o(G.f64(o).reshape(-1, w.d)[rows], o_ref, what="O (no-alloc, automatic splits)")
+    G.assert_lse(G.f64(lse).reshape(-1)[rows], lse_ref)
 
 
 def test_noalloc_refuses_shapes_beyond_the_fixed_scratch():
