@@ -440,8 +440,11 @@ def run_libfa(args, rank, world, local):
     # long MHA one (B=2, H=32, N=4096, d=128, causal, every 64th query row x8) held
     # to the same bar, and the d = 64 MHA one (B=4, H=16, N=1024), causal and not
     other = {}
-    for name in ("mha_4k_long", "mha_1k", "mha_1k_noncausal"):
-        wo = synth.WORKLOADS[name].with_(seed=rank_seed(synth.WORKLOADS[name].seed, rank))
+    # the step workload's shape at head size 256 (the feature-split backward)
+    extra = {"gqa_8k_d256": synth.WORKLOADS[STEP_WORKLOAD].with_(name="gqa_8k_d256", d=256)}
+    for name in ("mha_4k_long", "mha_1k", "mha_1k_noncausal", "gqa_8k_d256"):
+        base = extra.get(name) or synth.WORKLOADS[name]
+        wo = base.with_(seed=rank_seed(base.seed, rank))
         xo = {k_: v_.to(dev) for k_, v_ in synth.make_inputs(wo).items()}
         oo = torch.empty_like(xo["q"])
         lo = torch.empty((wo.B, wo.Hq, wo.Nq), dtype=torch.float32, device=dev)
@@ -462,7 +465,7 @@ def run_libfa(args, rank, world, local):
         torch.cuda.synchronize()
         f_ms = statistics.median(timed(fo, max(10, args.steps)))
         b_ms = statistics.median(timed(bo, max(10, args.steps)))
-        other[name] = {"workload": f"B={wo.B}, H={wo.Hq}, N={wo.Nq}, d={wo.d}, "
+        other[name] = {"workload": f"B={wo.B}, Hq={wo.Hq}, Hkv={wo.Hkv}, N={wo.Nq}, d={wo.d}, "
                                    f"{'causal' if wo.causal else 'non-causal'}",
                        "fwd_ms": f_ms, "fwd_tflops": wo.fwd_flops() / (f_ms * 1e-3) / 1e12,
                        "bwd_ms": b_ms, "bwd_tflops": wo.bwd_flops() / (b_ms * 1e-3) / 1e12}
@@ -620,6 +623,9 @@ PROFILE_CASES = {
     "bwd": ("gqa_8k", dict(Nq=4096, Nk=4096)),
     "decode": ("gqa_decode", dict(B=16)),
     "fwd_fp8": ("gqa_8k", dict(Nq=4096, Nk=4096)),
+    # head size 256: Q and O 64 MiB each, K and V 16 MiB each
+    "fwd_d256": ("gqa_8k", dict(Nq=4096, Nk=4096, d=256)),
+    "bwd_d256": ("gqa_8k", dict(Nq=4096, Nk=4096, d=256)),
 }
 
 
@@ -636,7 +642,7 @@ def run_profile(which: str, launches: int = 3) -> int:
         DS = synth.FP8_DESCALE
         x = {k: v.cuda() for k, v in synth.make_inputs_fp8(w).items()}
     for _ in range(launches):
-        if which == "bwd":
+        if which in ("bwd", "bwd_d256"):
             fa.fa_bwd(x["q"], x["k"], x["v"], o, x["dout"], lse, causal=w.causal, scale=w.scale)
         elif which == "fwd_fp8":
             fa.fa_fwd_fp8(x["q"], x["k"], x["v"], DS["q"], DS["k"], DS["v"], o, lse, causal=w.causal,

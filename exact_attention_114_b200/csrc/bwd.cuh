@@ -35,6 +35,18 @@
 //              for the other's previous step.
 // Tensor memory (512 columns): dK | dV (d each) | S^T/P^T x2 (64 each) | dP^T 64
 // | dQ^T 64  (for d = 64 the last 128 columns are unused).
+//
+// Head size 256: dK and dV of a 128-key block would fill all 512 columns, so
+// the features are split in two halves.  A CTA owns (key block, kv head,
+// feature half fh): S^T and dP^T still contract over all 256 features (the
+// two CTAs of a key block both recompute them), while dV, dK and dQ^T cover
+// only features 128 fh .. 128 fh + 127, with the tensor-memory layout of
+// d = 128.  K and V of the block take 128 KB of shared memory, which leaves
+// room for a single Q / dO step slot and no dQ staging tile: the drain warps
+// add dQ^T to the accumulator straight from registers with fp32 reductions
+// (one 128-byte row segment per warp instruction), and the MMA warp issues a
+// step's gradient MMAs before the next step's S^T / dP^T (whose Q and dO can
+// only land once the gradient MMAs have read the slot).
 #pragma once
 
 #include "sm100.cuh"
@@ -59,6 +71,11 @@ __device__ __forceinline__ void bulk_reduce_add_f32(float* dst, const void* src,
     asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
                  "r"(smem_u32(src)), "r"(bytes)
                  : "memory");
+}
+
+__device__ __forceinline__ void red_add_f32(float* dst, float x)
+{
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(dst), "f"(x) : "memory");
 }
 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
@@ -87,15 +104,29 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdParams p)
         if (row >= total)
             continue;
         float* acc = p.dq_acc + (size_t)row * D + lane * E;
-        if constexpr (E == 4)
+        if constexpr (E == 8) {
+            reinterpret_cast<float4*>(acc)[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+            reinterpret_cast<float4*>(acc)[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else if constexpr (E == 4) {
             *reinterpret_cast<float4*>(acc) = make_float4(0.f, 0.f, 0.f, 0.f);
-        else
+        } else {
             *reinterpret_cast<float2*>(acc) = make_float2(0.f, 0.f);
+        }
         const int bh = row / p.Nq_pad, i = row - bh * p.Nq_pad;
         if (i >= p.Nq || lane * E >= p.d_io)   // padded row, or padded columns of a narrower head
             continue;
         const size_t src = ((size_t)bh * p.Nq + i) * p.d_io + lane * E;
-        if constexpr (E == 4) {
+        if constexpr (E == 8) {
+            const uint4 a = *reinterpret_cast<const uint4*>(po + src);
+            const uint4 c = *reinterpret_cast<const uint4*>(pd + src);
+            const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 x = Elt<T>::unpack(aw[e]), y = Elt<T>::unpack(cw[e]);
+                s[r] = fmaf(x.x, y.x, s[r]);
+                s[r] = fmaf(x.y, y.y, s[r]);
+            }
+        } else if constexpr (E == 4) {
             const uint2 a = *reinterpret_cast<const uint2*>(po + src);
             const uint2 c = *reinterpret_cast<const uint2*>(pd + src);
             const float2 x0 = Elt<T>::unpack(a.x), y0 = Elt<T>::unpack(c.x);
@@ -142,11 +173,11 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdParams p)
 template <int D, typename T = __nv_bfloat16>
 __global__ void __launch_bounds__(256) bwd_post_kernel(BwdParams p)
 {
-    const int lane = threadIdx.x & 31, c = lane * 4;
-    if (c >= p.d_io)
-        return;
+    const int lane = threadIdx.x & 31;
     const long long BH = (long long)p.B * p.Hq;
     const int i_step = (int)gridDim.x * 16;
+#pragma unroll 1
+    for (int c = lane * 4; c < p.d_io; c += 128)   // one pass per 128 columns
     for (long long bh = blockIdx.y; bh < BH; bh += gridDim.y) {
         const float* acc = p.dq_acc + bh * p.Nq_pad * D + c;
         T* dq = static_cast<T*>(p.dq) + bh * p.Nq * p.d_io + c;
@@ -177,12 +208,15 @@ struct BwdCfg {
     static constexpr int kThreads = 384;
     // registers per thread after the split: 128 x (208 + 112 + 144) <= 384 x 168
     static constexpr uint32_t kRegsDS = 208, kRegsDQ = 112, kRegsOther = 144;
+    static constexpr int kFeatSplit = (D == 256) ? 2 : 1;   // CTAs per (key block, kv head)
+    static constexpr int kDO = D / kFeatSplit;               // dK / dV / dQ features of one CTA
+    static constexpr bool kStagedDQ = (D <= 128);            // dQ through a shared staging tile
     static constexpr int kKPanel = 128 * 128;          // 128 keys x 64 bf16
     static constexpr int kKTile = (D / 64) * kKPanel;  // K or V block
     static constexpr int kQPanel = 64 * 128;           // 64 rows x 64 bf16
     static constexpr int kQTile = (D / 64) * kQPanel;  // Q or dO block
     static constexpr int kSlot = 2 * kQTile + 1024;    // Q, dO, -lse_log2[64], -delta[64] (1 KB-aligned)
-    static constexpr int kSlots = 3;                   // step slots in flight (TMA latency cover)
+    static constexpr int kSlots = (D == 256) ? 1 : 3;  // step slots in flight (TMA latency cover)
     static constexpr int kPTile = 128 * 128;           // dS^T: 128 keys x 64 q bf16
     static constexpr int kOffK = 0;
     static constexpr int kOffV = kOffK + kKTile;
@@ -190,11 +224,18 @@ struct BwdCfg {
     static constexpr int kOffSlots = kOffZero + (D == 64 ? kKPanel : 0);
     static constexpr int kOffDS = kOffSlots + kSlots * kSlot;       // dS^T, two buffers
     static constexpr int kOffDQ = kOffDS + 2 * kPTile;              // fp32 [32][D] staging (half a step)
-    static constexpr int kOffBar = kOffDQ + 32 * D * 4;
+    static constexpr int kOffBar = kOffDQ + (kStagedDQ ? 32 * D * 4 : 0);
     static constexpr int kSmemBytes = kOffBar + 256 + 1024;
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kColDK = 0, kColDV = D, kColS = 2 * D, kColDP = 2 * D + 128,
-                              kColDQ = 2 * D + 192;
+    static constexpr uint32_t kColDK = 0, kColDV = kDO, kColS = 2 * kDO, kColDP = 2 * kDO + 128,
+                              kColDQ = 2 * kDO + 192;
+    static_assert(kSmemBytes <= 232448, "shared memory per block");
+    // setmaxnreg: the launch gives every thread 168 registers (384 threads, one
+    // block per SM); .dec may only lower a warpgroup's count and .inc only raise
+    // it, and the three counts must add up to the launch's total
+    static_assert(kRegsDQ <= 168 && kRegsOther <= 168 && kRegsDS >= 168, "register split direction");
+    static_assert(kRegsDS + kRegsDQ + kRegsOther <= 3 * 168, "register split total");
+    static_assert(kColDQ + 64 <= kTmemCols || D == 64, "tensor memory columns");
 };
 
 __device__ __forceinline__ void bwd_q_range(const BwdParams& p, int kb, int& qb0, int& nqb)
@@ -246,8 +287,10 @@ __global__ void __launch_bounds__(384, 1)
 
     const int warp = warp_id(), lane = lane_id();
     const int n_kb = (p.Nk + 127) / 128;
-    const int kb = (int)blockIdx.x / (p.B * p.Hkv);   // small key blocks (most work) first
-    const int kvh = (int)blockIdx.x % (p.B * p.Hkv);
+    const int units = p.B * p.Hkv * C::kFeatSplit;
+    const int kb = (int)blockIdx.x / units;   // small key blocks (most work) first
+    const int kvh = ((int)blockIdx.x % units) / C::kFeatSplit;
+    const int fh = ((int)blockIdx.x % units) % C::kFeatSplit;   // feature half (head size 256)
     const int b = kvh / p.Hkv, hk = kvh % p.Hkv;
     int qb0, nqb;
     bwd_q_range(p, kb, qb0, nqb);
@@ -342,9 +385,9 @@ __global__ void __launch_bounds__(384, 1)
         // (the whole warp runs this loop; one elected lane issues each MMA)
         {
             constexpr uint32_t fmt = Elt<T>::kMmaFmt;
-            const uint32_t id_sdp = idesc_f16kind(fmt, 128, 64, false, false);   // S^T, dP^T
-            const uint32_t id_grad = idesc_f16kind(fmt, 128, D, false, true);    // dV, dK
-            const uint32_t id_dq = idesc_f16kind(fmt, 128, 64, true, true);      // dQ^T
+            const uint32_t id_sdp = idesc_f16kind(fmt, 128, 64, false, false);      // S^T, dP^T
+            const uint32_t id_grad = idesc_f16kind(fmt, 128, C::kDO, false, true);  // dV, dK
+            const uint32_t id_dq = idesc_f16kind(fmt, 128, 64, true, true);         // dQ^T
             const uint32_t tDK = tmem + C::kColDK, tDV = tmem + C::kColDV, tS = tmem + C::kColS,
                            tDP = tmem + C::kColDP, tDQ = tmem + C::kColDQ;
             // base descriptors; a byte offset `o` inside an operand is added as o >> 4
@@ -352,9 +395,13 @@ __global__ void __launch_bounds__(384, 1)
             const uint64_t dK_k = sdesc_sw128(smem_u32(smem + C::kOffK), 16, 1024);      // K as K-major A
             const uint64_t dV_k = sdesc_sw128(smem_u32(smem + C::kOffV), 16, 1024);      // V as K-major A
             // K^T as the M = 128 (feature) MN-major operand of dQ^T: the second 64-feature
-            // panel is 16 KB on for d = 128, the zero panel for d = 64
-            const uint32_t lbo_kt = (D == 128) ? (uint32_t)C::kKPanel : (uint32_t)(C::kOffZero - C::kOffK);
-            const uint64_t dK_mn = sdesc_sw128(smem_u32(smem + C::kOffK), lbo_kt, 1024);
+            // panel is 16 KB on for d = 128 (and for the feature half of d = 256), the
+            // zero panel for d = 64
+            const uint32_t lbo_kt = (D >= 128) ? (uint32_t)C::kKPanel : (uint32_t)(C::kOffZero - C::kOffK);
+            const uint64_t dK_mn =
+                sdesc_sw128(smem_u32(smem + C::kOffK + fh * 2 * C::kKPanel), lbo_kt, 1024);
+            // the feature half's two panels of a Q / dO tile (the B operands of dK / dV)
+            const uint32_t fo = (uint32_t)(fh * 2 * C::kQPanel);
             const uint64_t dSlot_k = sdesc_sw128(smem_u32(smem + C::kOffSlots), 16, 1024);   // Q / dO K-major
             const uint64_t dSlot_mn = sdesc_sw128(smem_u32(smem + C::kOffSlots), C::kQPanel, 1024);
             const uint64_t dDS_mn = sdesc_sw128(smem_u32(smem + C::kOffDS), C::kPTile, 1024);
@@ -363,13 +410,14 @@ __global__ void __launch_bounds__(384, 1)
             auto issue_sdp = [&](int it) {
                 const uint32_t so = (uint32_t)((it % C::kSlots) * C::kSlot);
                 const uint32_t tSb = tS + (uint32_t)(64 * (it & 1));
-#pragma unroll
+                constexpr int kUnroll = D / 16 <= 8 ? D / 16 : 4;   // fewer live descriptors at d = 256
+#pragma unroll kUnroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ok_ = (uint32_t)((kk >> 2) * C::kKPanel + (kk & 3) * 32);
                     const uint32_t oq = (uint32_t)((kk >> 2) * C::kQPanel + (kk & 3) * 32);
                     mma_ss_w(tSb, dK_k + off(ok_), dSlot_k + off(so + oq), id_sdp, kk > 0 ? 1u : 0u);
                 }
-#pragma unroll
+#pragma unroll kUnroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ok_ = (uint32_t)((kk >> 2) * C::kKPanel + (kk & 3) * 32);
                     const uint32_t oq = (uint32_t)((kk >> 2) * C::kQPanel + (kk & 3) * 32);
@@ -378,6 +426,17 @@ __global__ void __launch_bounds__(384, 1)
                 mma_commit_w(bar_sdp);
             };
 
+            // step it's S^T / dP^T are in registers: the next step's may overwrite dP^T
+            // and the other S^T buffer once its Q / dO have landed
+            auto next_sdp = [&](int it) -> bool {
+                const int in = it + 1;
+                if (!mbar_wait_w(bar_sdp_read, (uint32_t)(it & 1), abort_flag))
+                    return false;
+                if (!mbar_wait_w(&bar_full[in % C::kSlots], (uint32_t)((in / C::kSlots) & 1), abort_flag))
+                    return false;
+                issue_sdp(in);
+                return true;
+            };
             bool ok = mbar_wait_w(bar_kv, 0, abort_flag);
             if (ok && n_it > 0) {
                 ok = mbar_wait_w(&bar_full[0], 0, abort_flag);
@@ -385,16 +444,10 @@ __global__ void __launch_bounds__(384, 1)
                     issue_sdp(0);
             }
             for (int it = 0; ok && it < n_it; ++it) {
-                if (it + 1 < n_it) {
-                    // step it's S^T / dP^T are in registers: the next step's may overwrite
-                    // dP^T and the other S^T buffer
-                    const int in = it + 1;
-                    if (!(ok = mbar_wait_w(bar_sdp_read, (uint32_t)(it & 1), abort_flag)))
-                        break;
-                    if (!(ok = mbar_wait_w(&bar_full[in % C::kSlots], (uint32_t)((in / C::kSlots) & 1), abort_flag)))
-                        break;
-                    issue_sdp(in);
-                }
+                // with one step slot the next step's Q / dO land only after this step's
+                // gradient MMAs have read the slot, so its S^T / dP^T come after them
+                if (C::kSlots > 1 && it + 1 < n_it && !(ok = next_sdp(it)))
+                    break;
                 if (!(ok = mbar_wait_w(&bar_ds[it & 1], (uint32_t)((it >> 1) & 1), abort_flag)))
                     break;
                 tc_fence_after();
@@ -410,14 +463,17 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                    mma_ts_w(tDV, tP + (uint32_t)(kk * 8), dSlot_mn + off(so + C::kQTile + kk * 2048), id_grad, acc);
-                    mma_ts_w(tDK, tP + 32u + (uint32_t)(kk * 8), dSlot_mn + off(so + kk * 2048), id_grad, acc);
+                    mma_ts_w(tDV, tP + (uint32_t)(kk * 8), dSlot_mn + off(so + C::kQTile + fo + kk * 2048), id_grad,
+                             acc);
+                    mma_ts_w(tDK, tP + 32u + (uint32_t)(kk * 8), dSlot_mn + off(so + fo + kk * 2048), id_grad, acc);
                 }
                 // dQ^T = K^T dS^T   (K dimension = 128 keys)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ss_w(tDQ, dK_mn + off(kk * 2048), dDS_mn + off(dso + kk * 2048), id_dq, kk > 0 ? 1u : 0u);
                 mma_commit_w(&bar_gdone[it & 3]);
+                if (C::kSlots == 1 && it + 1 < n_it && !(ok = next_sdp(it)))
+                    break;
             }
             mma_commit_w(bar_final);
             if (!ok)
@@ -518,10 +574,11 @@ __global__ void __launch_bounds__(384, 1)
             const bool key_ok = key < p.Nk;
             const int d_io = p.d_io;
 #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                if (c0 >= d_io)   // padded columns of a narrower head
+            for (int c0 = 0; c0 < C::kDO; c0 += 32) {
+                const int col = fh * C::kDO + c0;   // feature of the tensors in memory
+                if (col >= d_io)   // padded columns of a narrower head
                     break;
-                const size_t krow = ((size_t)kvh * p.Nk + key) * d_io;
+                const size_t krow = ((size_t)kvh * p.Nk + key) * d_io + fh * C::kDO;
                 uint32_t a[32], v[32];
                 if (n_it > 0) {
                     tmem_ld32(tmem + lane_off + C::kColDK + c0, a);
@@ -566,6 +623,29 @@ __global__ void __launch_bounds__(384, 1)
             if (!ok)
                 break;
             tc_fence_after();
+            if constexpr (!C::kStagedDQ) {
+                // fp32 reductions straight from registers: for query row c the 32 lanes
+                // of a warp add 32 consecutive features, one 128-byte segment per
+                // instruction (this CTA's feature half of the accumulator row); the
+                // 64 query columns are read in two halves of 32
+                float* dst = p.dq_acc + ((size_t)(b * p.Hq + h) * p.Nq_pad + (size_t)qb * 64) * D +
+                             fh * C::kDO + f;
+                uint32_t a[32];
+#pragma unroll
+                for (int hq = 0; hq < 2; ++hq) {
+                    tmem_ld32(tDQ + (uint32_t)(32 * hq), a);
+                    if (hq == 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0)
+                            mbar_arrive(bar_dqfree);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        red_add_f32(dst + (size_t)(32 * hq + c) * D, __uint_as_float(a[c]));
+                }
+                continue;
+            }
             uint32_t a[64];
             tmem_ld64(tDQ, a);
             tc_fence_before();

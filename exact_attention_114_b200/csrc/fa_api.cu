@@ -596,7 +596,7 @@ fa_status_t launch_bwd(const fa::BwdParams& p, const void* q, const void* k, con
     if ((st = make_map(&mv, v, p.d_io, p.Nk, (uint64_t)p.B * p.Hkv, 128, dt)) != FA_OK) return st;
     auto kern = fa::bwd_main_kernel<D, CAUSAL, T>;
     if ((st = ensure_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes)) != FA_OK) return st;
-    const long long grid = (long long)((p.Nk + 127) / 128) * p.B * p.Hkv;
+    const long long grid = (long long)((p.Nk + 127) / 128) * p.B * p.Hkv * C::kFeatSplit;
     kern<<<(unsigned)grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mdo, p);
     if ((st = check_launch("bwd_main_kernel launch")) != FA_OK) return st;
 
@@ -605,6 +605,17 @@ fa_status_t launch_bwd(const fa::BwdParams& p, const void* q, const void* k, con
                      (unsigned)std::max<long long>(1, std::min<long long>((long long)p.B * p.Hq, 65535)));
     fa::bwd_post_kernel<D, T><<<pgrid, 256, 0, stream>>>(p);
     return check_launch("bwd_post_kernel launch");
+}
+
+template <typename T>
+fa_status_t bwd_dispatch(const fa::BwdParams& p, const void* q, const void* k, const void* v, const void* dout,
+                         int kd, int causal, cudaStream_t s)
+{
+    if (kd == 256)
+        return causal ? launch_bwd<256, true, T>(p, q, k, v, dout, s) : launch_bwd<256, false, T>(p, q, k, v, dout, s);
+    if (kd == 128)
+        return causal ? launch_bwd<128, true, T>(p, q, k, v, dout, s) : launch_bwd<128, false, T>(p, q, k, v, dout, s);
+    return causal ? launch_bwd<64, true, T>(p, q, k, v, dout, s) : launch_bwd<64, false, T>(p, q, k, v, dout, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -969,7 +980,7 @@ fa_status_t fa_fwd_paged_ex(fa_dtype_t dtype, const void* q, const void* k_cache
 
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d)
 {
-    if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || Hq % Hkv != 0 || d < 1 || d > 128)
+    if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || Hq % Hkv != 0 || d < 1 || d > 256)
         return 0;
     return bwd_plan(B, Hq, Nq, d).total;
 }
@@ -991,10 +1002,6 @@ static fa_status_t bwd_entry(int dtype, const void* q, const void* k, const void
         return st;
     if ((st = check_shape(B, Hq, Hkv, Nq, Nk, d, scale, causal)) != FA_OK)
         return st;
-    if (d > 128) {
-        set_error("the backward takes d up to 128 (got %d)", d);
-        return FA_ERR_UNSUPPORTED;
-    }
     if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) {
         set_error("workspace is not 256-byte aligned");
         return FA_ERR_INVALID_ARGUMENT;
@@ -1038,21 +1045,8 @@ static fa_status_t bwd_entry(int dtype, const void* q, const void* k, const void
     p.causal = causal;
     p.scale = scale;
     p.scale_log2 = scale * kLog2e;
-    if (dtype == FA_DTYPE_FP16) {
-        if (kernel_d(d) == 128)
-            st = causal ? launch_bwd<128, true, __half>(p, q, k, v, dout, s)
-                        : launch_bwd<128, false, __half>(p, q, k, v, dout, s);
-        else
-            st = causal ? launch_bwd<64, true, __half>(p, q, k, v, dout, s)
-                        : launch_bwd<64, false, __half>(p, q, k, v, dout, s);
-    } else {
-        if (kernel_d(d) == 128)
-            st = causal ? launch_bwd<128, true, __nv_bfloat16>(p, q, k, v, dout, s)
-                        : launch_bwd<128, false, __nv_bfloat16>(p, q, k, v, dout, s);
-        else
-            st = causal ? launch_bwd<64, true, __nv_bfloat16>(p, q, k, v, dout, s)
-                        : launch_bwd<64, false, __nv_bfloat16>(p, q, k, v, dout, s);
-    }
+    st = dtype == FA_DTYPE_FP16 ? bwd_dispatch<__half>(p, q, k, v, dout, kernel_d(d), causal, s)
+                                : bwd_dispatch<__nv_bfloat16>(p, q, k, v, dout, kernel_d(d), causal, s);
     if (owned) {
         cudaError_t e = cudaFreeAsync(ws, s);
         if (e != cudaSuccess && st == FA_OK)

@@ -75,6 +75,10 @@ struct FwdCfg {
     static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + barriers + alignment slack
     static constexpr uint32_t kTmemCols = 512;
     static_assert(!F8 || D == 128, "the e4m3 kernel is built for d = 128");
+    // setmaxnreg: 168 registers per thread at launch (384 threads); the two softmax
+    // warpgroups raise theirs, the third lowers its, within the launch's total
+    static_assert(kRegsSoftmax >= 168 && kRegsOther <= 168 && 2 * kRegsSoftmax + kRegsOther <= 3 * 168,
+                  "register split");
     static_assert(kTiles == 2 || 128 + D <= (int)kTmemCols, "one tile: S and O must fit in TMEM");
 };
 

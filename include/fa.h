@@ -20,12 +20,13 @@
  *    hold bf16 (fp16 through the *_ex calls), lse holds fp32 (natural log of
  *    the scaled scores).
  *  - Every tensor pointer is a DEVICE pointer, non-NULL and 16-byte aligned.
- *  - d is a multiple of 32 up to 256 for the forward and up to 128 for the
- *    backward (page "AI infra 一层全看懂(五) Flash Attention", §五, gives 64 to
- *    128 as the usual head dimension; other sizes run on the 64, 128 or 256
- *    kernels with the missing columns zero-filled on chip; d > 128 uses one
- *    128-row query tile per CTA).  The split-KV and paged calls take d up to
- *    128, the e4m3 call d = 128 only.  Hq must be a multiple of Hkv.
+ *  - d is a multiple of 32 up to 256 (page "AI infra 一层全看懂(五) Flash
+ *    Attention", §五, gives 64 to 128 as the usual head dimension; other sizes
+ *    run on the 64, 128 or 256 kernels with the missing columns zero-filled on
+ *    chip; d > 128 uses one 128-row query tile per CTA in the forward and two
+ *    CTAs per key block, one per half of the features, in the backward).  The
+ *    split-KV and paged calls take d up to 128, the e4m3 call d = 128 only.
+ *    Hq must be a multiple of Hkv.
  *    B, Hq, Hkv, Nq, Nk >= 1.
  *  - causal is 0 or 1.  With causal = 1, key j is visible to query i iff
  *    j <= i + (Nk - Nq) (the mask is aligned to the bottom-right corner; for
@@ -59,7 +60,7 @@ extern "C" {
 typedef enum {
     FA_OK = 0,
     FA_ERR_INVALID_ARGUMENT = 1, /* NULL / misaligned pointer, bad size or flag */
-    FA_ERR_UNSUPPORTED = 2,      /* valid but not implemented (e.g. d = 80, or d > 128 in the backward) */
+    FA_ERR_UNSUPPORTED = 2,      /* valid but not implemented (e.g. d = 80) */
     FA_ERR_WORKSPACE = 3,        /* workspace given but smaller than required */
     FA_ERR_CUDA = 4,             /* a CUDA runtime / driver call failed */
     FA_ERR_TIMEOUT = 5,          /* a bounded device wait ran out */
@@ -244,6 +245,9 @@ fa_status_t fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, 
  *   workspace: device scratch of at least fa_bwd_workspace_size(...) bytes,
  *   256-byte aligned (it holds D = rowsum(dout * o) and the fp32 dq
  *   accumulator); NULL makes the call allocate it stream-ordered.
+ *   For d > 128 the features are split in two halves: each key block is
+ *   handled by two CTAs that both recompute S and dP over all d features and
+ *   each accumulate their half of dk, dv and dq.
  */
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d);
 fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o,

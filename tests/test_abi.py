@@ -85,8 +85,10 @@ def test_bwd_rejects_bad_arguments():
         bad[i] = None
         assert call(bad) == fa.FA_ERR_INVALID_ARGUMENT
     assert call(args, d=80) == fa.FA_ERR_UNSUPPORTED
-    assert call(args, d=256) == fa.FA_ERR_UNSUPPORTED    # forward only at d > 128
-    assert fa.fa_bwd_workspace_size(1, 2, 1, 8, 8, 256) == 0
+    assert call(args, d=288) == fa.FA_ERR_UNSUPPORTED    # head sizes stop at 256
+    assert fa.fa_bwd_workspace_size(1, 2, 1, 8, 8, 288) == 0
+    # d = 256: D and -LSE rows (64 padded rows each) and the fp32 accumulator, 256 wide
+    assert fa.fa_bwd_workspace_size(1, 2, 1, 8, 8, 256) == 2 * 512 + 2 * 64 * 256 * 4
     # a workspace that is too small is refused before any launch
     need = fa.fa_bwd_workspace_size(1, 2, 1, 8, 8, 128)
     assert call(args, ws=ctypes.c_void_p(0x100000), ws_bytes=need - 1) == fa.FA_ERR_WORKSPACE

@@ -44,8 +44,6 @@ def test_forward_backward_stay_inside(shape):
     torch.cuda.synchronize()
     fa.fa_check_device_status()
     assert o.intact() and lse.intact()
-    if d > 128:
-        return
     g = [Guarded(tuple(x[n].shape), torch.bfloat16) for n in ("q", "k", "v")]
     ws = Guarded((fa.fa_bwd_workspace_size(B, Hq, Hkv, Nq, Nk, d),), torch.uint8)
     fa.fa_bwd(x["q"], x["k"], x["v"], o.t, x["dout"], lse.t, g[0].t, g[1].t, g[2].t, causal=causal,

@@ -1,7 +1,9 @@
 """GPU parity for head dims other than 64 and 128 against the oracle: 32 and 96
-(on the 64 and 128 kernels with the missing columns zero-filled by TMA; forward
-and backward) and 160 .. 256 (the one-tile forward kernel; the backward takes
-d <= 128).  Tails around the tiles, GQA, causal and not."""
+(on the 64 and 128 kernels with the missing columns zero-filled by TMA) and
+160 .. 256 (the one-tile forward kernel and the feature-split d = 256
+backward, whose two CTAs per key block each own half of dK, dV and dQ);
+forward and backward.  Tails around the tiles, GQA, causal and not."""
+import numpy as np
 import pytest
 import torch
 
@@ -23,6 +25,16 @@ SHAPES = [
     (1, 2, 2, 333, 200, 96, True),
     (1, 8, 1, 70, 640, 96, False),
     (2, 2, 2, 513, 513, 96, True),
+    (1, 2, 1, 1, 1, 256, False),
+    (1, 2, 1, 63, 63, 256, True),
+    (2, 2, 1, 129, 129, 256, True),
+    (1, 4, 2, 300, 300, 256, True),
+    (1, 2, 2, 333, 200, 256, True),     # rows that see no key
+    (1, 2, 2, 200, 333, 256, False),
+    (1, 8, 1, 70, 640, 256, False),
+    (1, 4, 1, 257, 257, 192, True),
+    (1, 2, 2, 130, 130, 160, False),
+    (1, 4, 4, 128, 128, 224, True),
 ]
 DTYPES = [torch.bfloat16, torch.float16]
 
@@ -86,9 +98,11 @@ def test_large_headdim_forward(shape, dtype):
 
 
 def test_large_headdim_sampled_long():
-    """d = 256, N = 4096 causal GQA: sampled rows of a multi-wave launch."""
+    """d = 256, N = 4096 causal GQA: sampled rows of a multi-wave launch, and
+    the backward on sampled query rows (dQ) and on the heaviest and the last
+    keys (dK, dV) of the first and last kv heads."""
     w = synth.Workload("headdim_long", 1, 16, 4, 4096, 4096, 256, True, 6450)
-    x = synth.make_inputs(w, dout=False)
+    x = synth.make_inputs(w)
     xd = {k: v.cuda() for k, v in x.items()}
     o, lse = fa.fa_fwd(xd["q"], xd["k"], xd["v"], causal=True)
     torch.cuda.synchronize()
@@ -97,3 +111,11 @@ def test_large_headdim_sampled_long():
     o_ref, lse_ref = oracle.fwd(x["q"], x["k"], x["v"], w.scale, True, rows=rows)
     G.assert_o(G.f64(o).reshape(-1, w.d)[rows], o_ref)
     G.assert_lse(G.f64(lse).reshape(-1)[rows], lse_ref)
+    dq, dk, dv = G.gpu_backward(xd, o, lse, w)
+    rq = oracle.bwd_dq_rows(x["q"], x["k"], x["v"], x["dout"], w.scale, True, rows)
+    G.assert_grad(G.f64(dq).reshape(-1, w.d)[rows], rq, "dQ (sampled rows)")
+    keys = np.concatenate([G.sample_keys_heavy(w, kv_heads=(0, w.Hkv - 1)),
+                           G.sample_keys_cheap(w, kv_heads=(0, w.Hkv - 1))])
+    rk, rv = oracle.bwd_dkv_rows(x["q"], x["k"], x["v"], x["dout"], w.scale, True, keys)
+    G.assert_grad(G.f64(dk).reshape(-1, w.d)[keys], rk, "dK (sampled keys)")
+    G.assert_grad(G.f64(dv).reshape(-1, w.d)[keys], rv, "dV (sampled keys)")
