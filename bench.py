@@ -437,6 +437,32 @@ def run_libfa(args, rank, world, local):
     e2e_value = world * flops_step / (e2e_ms * 1e-3) / 1e12
     del bufs[1]
 
+    # The end-to-end step's own bound: the same bytes moved by plain copies alone (the
+    # step's four inputs host -> device, its three gradients device -> host, each
+    # direction on its own), against the compute time of the step.
+    def copy_ms(fn, reps=5):
+        fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    def h2d_only():
+        for kk in ("q", "k", "v", "dout"):
+            xd[kk].copy_(hx[kk], non_blocking=True)
+
+    def d2h_only():
+        hdq.copy_(dq, non_blocking=True)
+        hdk.copy_(dk, non_blocking=True)
+        hdv.copy_(dv, non_blocking=True)
+
+    h2d_ms, d2h_ms = copy_ms(h2d_only), copy_ms(d2h_only)
+    e2e_bound_ms = max(h2d_ms, d2h_ms, ms_step)
+
     # ---- the other training-shape workloads, reported beside the step workload: the
     # long MHA one (B=2, H=32, N=4096, d=128, causal, every 64th query row x8) held
     # to the same bar, and the d = 64 MHA one (B=4, H=16, N=1024), causal and not
@@ -603,7 +629,13 @@ def run_libfa(args, rank, world, local):
                 "mode": "double-buffered: step i+1 inputs copied in and step i-1 gradients copied out "
                         "while step i computes (three streams)",
                 "serial_ms_per_step": e2e_serial_ms,
-                "serial_value": world * flops_step / (e2e_serial_ms * 1e-3) / 1e12},
+                "serial_value": world * flops_step / (e2e_serial_ms * 1e-3) / 1e12,
+                "copy_bound": {"h2d_ms": h2d_ms, "h2d_gbs": h2d / (h2d_ms * 1e-3) / 1e9,
+                               "d2h_ms": d2h_ms, "d2h_gbs": d2h / (d2h_ms * 1e-3) / 1e9,
+                               "bound_ms_per_step": e2e_bound_ms,
+                               "frac": e2e_bound_ms / e2e_ms,
+                               "rule": "max(plain H2D copies, plain D2H copies, compute) of one step over the "
+                                       "double-buffered step time"}},
         "gpu_launches": args.steps * 4,  # timed region: fwd (1) + bwd (pre, main, post) per step
         "gpu_name": torch.cuda.get_device_name(dev),
         "clocks": clocks,
