@@ -61,7 +61,8 @@ def test_forward_config_sampled(name):
     rows = G.sample_rows(w, n_random=48)
     o_ref, lse_ref = oracle.fwd(x["q"], x["k"], x["v"], w.scale, w.causal, rows=rows)
     d = w.d
-    G.assert_o(G.f64(o).reshape(-1, d)[rows], o_ref)
+    G.assert_o(G.f64(o).reshape(-1, d)[rows], o_ref,
+               o_abs=G.o_abs_ref(x["q"], x["k"], x["v"], w.scale, w.causal, rows=rows))
     G.assert_lse(G.f64(lse).reshape(-1)[rows], lse_ref)
     # every output is finite and every row's LSE is finite (no fully masked rows here)
     assert torch.isfinite(o).all() and torch.isfinite(lse).all()

@@ -62,7 +62,8 @@ def run_case(B, Hq, Hkv, Nq, page_size, seq_lens, causal, splits, seed, d=128, f
             continue
         kb, vb = gather(kp, table[b], L, page_size), gather(vp, table[b], L, page_size)
         o_ref, lse_ref = oracle.fwd(q[b:b + 1], kb, vb, scale, causal)
-        G.assert_o(og, o_ref, what=f"O (sequence {b}, {L} keys)")
+        G.assert_o(og, o_ref, what=f"O (sequence {b}, {L} keys)",
+                   o_abs=G.o_abs_ref(q[b:b + 1], kb, vb, scale, causal))
         G.assert_lse(lg, lse_ref)
 
 

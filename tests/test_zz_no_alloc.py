@@ -88,7 +88,8 @@ def test_noalloc_matches_oracle_and_workspace_entry_point_two_calls():
     fa.fa_check_device_status()
     for (w, splits), x, xd, (o, lse) in zip(CASES, hosts, inputs, outs):
         o_ref, lse_ref = oracle.fwd(x["q"], x["k"], x["v"], w.scale, w.causal)
-        G.assert_o(G.f64(o), o_ref, what="O (no-alloc vs oracle)")
+        G.assert_o(G.f64(o), o_ref, what="O (no-alloc vs oracle)",
+                   o_abs=G.o_abs_ref(x["q"], x["k"], x["v"], w.scale, w.causal))
         G.assert_lse(G.f64(lse), lse_ref)
         o_ws, lse_ws = _with_workspace(xd, w, splits)
         torch.cuda.synchronize()
@@ -119,7 +120,8 @@ def test_noalloc_automatic_split_count_fits_the_fixed_scratch():
     fa.fa_check_device_status()
     rows = G.sample_rows(w, n_random=24)
     o_ref, lse_ref = oracle.fwd(x["q"], x["k"], x["v"], w.scale, True, rows=rows)
-    G.assert_o(G.f64(o).reshape(-1, w.d)[rows], o_ref, what="O (no-alloc, automatic splits)")
+    G.assert_o(G.f64(o).reshape(-1, w.d)[rows], o_ref, what="O (no-alloc, automatic splits)",
+               o_abs=G.o_abs_ref(x["q"], x["k"], x["v"], w.scale, True, rows=rows))
     G.assert_lse(G.f64(lse).reshape(-1)[rows], lse_ref)
 
 
