@@ -42,11 +42,13 @@
 // two CTAs of a key block both recompute them), while dV, dK and dQ^T cover
 // only features 128 fh .. 128 fh + 127, with the tensor-memory layout of
 // d = 128.  K and V of the block take 128 KB of shared memory, which leaves
-// room for a single Q / dO step slot and no dQ staging tile: the drain warps
-// add dQ^T to the accumulator straight from registers with fp32 reductions
-// (one 128-byte row segment per warp instruction), and the MMA warp issues a
-// step's gradient MMAs before the next step's S^T / dP^T (whose Q and dO can
-// only land once the gradient MMAs have read the slot).
+// room for two half slots of a step's Q / dO (32 KB each) and no dQ staging
+// tile: the drain warps add dQ^T to the accumulator straight from registers
+// with fp32 reductions (one 128-byte row segment per warp instruction).  Half
+// slot 0 holds the features this CTA does not own, which only S^T and dP^T
+// read: it is refilled for the next step as soon as those MMAs are done.  Half
+// slot 1 holds the owned features, which dV and dK read too: it is refilled
+// once they are done, while dQ^T and the next step's first-half MMAs run.
 #pragma once
 
 #include "sm100.cuh"
@@ -215,14 +217,20 @@ struct BwdCfg {
     static constexpr int kKTile = (D / 64) * kKPanel;  // K or V block
     static constexpr int kQPanel = 64 * 128;           // 64 rows x 64 bf16
     static constexpr int kQTile = (D / 64) * kQPanel;  // Q or dO block
-    static constexpr int kSlot = 2 * kQTile + 1024;    // Q, dO, -lse_log2[64], -delta[64] (1 KB-aligned)
-    static constexpr int kSlots = (D == 256) ? 1 : 3;  // step slots in flight (TMA latency cover)
+    // d = 256: a step's Q / dO in two half slots (the other CTA's features, then
+    // this CTA's own), with -lse_log2 / -delta in a separate pair of buffers
+    static constexpr bool kHalves = (D == 256);
+    static constexpr int kQTileH = kHalves ? 2 * kQPanel : kQTile;   // Q or dO part of one slot
+    static constexpr int kSlot = kHalves ? 2 * kQTileH                // Q, dO of one feature half
+                                         : 2 * kQTile + 1024;         // Q, dO, -lse_log2[64], -delta[64]
+    static constexpr int kSlots = kHalves ? 2 : 3;     // step slots in flight (TMA latency cover)
     static constexpr int kPTile = 128 * 128;           // dS^T: 128 keys x 64 q bf16
     static constexpr int kOffK = 0;
     static constexpr int kOffV = kOffK + kKTile;
     static constexpr int kOffZero = kOffV + kKTile;                 // zero panel (D = 64 only)
     static constexpr int kOffSlots = kOffZero + (D == 64 ? kKPanel : 0);
-    static constexpr int kOffDS = kOffSlots + kSlots * kSlot;       // dS^T, two buffers
+    static constexpr int kOffVec = kOffSlots + kSlots * kSlot;      // d = 256: [2][-lse_log2 64, -delta 64]
+    static constexpr int kOffDS = kOffVec + (kHalves ? 1024 : 0);   // dS^T, two buffers
     static constexpr int kOffDQ = kOffDS + 2 * kPTile;              // fp32 [32][D] staging (half a step)
     static constexpr int kOffBar = kOffDQ + (kStagedDQ ? 32 * D * 4 : 0);
     static constexpr int kSmemBytes = kOffBar + 256 + 1024;
@@ -283,6 +291,9 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* bar_final = bars + 15;    // all MMAs done
     uint64_t* bar_sdp_read = bars + 16; // S^T, dP^T of a step loaded into registers (count 4)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+    // d = 256: half slot 0 read by the step's S^T / dP^T MMAs, half slot 1 by its dV / dK MMAs
+    uint64_t* bar_h0free = bars + 18;
+    uint64_t* bar_h1free = bars + 19;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = warp_id(), lane = lane_id();
@@ -313,6 +324,8 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(&bar_gdone[i], 1);
         mbar_init(bar_dqfree, 4);
         mbar_init(bar_final, 1);
+        mbar_init(bar_h0free, 1);
+        mbar_init(bar_h1free, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -350,6 +363,60 @@ __global__ void __launch_bounds__(384, 1)
                 tma_load_3d(smem + C::kOffK + pn * C::kKPanel, &tmK, bar_kv, pn * 64, kb * 128, kvh);
                 tma_load_3d(smem + C::kOffV + pn * C::kKPanel, &tmV, bar_kv, pn * 64, kb * 128, kvh);
             }
+            if constexpr (C::kHalves) {
+                // half slot 0: the features of the other CTA of the pair, which only the
+                // step's S^T / dP^T read; half slot 1: this CTA's own features, which its
+                // dV / dK read too, plus the step's -lse_log2 / -delta.  Loads go out in
+                // the order their slots are freed: half 0 of step s + 1 before half 1 of s.
+                int issued0 = 0, issued1 = 0;
+                auto load_half = [&](int st, int hs) {
+                    int h, qb;
+                    step_coords(st, h, qb);
+                    const int bh = b * p.Hq + h;
+                    uint8_t* hslot = smem + C::kOffSlots + hs * C::kSlot;
+                    const int pn0 = 2 * (hs ? fh : 1 - fh);   // first 64-feature panel of the half
+                    mbar_arrive_expect_tx(&bar_full[hs], 2 * C::kQTileH + (hs ? 512 : 0));
+                    for (int j = 0; j < 2; ++j) {
+                        tma_load_3d(hslot + j * C::kQPanel, &tmQ, &bar_full[hs], (pn0 + j) * 64, qb * 64, bh);
+                        tma_load_3d(hslot + C::kQTileH + j * C::kQPanel, &tmDO, &bar_full[hs], (pn0 + j) * 64,
+                                    qb * 64, bh);
+                    }
+                    if (hs) {
+                        const size_t vrow = (size_t)bh * p.Nq_pad + (size_t)qb * 64;
+                        uint8_t* vec = smem + C::kOffVec + (st & 1) * 512;
+                        bulk_load(vec, p.neg_lse_log2 + vrow, 256, &bar_full[1]);
+                        bulk_load(vec + 256, p.neg_delta + vrow, 256, &bar_full[1]);
+                        ++issued1;
+                    } else {
+                        ++issued0;
+                    }
+                };
+                if (n_it > 0) {
+                    load_half(0, 0);
+                    load_half(0, 1);
+                }
+                for (int st = 0; st < n_it; ++st) {
+                    // half 0 of step st + 1 once step st's S^T / dP^T have read it
+                    if (st + 1 < n_it) {
+                        if (!mbar_wait(bar_h0free, (uint32_t)(st & 1), abort_flag))
+                            break;
+                        load_half(st + 1, 0);
+                    }
+                    // half 1 of step st once step st - 1's dV / dK have read it
+                    if (st > 0) {
+                        if (!mbar_wait(bar_h1free, (uint32_t)((st - 1) & 1), abort_flag))
+                            break;
+                        load_half(st, 1);
+                    }
+                }
+                if (*abort_flag) {
+                    mbar_wait_limited(bar_kv, 0, FA_WAIT_LIMIT_CYCLES);
+                    if (issued0 > 0)
+                        mbar_wait_limited(&bar_full[0], (uint32_t)((issued0 - 1) & 1), FA_WAIT_LIMIT_CYCLES);
+                    if (issued1 > 0)
+                        mbar_wait_limited(&bar_full[1], (uint32_t)((issued1 - 1) & 1), FA_WAIT_LIMIT_CYCLES);
+                }
+            } else {
             int issued = 0;
             for (int it = 0; it < n_it; ++it) {
                 const int s = it % C::kSlots;
@@ -379,6 +446,7 @@ __global__ void __launch_bounds__(384, 1)
                     mbar_wait_limited(&bar_full[i % C::kSlots], (uint32_t)((i / C::kSlots) & 1),
                                       FA_WAIT_LIMIT_CYCLES);
             }
+            }
         }
       } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
@@ -400,8 +468,9 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t lbo_kt = (D >= 128) ? (uint32_t)C::kKPanel : (uint32_t)(C::kOffZero - C::kOffK);
             const uint64_t dK_mn =
                 sdesc_sw128(smem_u32(smem + C::kOffK + fh * 2 * C::kKPanel), lbo_kt, 1024);
-            // the feature half's two panels of a Q / dO tile (the B operands of dK / dV)
-            const uint32_t fo = (uint32_t)(fh * 2 * C::kQPanel);
+            // the feature half's two panels of a Q / dO tile (the B operands of dK / dV);
+            // with half slots they are the whole of half slot 1
+            const uint32_t fo = C::kHalves ? (uint32_t)C::kSlot : (uint32_t)(fh * 2 * C::kQPanel);
             const uint64_t dSlot_k = sdesc_sw128(smem_u32(smem + C::kOffSlots), 16, 1024);   // Q / dO K-major
             const uint64_t dSlot_mn = sdesc_sw128(smem_u32(smem + C::kOffSlots), C::kQPanel, 1024);
             const uint64_t dDS_mn = sdesc_sw128(smem_u32(smem + C::kOffDS), C::kPTile, 1024);
@@ -410,14 +479,13 @@ __global__ void __launch_bounds__(384, 1)
             auto issue_sdp = [&](int it) {
                 const uint32_t so = (uint32_t)((it % C::kSlots) * C::kSlot);
                 const uint32_t tSb = tS + (uint32_t)(64 * (it & 1));
-                constexpr int kUnroll = D / 16 <= 8 ? D / 16 : 4;   // fewer live descriptors at d = 256
-#pragma unroll kUnroll
+#pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ok_ = (uint32_t)((kk >> 2) * C::kKPanel + (kk & 3) * 32);
                     const uint32_t oq = (uint32_t)((kk >> 2) * C::kQPanel + (kk & 3) * 32);
                     mma_ss_w(tSb, dK_k + off(ok_), dSlot_k + off(so + oq), id_sdp, kk > 0 ? 1u : 0u);
                 }
-#pragma unroll kUnroll
+#pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ok_ = (uint32_t)((kk >> 2) * C::kKPanel + (kk & 3) * 32);
                     const uint32_t oq = (uint32_t)((kk >> 2) * C::kQPanel + (kk & 3) * 32);
@@ -437,16 +505,80 @@ __global__ void __launch_bounds__(384, 1)
                 issue_sdp(in);
                 return true;
             };
+            // d = 256: S^T / dP^T of step it over one half slot (hs 0: the other CTA's
+            // features, K dimension first; hs 1: this CTA's own, accumulating on top)
+            auto issue_sdp_half = [&](int it, int hs) {
+                const uint32_t so = (uint32_t)(hs * C::kSlot);
+                const uint32_t tSb = tS + (uint32_t)(64 * (it & 1));
+                const int pn0 = 2 * (hs ? fh : 1 - fh);
+#pragma unroll 4   // fewer live descriptors
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t ok_ = (uint32_t)((pn0 + (kk >> 2)) * C::kKPanel + (kk & 3) * 32);
+                    const uint32_t oq = (uint32_t)((kk >> 2) * C::kQPanel + (kk & 3) * 32);
+                    mma_ss_w(tSb, dK_k + off(ok_), dSlot_k + off(so + oq), id_sdp, (hs || kk > 0) ? 1u : 0u);
+                }
+#pragma unroll 4   // fewer live descriptors
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t ok_ = (uint32_t)((pn0 + (kk >> 2)) * C::kKPanel + (kk & 3) * 32);
+                    const uint32_t oq = (uint32_t)((kk >> 2) * C::kQPanel + (kk & 3) * 32);
+                    mma_ss_w(tDP, dV_k + off(ok_), dSlot_k + off(so + C::kQTileH + oq), id_sdp,
+                             (hs || kk > 0) ? 1u : 0u);
+                }
+                mma_commit_w(hs ? bar_sdp : bar_h0free);
+            };
+            auto sdp_half = [&](int it, int hs) -> bool {
+                if (!mbar_wait_w(&bar_full[hs], (uint32_t)(it & 1), abort_flag))
+                    return false;
+                tc_fence_after();
+                issue_sdp_half(it, hs);
+                return true;
+            };
             bool ok = mbar_wait_w(bar_kv, 0, abort_flag);
+            if constexpr (C::kHalves) {
+            // per step it: S^T / dP^T of step it + 1 over half slot 0 (under step it's
+            // exponentials), then step it's gradients, then step it + 1's half slot 1
+            // (whose load the gradient MMAs' reads of it held back)
+            if (ok && n_it > 0)
+                ok = sdp_half(0, 0) && sdp_half(0, 1);
+            for (int it = 0; ok && it < n_it; ++it) {
+                if (it + 1 < n_it) {
+                    if (!(ok = mbar_wait_w(bar_sdp_read, (uint32_t)(it & 1), abort_flag)))
+                        break;
+                    if (!(ok = sdp_half(it + 1, 0)))
+                        break;
+                }
+                if (!(ok = mbar_wait_w(&bar_ds[it & 1], (uint32_t)((it >> 1) & 1), abort_flag)))
+                    break;
+                tc_fence_after();
+                if (it > 0) {
+                    if (!(ok = mbar_wait_w(bar_dqfree, (uint32_t)((it - 1) & 1), abort_flag)))
+                        break;
+                    tc_fence_after();
+                }
+                const uint32_t dso = (uint32_t)((it & 1) * C::kPTile);
+                const uint32_t tP = tS + (uint32_t)(64 * (it & 1));
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+                    mma_ts_w(tDV, tP + (uint32_t)(kk * 8), dSlot_mn + off(fo + C::kQTileH + kk * 2048), id_grad, acc);
+                    mma_ts_w(tDK, tP + 32u + (uint32_t)(kk * 8), dSlot_mn + off(fo + kk * 2048), id_grad, acc);
+                }
+                mma_commit_w(bar_h1free);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss_w(tDQ, dK_mn + off(kk * 2048), dDS_mn + off(dso + kk * 2048), id_dq, kk > 0 ? 1u : 0u);
+                mma_commit_w(&bar_gdone[it & 3]);
+                if (it + 1 < n_it && !(ok = sdp_half(it + 1, 1)))
+                    break;
+            }
+            } else {
             if (ok && n_it > 0) {
                 ok = mbar_wait_w(&bar_full[0], 0, abort_flag);
                 if (ok)
                     issue_sdp(0);
             }
             for (int it = 0; ok && it < n_it; ++it) {
-                // with one step slot the next step's Q / dO land only after this step's
-                // gradient MMAs have read the slot, so its S^T / dP^T come after them
-                if (C::kSlots > 1 && it + 1 < n_it && !(ok = next_sdp(it)))
+                if (it + 1 < n_it && !(ok = next_sdp(it)))
                     break;
                 if (!(ok = mbar_wait_w(&bar_ds[it & 1], (uint32_t)((it >> 1) & 1), abort_flag)))
                     break;
@@ -463,7 +595,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                    mma_ts_w(tDV, tP + (uint32_t)(kk * 8), dSlot_mn + off(so + C::kQTile + fo + kk * 2048), id_grad,
+                    mma_ts_w(tDV, tP + (uint32_t)(kk * 8), dSlot_mn + off(so + C::kQTileH + fo + kk * 2048), id_grad,
                              acc);
                     mma_ts_w(tDK, tP + 32u + (uint32_t)(kk * 8), dSlot_mn + off(so + fo + kk * 2048), id_grad, acc);
                 }
@@ -472,8 +604,7 @@ __global__ void __launch_bounds__(384, 1)
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ss_w(tDQ, dK_mn + off(kk * 2048), dDS_mn + off(dso + kk * 2048), id_dq, kk > 0 ? 1u : 0u);
                 mma_commit_w(&bar_gdone[it & 3]);
-                if (C::kSlots == 1 && it + 1 < n_it && !(ok = next_sdp(it)))
-                    break;
+            }
             }
             mma_commit_w(bar_final);
             if (!ok)
@@ -501,7 +632,8 @@ __global__ void __launch_bounds__(384, 1)
             // -LSE * log2(e) and -D of the step's 64 query rows, read four at a time: each
             // load is a broadcast, and 16-byte ones take a quarter of the shared-memory cycles
             const float4* nlse4 = reinterpret_cast<const float4*>(
-                smem + C::kOffSlots + (it % C::kSlots) * C::kSlot + 2 * C::kQTile);
+                C::kHalves ? smem + C::kOffVec + (it & 1) * 512
+                           : smem + C::kOffSlots + (it % C::kSlots) * C::kSlot + 2 * C::kQTile);
             const float4* ndlt4 = nlse4 + 16;
             const uint32_t tSb = tS + (uint32_t)(64 * (it & 1));
             uint32_t sr[64], dr[64];
