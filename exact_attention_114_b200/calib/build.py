@@ -6,6 +6,8 @@ co-running-load measurements quoted for the kernels) into calib/_build/.
 mma_bench   cycles per tcgen05.mma (kind::f16, M = 128, K = 16) for N = 64 / 128 / 256, SS and TS operands
 mufu_bench  MUFU ex2 results per clock per SM for f32, f16x2 and bf16x2
 load_bench  the forward kernel's MMA sequence while other warps run MUFU, FMA, ALU or TMEM load/store work
+softmax_pass_bench  the backward's P / dS pass of one query step alone on one SM, and with pieces left out
+convert_bench  ex2 against the e4m3 / bf16 conversions (shared pipe or not), and an arithmetic e4m3 conversion
 """
 import os
 import subprocess
@@ -14,7 +16,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(os.path.dirname(HERE), "csrc")
 OUT = os.path.join(HERE, "_build")
-BENCHES = ("mma_bench", "mufu_bench", "load_bench")
+BENCHES = ("mma_bench", "mufu_bench", "load_bench", "softmax_pass_bench", "convert_bench")
 
 
 def build() -> list:
