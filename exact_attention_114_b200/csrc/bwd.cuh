@@ -217,21 +217,25 @@ struct BwdCfg {
     static constexpr int kKTile = (D / 64) * kKPanel;  // K or V block
     static constexpr int kQPanel = 64 * 128;           // 64 rows x 64 bf16
     static constexpr int kQTile = (D / 64) * kQPanel;  // Q or dO block
-    // d = 256: a step's Q / dO in two half slots (the other CTA's features, then
-    // this CTA's own), with -lse_log2 / -delta in a separate pair of buffers
+    // d = 256: a step's Q / dO by feature half (kQTileH bytes each): the other CTA's
+    // half (Q, dO: read by S^T / dP^T only), this CTA's Q half in two buffers (read
+    // by S^T and dK) and its dO half in one (read by dP^T and dV); -lse_log2 / -delta
+    // in a separate pair of buffers; one dS^T buffer
     static constexpr bool kHalves = (D == 256);
-    static constexpr int kQTileH = kHalves ? 2 * kQPanel : kQTile;   // Q or dO part of one slot
-    static constexpr int kSlot = kHalves ? 2 * kQTileH                // Q, dO of one feature half
-                                         : 2 * kQTile + 1024;         // Q, dO, -lse_log2[64], -delta[64]
-    static constexpr int kSlots = kHalves ? 2 : 3;     // step slots in flight (TMA latency cover)
+    static constexpr int kQTileH = kHalves ? 2 * kQPanel : kQTile;   // Q or dO of one feature half
+    static constexpr int kSlot = 2 * kQTile + 1024;    // d <= 128: Q, dO, -lse_log2[64], -delta[64]
+    static constexpr int kSlots = 3;                   // d <= 128: step slots in flight (TMA latency cover)
+    static constexpr int kOffOther = 0, kOffQOwn = 2 * kQTileH, kOffDOOwn = 4 * kQTileH;   // d = 256, in the slot area
+    static constexpr int kSlotArea = kHalves ? 5 * kQTileH : kSlots * kSlot;
     static constexpr int kPTile = 128 * 128;           // dS^T: 128 keys x 64 q bf16
+    static constexpr int kDSBufs = kHalves ? 1 : 2;
     static constexpr int kOffK = 0;
     static constexpr int kOffV = kOffK + kKTile;
     static constexpr int kOffZero = kOffV + kKTile;                 // zero panel (D = 64 only)
     static constexpr int kOffSlots = kOffZero + (D == 64 ? kKPanel : 0);
-    static constexpr int kOffVec = kOffSlots + kSlots * kSlot;      // d = 256: [2][-lse_log2 64, -delta 64]
-    static constexpr int kOffDS = kOffVec + (kHalves ? 1024 : 0);   // dS^T, two buffers
-    static constexpr int kOffDQ = kOffDS + 2 * kPTile;              // fp32 [32][D] staging (half a step)
+    static constexpr int kOffVec = kOffSlots + kSlotArea;           // d = 256: [2][-lse_log2 64, -delta 64]
+    static constexpr int kOffDS = kOffVec + (kHalves ? 1024 : 0);   // dS^T buffers
+    static constexpr int kOffDQ = kOffDS + kDSBufs * kPTile;        // fp32 [32][D] staging (half a step)
     static constexpr int kOffBar = kOffDQ + (kStagedDQ ? 32 * D * 4 : 0);
     static constexpr int kSmemBytes = kOffBar + 256 + 1024;
     static constexpr uint32_t kTmemCols = 512;
@@ -291,9 +295,13 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* bar_final = bars + 15;    // all MMAs done
     uint64_t* bar_sdp_read = bars + 16; // S^T, dP^T of a step loaded into registers (count 4)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
-    // d = 256: half slot 0 read by the step's S^T / dP^T MMAs, half slot 1 by its dV / dK MMAs
+    // d = 256: bar_full[0] the other half landed, [1 + b] Q own in buffer b, [3] dO own;
+    // the other half read by the step's S^T / dP^T, Q own in buffer b by its dK
+    // ([b]: one barrier per buffer, so a buffer's next read waits for its next load),
+    // dO own by its dV
     uint64_t* bar_h0free = bars + 18;
-    uint64_t* bar_h1free = bars + 19;
+    uint64_t* bar_qfree = bars + 19;   // [2]
+    uint64_t* bar_dofree = bars + 21;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = warp_id(), lane = lane_id();
@@ -314,7 +322,7 @@ __global__ void __launch_bounds__(384, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(bar_kv, 1);
-        for (int s = 0; s < C::kSlots; ++s)
+        for (int s = 0; s < (C::kHalves ? 4 : C::kSlots); ++s)
             mbar_init(&bar_full[s], 1);
         mbar_init(bar_sdp, 1);
         mbar_init(&bar_ds[0], 4);
@@ -325,7 +333,9 @@ __global__ void __launch_bounds__(384, 1)
         mbar_init(bar_dqfree, 4);
         mbar_init(bar_final, 1);
         mbar_init(bar_h0free, 1);
-        mbar_init(bar_h1free, 1);
+        mbar_init(&bar_qfree[0], 1);
+        mbar_init(&bar_qfree[1], 1);
+        mbar_init(bar_dofree, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -364,57 +374,71 @@ __global__ void __launch_bounds__(384, 1)
                 tma_load_3d(smem + C::kOffV + pn * C::kKPanel, &tmV, bar_kv, pn * 64, kb * 128, kvh);
             }
             if constexpr (C::kHalves) {
-                // half slot 0: the features of the other CTA of the pair, which only the
-                // step's S^T / dP^T read; half slot 1: this CTA's own features, which its
-                // dV / dK read too, plus the step's -lse_log2 / -delta.  Loads go out in
-                // the order their slots are freed: half 0 of step s + 1 before half 1 of s.
-                int issued0 = 0, issued1 = 0;
-                auto load_half = [&](int st, int hs) {
+                // part 0: the other CTA's feature half (Q and dO), read only by the step's
+                // S^T / dP^T; part 1: this CTA's Q half (buffer st & 1) with the step's
+                // -lse_log2 / -delta; part 2: its dO half.  Loads go out in the order their
+                // buffers are freed: the other half of step st + 1, the dO half of st, the
+                // Q half of st + 1.
+                int issued[3] = {0, 0, 0};
+                auto load_part = [&](int st, int part) {
                     int h, qb;
                     step_coords(st, h, qb);
                     const int bh = b * p.Hq + h;
-                    uint8_t* hslot = smem + C::kOffSlots + hs * C::kSlot;
-                    const int pn0 = 2 * (hs ? fh : 1 - fh);   // first 64-feature panel of the half
-                    mbar_arrive_expect_tx(&bar_full[hs], 2 * C::kQTileH + (hs ? 512 : 0));
+                    const int pn0 = 2 * (part ? fh : 1 - fh);   // first 64-feature panel of the half
+                    uint64_t* bar = &bar_full[part == 0 ? 0 : part == 1 ? 1 + (st & 1) : 3];
+                    uint8_t* dst = smem + C::kOffSlots +
+                                   (part == 0 ? C::kOffOther : part == 1 ? C::kOffQOwn + (st & 1) * C::kQTileH
+                                                                         : C::kOffDOOwn);
+                    mbar_arrive_expect_tx(bar, (part ? 1 : 2) * C::kQTileH + (part == 1 ? 512 : 0));
                     for (int j = 0; j < 2; ++j) {
-                        tma_load_3d(hslot + j * C::kQPanel, &tmQ, &bar_full[hs], (pn0 + j) * 64, qb * 64, bh);
-                        tma_load_3d(hslot + C::kQTileH + j * C::kQPanel, &tmDO, &bar_full[hs], (pn0 + j) * 64,
-                                    qb * 64, bh);
+                        if (part != 2)
+                            tma_load_3d(dst + j * C::kQPanel, &tmQ, bar, (pn0 + j) * 64, qb * 64, bh);
+                        if (part != 1)
+                            tma_load_3d(dst + (part ? 0 : C::kQTileH) + j * C::kQPanel, &tmDO, bar,
+                                        (pn0 + j) * 64, qb * 64, bh);
                     }
-                    if (hs) {
+                    if (part == 1) {
                         const size_t vrow = (size_t)bh * p.Nq_pad + (size_t)qb * 64;
                         uint8_t* vec = smem + C::kOffVec + (st & 1) * 512;
-                        bulk_load(vec, p.neg_lse_log2 + vrow, 256, &bar_full[1]);
-                        bulk_load(vec + 256, p.neg_delta + vrow, 256, &bar_full[1]);
-                        ++issued1;
-                    } else {
-                        ++issued0;
+                        bulk_load(vec, p.neg_lse_log2 + vrow, 256, bar);
+                        bulk_load(vec + 256, p.neg_delta + vrow, 256, bar);
                     }
+                    ++issued[part];
                 };
-                if (n_it > 0) {
-                    load_half(0, 0);
-                    load_half(0, 1);
-                }
+                if (n_it > 0)
+                    for (int part = 0; part < 3; ++part)
+                        load_part(0, part);
+                if (n_it > 1)
+                    load_part(1, 1);   // the second Q buffer starts free
                 for (int st = 0; st < n_it; ++st) {
-                    // half 0 of step st + 1 once step st's S^T / dP^T have read it
+                    // the other half of step st + 1 once step st's S^T / dP^T have read it
                     if (st + 1 < n_it) {
                         if (!mbar_wait(bar_h0free, (uint32_t)(st & 1), abort_flag))
                             break;
-                        load_half(st + 1, 0);
+                        load_part(st + 1, 0);
                     }
-                    // half 1 of step st once step st - 1's dV / dK have read it
                     if (st > 0) {
-                        if (!mbar_wait(bar_h1free, (uint32_t)((st - 1) & 1), abort_flag))
+                        // the dO half of step st once step st - 1's dV has read it
+                        if (!mbar_wait(bar_dofree, (uint32_t)((st - 1) & 1), abort_flag))
                             break;
-                        load_half(st, 1);
+                        load_part(st, 2);
+                        // the Q half of step st + 1 into the buffer step st - 1's dK has read
+                        if (st + 1 < n_it) {
+                            if (!mbar_wait(&bar_qfree[(st - 1) & 1], (uint32_t)(((st - 1) >> 1) & 1), abort_flag))
+                                break;
+                            load_part(st + 1, 1);
+                        }
                     }
                 }
                 if (*abort_flag) {
                     mbar_wait_limited(bar_kv, 0, FA_WAIT_LIMIT_CYCLES);
-                    if (issued0 > 0)
-                        mbar_wait_limited(&bar_full[0], (uint32_t)((issued0 - 1) & 1), FA_WAIT_LIMIT_CYCLES);
-                    if (issued1 > 0)
-                        mbar_wait_limited(&bar_full[1], (uint32_t)((issued1 - 1) & 1), FA_WAIT_LIMIT_CYCLES);
+                    // the last load of each buffer: part 1 alternates between two barriers
+                    if (issued[0] > 0)
+                        mbar_wait_limited(&bar_full[0], (uint32_t)((issued[0] - 1) & 1), FA_WAIT_LIMIT_CYCLES);
+                    for (int i = max(0, issued[1] - 2); i < issued[1]; ++i)
+                        mbar_wait_limited(&bar_full[1 + (i & 1)], (uint32_t)((i >> 1) & 1), FA_WAIT_LIMIT_CYCLES);
+                    if (issued[2] > 0)
+                        mbar_wait_limited(&bar_full[3], (uint32_t)((issued[2] - 1) & 1), FA_WAIT_LIMIT_CYCLES);
                 }
             } else {
             int issued = 0;
@@ -468,9 +492,8 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t lbo_kt = (D >= 128) ? (uint32_t)C::kKPanel : (uint32_t)(C::kOffZero - C::kOffK);
             const uint64_t dK_mn =
                 sdesc_sw128(smem_u32(smem + C::kOffK + fh * 2 * C::kKPanel), lbo_kt, 1024);
-            // the feature half's two panels of a Q / dO tile (the B operands of dK / dV);
-            // with half slots they are the whole of half slot 1
-            const uint32_t fo = C::kHalves ? (uint32_t)C::kSlot : (uint32_t)(fh * 2 * C::kQPanel);
+            // the feature half's two panels of a Q / dO tile (the B operands of dK / dV)
+            const uint32_t fo = (uint32_t)(fh * 2 * C::kQPanel);
             const uint64_t dSlot_k = sdesc_sw128(smem_u32(smem + C::kOffSlots), 16, 1024);   // Q / dO K-major
             const uint64_t dSlot_mn = sdesc_sw128(smem_u32(smem + C::kOffSlots), C::kQPanel, 1024);
             const uint64_t dDS_mn = sdesc_sw128(smem_u32(smem + C::kOffDS), C::kPTile, 1024);
@@ -507,45 +530,66 @@ __global__ void __launch_bounds__(384, 1)
             };
             // d = 256: S^T / dP^T of step it over one half slot (hs 0: the other CTA's
             // features, K dimension first; hs 1: this CTA's own, accumulating on top)
-            auto issue_sdp_half = [&](int it, int hs) {
-                const uint32_t so = (uint32_t)(hs * C::kSlot);
-                const uint32_t tSb = tS + (uint32_t)(64 * (it & 1));
+            // d = 256: S^T (dp false) or dP^T (dp true) of step it over one feature half:
+            // hs 0 the other CTA's features, K dimension first; hs 1 this CTA's own,
+            // accumulating on top (Q own in buffer it & 1, dO own in its one buffer)
+            auto mma_half = [&](int it, int hs, bool dp) {
+                const uint32_t tdst = dp ? tDP : tS + (uint32_t)(64 * (it & 1));
+                const uint64_t a0 = dp ? dV_k : dK_k;
+                const uint32_t so = (uint32_t)(hs == 0 ? C::kOffOther + (dp ? C::kQTileH : 0)
+                                               : dp ? C::kOffDOOwn : C::kOffQOwn + (it & 1) * C::kQTileH);
                 const int pn0 = 2 * (hs ? fh : 1 - fh);
 #pragma unroll 4   // fewer live descriptors
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t ok_ = (uint32_t)((pn0 + (kk >> 2)) * C::kKPanel + (kk & 3) * 32);
                     const uint32_t oq = (uint32_t)((kk >> 2) * C::kQPanel + (kk & 3) * 32);
-                    mma_ss_w(tSb, dK_k + off(ok_), dSlot_k + off(so + oq), id_sdp, (hs || kk > 0) ? 1u : 0u);
+                    mma_ss_w(tdst, a0 + off(ok_), dSlot_k + off(so + oq), id_sdp, (hs || kk > 0) ? 1u : 0u);
                 }
-#pragma unroll 4   // fewer live descriptors
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t ok_ = (uint32_t)((pn0 + (kk >> 2)) * C::kKPanel + (kk & 3) * 32);
-                    const uint32_t oq = (uint32_t)((kk >> 2) * C::kQPanel + (kk & 3) * 32);
-                    mma_ss_w(tDP, dV_k + off(ok_), dSlot_k + off(so + C::kQTileH + oq), id_sdp,
-                             (hs || kk > 0) ? 1u : 0u);
-                }
-                mma_commit_w(hs ? bar_sdp : bar_h0free);
             };
-            auto sdp_half = [&](int it, int hs) -> bool {
-                if (!mbar_wait_w(&bar_full[hs], (uint32_t)(it & 1), abort_flag))
+            // bar_full[part] of step it landed: part 0 the other half, 1 Q own, 2 dO own
+            auto wait_part = [&](int it, int part) -> bool {
+                uint64_t* bar = &bar_full[part == 0 ? 0 : part == 1 ? 1 + (it & 1) : 3];
+                const uint32_t ph = (uint32_t)((part == 1 ? (it >> 1) : it) & 1);
+                if (!mbar_wait_w(bar, ph, abort_flag))
                     return false;
                 tc_fence_after();
-                issue_sdp_half(it, hs);
+                return true;
+            };
+            // this CTA's half of step it: S^T on Q own, dP^T on dO own, then the signal
+            auto own_half = [&](int it) -> bool {
+                if (!wait_part(it, 1))
+                    return false;
+                mma_half(it, 1, false);
+                if (!wait_part(it, 2))
+                    return false;
+                mma_half(it, 1, true);
+                mma_commit_w(bar_sdp);
                 return true;
             };
             bool ok = mbar_wait_w(bar_kv, 0, abort_flag);
             if constexpr (C::kHalves) {
-            // per step it: S^T / dP^T of step it + 1 over half slot 0 (under step it's
-            // exponentials), then step it's gradients, then step it + 1's half slot 1
-            // (whose load the gradient MMAs' reads of it held back)
-            if (ok && n_it > 0)
-                ok = sdp_half(0, 0) && sdp_half(0, 1);
+            // per step it: S^T / dP^T of step it + 1 over the other half (under step it's
+            // exponentials); step it's dV (frees the dO half), dK (frees its Q buffer)
+            // and dQ^T; then step it + 1's own half: its Q half was loaded a step ahead,
+            // and its dO half's load runs under dK, dQ^T and the own-half S^T
+            if (ok && n_it > 0) {
+                ok = wait_part(0, 0);
+                if (ok) {
+                    mma_half(0, 0, false);
+                    mma_half(0, 0, true);
+                    mma_commit_w(bar_h0free);
+                    ok = own_half(0);
+                }
+            }
             for (int it = 0; ok && it < n_it; ++it) {
                 if (it + 1 < n_it) {
                     if (!(ok = mbar_wait_w(bar_sdp_read, (uint32_t)(it & 1), abort_flag)))
                         break;
-                    if (!(ok = sdp_half(it + 1, 0)))
+                    if (!(ok = wait_part(it + 1, 0)))
                         break;
+                    mma_half(it + 1, 0, false);
+                    mma_half(it + 1, 0, true);
+                    mma_commit_w(bar_h0free);
                 }
                 if (!(ok = mbar_wait_w(&bar_ds[it & 1], (uint32_t)((it >> 1) & 1), abort_flag)))
                     break;
@@ -555,20 +599,23 @@ __global__ void __launch_bounds__(384, 1)
                         break;
                     tc_fence_after();
                 }
-                const uint32_t dso = (uint32_t)((it & 1) * C::kPTile);
                 const uint32_t tP = tS + (uint32_t)(64 * (it & 1));
+                const uint32_t oq = (uint32_t)(C::kOffQOwn + (it & 1) * C::kQTileH);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                    mma_ts_w(tDV, tP + (uint32_t)(kk * 8), dSlot_mn + off(fo + C::kQTileH + kk * 2048), id_grad, acc);
-                    mma_ts_w(tDK, tP + 32u + (uint32_t)(kk * 8), dSlot_mn + off(fo + kk * 2048), id_grad, acc);
-                }
-                mma_commit_w(bar_h1free);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ts_w(tDV, tP + (uint32_t)(kk * 8), dSlot_mn + off(C::kOffDOOwn + kk * 2048), id_grad,
+                             (it > 0 || kk > 0) ? 1u : 0u);
+                mma_commit_w(bar_dofree);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ts_w(tDK, tP + 32u + (uint32_t)(kk * 8), dSlot_mn + off(oq + kk * 2048), id_grad,
+                             (it > 0 || kk > 0) ? 1u : 0u);
+                mma_commit_w(&bar_qfree[it & 1]);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ss_w(tDQ, dK_mn + off(kk * 2048), dDS_mn + off(dso + kk * 2048), id_dq, kk > 0 ? 1u : 0u);
+                    mma_ss_w(tDQ, dK_mn + off(kk * 2048), dDS_mn + off(kk * 2048), id_dq, kk > 0 ? 1u : 0u);
                 mma_commit_w(&bar_gdone[it & 3]);
-                if (it + 1 < n_it && !(ok = sdp_half(it + 1, 1)))
+                if (it + 1 < n_it && !(ok = own_half(it + 1)))
                     break;
             }
             } else {
@@ -674,14 +721,16 @@ __global__ void __launch_bounds__(384, 1)
             }
             // P^T over this step's S^T columns (the dV MMA reads it from there)
             tmem_st32(tSb, pp);
-            // dS^T into this step's buffer, free once the gradient MMAs of step it-2 are done
-            if (it >= 2) {
-                ok = mbar_wait(&bar_gdone[(it - 2) & 3], (uint32_t)(((it - 2) >> 2) & 1), abort_flag);
+            // dS^T into this step's buffer, free once the gradient MMAs of the step that
+            // used it last (it - 2; it - 1 with the single buffer of d = 256) are done
+            if (it >= C::kDSBufs) {
+                const int prev = it - C::kDSBufs;
+                ok = mbar_wait(&bar_gdone[prev & 3], (uint32_t)((prev >> 2) & 1), abort_flag);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok)
                     break;
             }
-            uint8_t* sDS = smem + C::kOffDS + (it & 1) * C::kPTile;
+            uint8_t* sDS = smem + C::kOffDS + (it % C::kDSBufs) * C::kPTile;
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch)
                 *reinterpret_cast<uint4*>(sDS + sw128_off(r, ch)) =
