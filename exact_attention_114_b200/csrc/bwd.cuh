@@ -583,22 +583,21 @@ __global__ void __launch_bounds__(384, 1)
             }
             for (int it = 0; ok && it < n_it; ++it) {
                 if (it + 1 < n_it) {
-                    if (!(ok = mbar_wait_w(bar_sdp_read, (uint32_t)(it & 1), abort_flag)))
+                    // step it's dP^T in registers, and the other half of step it + 1 landed
+                    if (!(ok = mbar_wait2_w(bar_sdp_read, (uint32_t)(it & 1), &bar_full[0],
+                                            (uint32_t)((it + 1) & 1), abort_flag)))
                         break;
-                    if (!(ok = wait_part(it + 1, 0)))
-                        break;
+                    tc_fence_after();
                     mma_half(it + 1, 0, false);
                     mma_half(it + 1, 0, true);
                     mma_commit_w(bar_h0free);
                 }
-                if (!(ok = mbar_wait_w(&bar_ds[it & 1], (uint32_t)((it >> 1) & 1), abort_flag)))
+                // dS of step it written, and dQ^T of step it - 1 read out (for it = 0 the
+                // second check is of the phase before the barrier's first, complete)
+                if (!(ok = mbar_wait2_w(&bar_ds[it & 1], (uint32_t)((it >> 1) & 1), bar_dqfree,
+                                        (uint32_t)((it - 1) & 1), abort_flag)))
                     break;
                 tc_fence_after();
-                if (it > 0) {
-                    if (!(ok = mbar_wait_w(bar_dqfree, (uint32_t)((it - 1) & 1), abort_flag)))
-                        break;
-                    tc_fence_after();
-                }
                 const uint32_t tP = tS + (uint32_t)(64 * (it & 1));
                 const uint32_t oq = (uint32_t)(C::kOffQOwn + (it & 1) * C::kQTileH);
 #pragma unroll

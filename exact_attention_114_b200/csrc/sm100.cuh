@@ -298,6 +298,27 @@ __device__ __forceinline__ bool mbar_wait_w(uint64_t* bar, uint32_t parity, vola
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
 }
 
+// Two barriers checked by one pair of try_waits in flight together (a shared-memory
+// round trip saved where the memory pipe is busy); the slow path waits for each in
+// turn.
+__device__ __forceinline__ bool mbar_wait2_w(uint64_t* a, uint32_t pa, uint64_t* b, uint32_t pb,
+                                             volatile int* abort_flag)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 q, [%3], %4;\n\t"
+        "and.pred p, p, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(a)), "r"(pa), "r"(smem_u32(b)), "r"(pb)
+        : "memory");
+    if (__all_sync(0xffffffffu, ok != 0))
+        return true;
+    return mbar_wait_w(a, pa, abort_flag) && mbar_wait_w(b, pb, abort_flag);
+}
+
 // Instruction descriptor, kind::f16: fp32 accumulate, A and B of one 16-bit type
 // (fmt 1 = bf16, 0 = fp16).
 //   bits [4,6) D format (1 = f32), [7,10) A format, [10,13) B format,
