@@ -820,9 +820,15 @@ __global__ void __launch_bounds__(384, 1)
                         if (lane == 0)
                             mbar_arrive(bar_dqfree);
                     }
+                    // paced: a short pause after every 8 reductions keeps them from filling
+                    // the memory pipe that the MMA warp's barrier checks go through (the
+                    // drain has most of a step to finish)
 #pragma unroll
-                    for (int c = 0; c < 32; ++c)
+                    for (int c = 0; c < 32; ++c) {
                         red_add_f32(dst + (size_t)(32 * hq + c) * D, __uint_as_float(a[c]));
+                        if ((c & 7) == 7)
+                            __nanosleep(64);
+                    }
                 }
                 continue;
             }
