@@ -41,14 +41,16 @@
 // feature half fh): S^T and dP^T still contract over all 256 features (the
 // two CTAs of a key block both recompute them), while dV, dK and dQ^T cover
 // only features 128 fh .. 128 fh + 127, with the tensor-memory layout of
-// d = 128.  K and V of the block take 128 KB of shared memory, which leaves
-// room for two half slots of a step's Q / dO (32 KB each) and no dQ staging
-// tile: the drain warps add dQ^T to the accumulator straight from registers
-// with fp32 reductions (one 128-byte row segment per warp instruction).  Half
-// slot 0 holds the features this CTA does not own, which only S^T and dP^T
-// read: it is refilled for the next step as soon as those MMAs are done.  Half
-// slot 1 holds the owned features, which dV and dK read too: it is refilled
-// once they are done, while dQ^T and the next step's first-half MMAs run.
+// d = 128.  K and V of the block take 128 KB of shared memory, which leaves no
+// room for a dQ staging tile: the drain warps add dQ^T to the accumulator
+// straight from registers with fp32 reductions (one 128-byte row segment per
+// warp instruction, paced so that they do not crowd the MMA warp's barrier
+// checks out of the memory pipe).  A step's Q / dO are staged by feature half:
+// the other CTA's half (Q and dO), which only S^T and dP^T read, is refilled for
+// the next step as soon as those MMAs are done; this CTA's Q half (read by S^T
+// and dK) sits in two buffers and lands a step ahead; its dO half (read by dP^T
+// and dV) sits in one buffer and is refilled once dV is done, while dK, dQ^T and
+// the own-half S^T run.  One dS^T buffer.
 #pragma once
 
 #include "sm100.cuh"
