@@ -79,7 +79,7 @@ struct FwdCfg {
     // warpgroups raise theirs, the third lowers its, within the launch's total
     static_assert(kRegsSoftmax >= 168 && kRegsOther <= 168 && 2 * kRegsSoftmax + kRegsOther <= 3 * 168,
                   "register split");
-    static_assert(kTiles == 2 || 128 + D <= (int)kTmemCols, "one tile: S and O must fit in TMEM");
+    static_assert(kTiles == 2 || 2 * 128 + D <= (int)kTmemCols, "one tile: two S buffers and O must fit in TMEM");
 };
 
 __device__ __forceinline__ int fwd_blocks_for_tile(int qt, int Nq, int Nk, bool causal)
@@ -233,6 +233,7 @@ __global__ void __launch_bounds__(384, 1)
         if (lane == 0) {
             int nq0 = 0, nq1 = 0;   // Q loads so far into tile slot 0 / 1
             int kvi = 0;            // K/V ring loads so far
+            int kn = 0, vn = 0;     // one-tile blocks: K loads (slot 0) and V loads (slot 1) so far
             bool ok = true;
             int tile = (int)blockIdx.x;
             // take the counter slot for this launch, or find it held by another one
@@ -265,6 +266,33 @@ __global__ void __launch_bounds__(384, 1)
                     else
                         ++nq0;
                 }
+                if constexpr (C::kTiles == 1) {
+                    // K blocks in slot 0, V blocks in slot 1, loaded in the order the MMA
+                    // warp frees them: it issues S(0), S(1), P.V(0), S(2), P.V(1), ...,
+                    // so K(j + 2) may land once S(j + 1) has read K(j + 1), and V(j + 1)
+                    // once P.V(j) has read V(j)
+                    auto load_kv = [&](int j, int kv) -> bool {
+                        int& cnt = kv ? vn : kn;
+                        if (!mbar_wait(&bar_empty[kv], ((uint32_t)cnt & 1u) ^ 1u, abort_flag))
+                            return false;
+                        uint8_t* dst = sKV + kv * C::kTileBytes;
+                        mbar_arrive_expect_tx(&bar_full[kv], C::kTileBytes);
+                        for (int pn = 0; pn < C::kPanels; ++pn)
+                            tma_load_3d(dst + pn * C::kPanelBytes, kv ? &tmV : &tmK, &bar_full[kv],
+                                        pn * C::kPanelElems, j * 128, w.kvh);
+                        ++cnt;
+                        return true;
+                    };
+                    const int n = w.n_iter;
+                    if (n > 0)
+                        ok = load_kv(0, 0) && load_kv(0, 1) && (n < 2 || load_kv(1, 0));
+                    for (int j = 0; ok && j < n; ++j) {
+                        if (j + 2 < n && !(ok = load_kv(j + 2, 0)))
+                            break;
+                        if (j + 1 < n && !(ok = load_kv(j + 1, 1)))
+                            break;
+                    }
+                } else
                 for (int j = 0; ok && j < w.n_iter; ++j) {
                     for (int kv = 0; kv < 2; ++kv) {
                         const int slot = kvi % C::kStages;
@@ -309,6 +337,10 @@ __global__ void __launch_bounds__(384, 1)
                 for (int i = max(0, kvi - C::kStages); i < kvi; ++i)
                     mbar_wait_limited(&bar_full[i % C::kStages], (uint32_t)(i / C::kStages) & 1u,
                                       FA_WAIT_LIMIT_CYCLES);
+                if (kn > 0)
+                    mbar_wait_limited(&bar_full[0], (uint32_t)((kn - 1) & 1), FA_WAIT_LIMIT_CYCLES);
+                if (vn > 0)
+                    mbar_wait_limited(&bar_full[1], (uint32_t)((vn - 1) & 1), FA_WAIT_LIMIT_CYCLES);
                 if (nq0 > 0)
                     mbar_wait_limited(&bar_q[0], (uint32_t)((nq0 - 1) & 1), FA_WAIT_LIMIT_CYCLES);
                 if (nq1 > 0)
@@ -374,6 +406,10 @@ __global__ void __launch_bounds__(384, 1)
             // 4 << t = parity of the blocks of slot t in earlier tiles (bar_p phases)
             uint32_t ph = 0;
             int kvi = 0;            // ring index of the tile's first K block
+            // one-tile blocks: K and V blocks read so far (slots 0 and 1), and the blocks of
+            // earlier tiles whose S went to S buffer 0 / 1 (bar_p phases)
+            int kc = 0, vc = 0;
+            int su[2] = {0, 0};
             for (int u = 0; ok; ++u) {
                 const int tile = fwd_take_tile(bar_tfull, bar_tfree, tile_ring, u, lane, abort_flag, ok);
                 if (!ok || tile >= n_tiles)
@@ -386,6 +422,64 @@ __global__ void __launch_bounds__(384, 1)
                     ph ^= 1u << t;
                 }
                 tc_fence_after();
+                if constexpr (C::kTiles == 1) {
+                    // S of block j goes to S buffer j & 1 (TMEM columns 128 (j & 1) ..), so
+                    // S(j + 1) runs while block j's softmax reads S(j): the order is S(0),
+                    // S(1), P.V(0), S(2), P.V(1), ... and the tensor core waits for a
+                    // softmax only when P.V(j) would run ahead of it
+                    const int n = w.n_iter;
+                    auto issue_S1 = [&](int j) -> bool {
+                        if (!mbar_wait_w(&bar_full[0], (uint32_t)(kc & 1), abort_flag))
+                            return false;
+                        tc_fence_after();
+                        constexpr int kUnrollS = C::kKSteps <= 4 ? C::kKSteps : 4;   // fewer live descriptors
+#pragma unroll kUnrollS
+                        for (int kk = 0; kk < C::kKSteps; ++kk) {
+                            const uint32_t o = (uint32_t)((kk >> 2) * C::kPanelBytes + (kk & 3) * 32);
+                            mma_ss_k<F8>(tS(j & 1), dQ_k + off(o), dKV_k + off(o), idS, kk > 0 ? 1u : 0u);
+                        }
+                        mma_commit_w(&bar_empty[0]);   // K slot free
+                        mma_commit_w(&bar_s[j & 1]);
+                        if (j == n - 1)
+                            mma_commit_w(&bar_qfree[0]);   // the tile's last Q.K^T
+                        ++kc;
+                        return true;
+                    };
+                    if (ok && n > 0)
+                        ok = issue_S1(0) && (n < 2 || issue_S1(1));
+                    for (int j = 0; ok && j < n; ++j) {
+                        const int b = j & 1;
+                        if (!(ok = mbar_wait_w(&bar_full[1], (uint32_t)(vc & 1), abort_flag)))
+                            break;
+                        tc_fence_after();
+                        const uint32_t pp = (uint32_t)((su[b] + (j >> 1)) & 1);
+                        for (int hf = 0; hf < 2 && ok; ++hf) {
+                            if (!(ok = mbar_wait_w(&bar_p[2 * b + hf], pp, abort_flag)))
+                                break;
+                            tc_fence_after();
+                            // O += P V for keys 64 hf .. 64 hf + 63 of block j (V in slot 1)
+#pragma unroll
+                            for (int k4 = 0; k4 < 4; ++k4) {
+                                const int kk = 4 * hf + k4;
+                                mma_ts_w(tO(0), tS(b) + (uint32_t)(kk * 8),
+                                         dKV_mn + off((uint32_t)C::kTileBytes + (uint32_t)(kk * 2048)), idPV,
+                                         (j > 0 || kk > 0) ? 1u : 0u);
+                            }
+                        }
+                        if (!ok)
+                            break;
+                        mma_commit_w(&bar_empty[1]);   // V slot free
+                        ++vc;
+                        mma_commit_w(&bar_o[1]);       // P.V(j) done: block j + 1 may rescale O
+                        if (j == n - 1)
+                            mma_commit_w(&bar_o[0]);
+                        if (j + 2 < n && !(ok = issue_S1(j + 2)))
+                            break;
+                    }
+                    su[0] += (n + 1) / 2;
+                    su[1] += n / 2;
+                    continue;
+                }
                 const int k0 = kvi;
                 if (ok && w.n_iter > 0) {
                     ok = mbar_wait_w(&bar_full[k0 % C::kStages], phase(k0), abort_flag);
@@ -459,6 +553,7 @@ __global__ void __launch_bounds__(384, 1)
         const float sl2 = p.scale_log2;
         int bt = 0;   // blocks of earlier tiles (bar_s phases)
         int no = 0;   // earlier tiles with at least one block (bar_o phases)
+        int su[2] = {0, 0};   // one-tile blocks: blocks of earlier tiles in S buffer 0 / 1
         bool ok = true;
 
         for (int u = 0; ok; ++u) {
@@ -472,13 +567,17 @@ __global__ void __launch_bounds__(384, 1)
             float m_ref = -INFINITY, l = 0.f;
 
             for (int j = 0; j < nb; ++j) {
-                ok = mbar_wait(&bar_s[t], (uint32_t)((bt + j) & 1), abort_flag);
+                // one-tile blocks alternate between two S buffers (TMEM columns 0 and 128)
+                const int sb = C::kTiles == 1 ? (j & 1) : t;
+                const uint32_t tSb = C::kTiles == 1 ? tmem + lane_off + 128u * (uint32_t)sb : tS;
+                const uint32_t sph = C::kTiles == 1 ? (uint32_t)((su[sb] + (j >> 1)) & 1) : (uint32_t)((bt + j) & 1);
+                ok = mbar_wait(&bar_s[sb], sph, abort_flag);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok)
                     break;
                 tc_fence_after();
                 uint32_t sr[128];
-                tmem_ld128(tS, sr);
+                tmem_ld128(tSb, sr);
                 float s[128];
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
@@ -510,6 +609,14 @@ __global__ void __launch_bounds__(384, 1)
                     l *= a;
                 }
                 if (__any_sync(0xffffffffu, resc)) {
+                    if constexpr (C::kTiles == 1) {
+                        // S(j) ran ahead of P.V(j - 1): O may be rescaled once that is done
+                        ok = mbar_wait(&bar_o[1], (uint32_t)((bt + j - 1) & 1), abort_flag);
+                        ok = __all_sync(0xffffffffu, ok);
+                        if (!ok)
+                            break;
+                        tc_fence_after();
+                    }
 #pragma unroll 1
                     for (int c0 = 0; c0 < D; c0 += 32) {
                         uint32_t o[32];
@@ -544,12 +651,12 @@ __global__ void __launch_bounds__(384, 1)
                         acc = fadd2(acc, fadd2(p0, p1));
                         pk[c] = pack_e4m3x4(p0.x, p0.y, p1.x, p1.y);
                     }
-                    tmem_st16(tS + (uint32_t)(16 * hf), pk);
+                    tmem_st16(tSb + (uint32_t)(16 * hf), pk);
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0)
-                        mbar_arrive(&bar_p[2 * t + hf]);
+                        mbar_arrive(&bar_p[2 * sb + hf]);
                 };
                 auto half_block_16 = [&](int hf, auto use_poly) {
                     uint32_t pk[32];
@@ -565,12 +672,12 @@ __global__ void __launch_bounds__(384, 1)
                         acc = fadd2(acc, pv);
                         pk[c] = Elt<T>::pack(pv.x, pv.y);
                     }
-                    tmem_st32(tS + (uint32_t)(32 * hf), pk);
+                    tmem_st32(tSb + (uint32_t)(32 * hf), pk);
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0)
-                        mbar_arrive(&bar_p[2 * t + hf]);
+                        mbar_arrive(&bar_p[2 * sb + hf]);
                 };
                 auto half_block = [&](int hf, auto use_poly) {
                     if constexpr (F8)
@@ -635,6 +742,8 @@ __global__ void __launch_bounds__(384, 1)
                     p.lse[row] = -INFINITY;
             }
             bt += nb;
+            su[0] += (nb + 1) / 2;
+            su[1] += nb / 2;
         }
     }
 
