@@ -279,7 +279,7 @@ def run_reference(args, rank, world):
 # ncu capture of this bench command on the current kernel (dram__bytes_read.sum +
 # dram__bytes_write.sum, the first timed-step launch); to be taken again whenever the
 # kernel changes.
-BWD_MAIN_DRAM_BYTES = 755.39e6 + 371.92e6
+BWD_MAIN_DRAM_BYTES = 699.24e6 + 321.14e6
 
 
 def run_libfa(args, rank, world, local):

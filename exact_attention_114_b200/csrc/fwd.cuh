@@ -31,8 +31,13 @@
 // neighbouring tiles' work instead of leaving the tensor core idle.
 //
 // At d = 256 the CTA holds one query tile (kTiles = 1): its O accumulator takes
-// 256 TMEM columns, so there is no room for a second tile's S and O; the second
-// softmax warpgroup then has no work, and the MMA order is S(0) | PV(j) S(j+1).
+// 256 TMEM columns, so there is no room for a second tile's S and O, and the
+// second softmax warpgroup has no work.  The other 256 columns hold two S
+// buffers instead: block j's S goes to buffer j & 1 and the MMA order is
+// S(0) S(1) | PV(j) S(j+2) | ..., so each block's Q.K^T runs during the previous
+// block's softmax.  K and V then keep fixed ring slots (K in 0, V in 1), loaded
+// in the order the MMAs free them, and a softmax that rescales O first waits for
+// the previous block's P.V (S(j) no longer follows it).
 //
 // Scores are kept in the log2 domain: x = s * scale * log2(e), p = 2^(x - m).
 // Rescaling is lazy: the reference max m moves (and U, l are multiplied by
