@@ -120,3 +120,28 @@ def test_large_headdim_sampled_long():
     rk, rv = oracle.bwd_dkv_rows(x["q"], x["k"], x["v"], x["dout"], w.scale, True, keys)
     G.assert_grad(G.f64(dk).reshape(-1, w.d)[keys], rk, "dK (sampled keys)")
     G.assert_grad(G.f64(dv).reshape(-1, w.d)[keys], rv, "dV (sampled keys)")
+
+
+@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+def test_forward_rescale_every_block(d, causal):
+    """Scores that climb by 6 (natural-log units, 8.7 in log2) from each 128-key
+    block to the next: every block's row max passes the lazy-rescale threshold,
+    so O is rescaled at every block.  At d = 256 (two S buffers, S(j) issued
+    ahead of P.V(j - 1)) each rescale first waits for the previous block's P.V;
+    d = 128 (two query tiles) is the control."""
+    B, Hq, Hkv, N = 1, 2, 1, 1024
+    scale = 1.0 / d ** 0.5
+    g = torch.Generator().manual_seed(20261203 + d + int(causal))
+    q = 0.1 * torch.randn(B, Hq, N, d, generator=g)
+    q[..., 0] = 1.0
+    k = torch.randn(B, Hkv, N, d, generator=g)
+    k[..., 0] = (6.0 / scale) * (torch.arange(N) // 128).float()   # s ~ 6 j on key block j
+    v = torch.randn(B, Hkv, N, d, generator=g)
+    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+    o, lse = fa.fa_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    fa.fa_check_device_status()
+    o_ref, lse_ref = oracle.fwd(q, k, v, scale, causal)
+    G.assert_o(G.f64(o), o_ref, o_abs=G.o_abs_ref(q, k, v, scale, causal))
+    G.assert_lse(G.f64(lse), lse_ref)
