@@ -145,3 +145,32 @@ def test_forward_rescale_every_block(d, causal):
     o_ref, lse_ref = oracle.fwd(q, k, v, scale, causal)
     G.assert_o(G.f64(o), o_ref, o_abs=G.o_abs_ref(q, k, v, scale, causal))
     G.assert_lse(G.f64(lse), lse_ref)
+
+
+def test_large_headdim_bench_shape():
+    """The step workload's shape at head size 256 as the benchmark times it (B=1,
+    Hq=32, Hkv=8, N=8192, causal; the feature-split backward walks 512 steps per
+    CTA of key block 0): forward on sampled rows, dQ on sampled rows, dK / dV on
+    the heaviest and the last keys of the first and last kv heads, and the dV
+    column-sum identity."""
+    w = synth.WORKLOADS["gqa_8k"].with_(name="gqa_8k_d256", d=256)
+    x = synth.make_inputs(w)
+    xd = G.to_gpu(x)
+    o, lse = G.gpu_forward(xd, w)
+    rows = G.sample_rows(w, n_random=16)
+    o_ref, lse_ref = oracle.fwd(x["q"], x["k"], x["v"], w.scale, True, rows=rows)
+    G.assert_o(G.f64(o).reshape(-1, w.d)[rows], o_ref,
+               o_abs=G.o_abs_ref(x["q"], x["k"], x["v"], w.scale, True, rows=rows))
+    G.assert_lse(G.f64(lse).reshape(-1)[rows], lse_ref)
+    dq, dk, dv = G.gpu_backward(xd, o, lse, w)
+    rq = oracle.bwd_dq_rows(x["q"], x["k"], x["v"], x["dout"], w.scale, True, rows)
+    G.assert_grad(G.f64(dq).reshape(-1, w.d)[rows], rq, "dQ (sampled rows)")
+    keys = np.concatenate([G.sample_keys_heavy(w, kv_heads=(0, w.Hkv - 1)),
+                           G.sample_keys_cheap(w, kv_heads=(0, w.Hkv - 1))])
+    rk, rv = oracle.bwd_dkv_rows(x["q"], x["k"], x["v"], x["dout"], w.scale, True, keys)
+    G.assert_grad(G.f64(dk).reshape(-1, w.d)[keys], rk, "dK (sampled keys)")
+    G.assert_grad(G.f64(dv).reshape(-1, w.d)[keys], rv, "dV (sampled keys)")
+    want = x["dout"].double().reshape(w.B, w.Hkv, w.G, w.Nq, w.d).sum(dim=(2, 3))
+    got = dv.double().cpu().sum(dim=2)
+    err = (got - want).abs().max().item()
+    assert err <= 1e-2 * want.abs().max().item() + 0.05 * np.sqrt(w.Nk), err
