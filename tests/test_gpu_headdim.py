@@ -174,3 +174,39 @@ def test_large_headdim_bench_shape():
     got = dv.double().cpu().sum(dim=2)
     err = (got - want).abs().max().item()
     assert err <= 1e-2 * want.abs().max().item() + 0.05 * np.sqrt(w.Nk), err
+
+
+LONG_256 = [
+    # B, Hq, Hkv, Nq, Nk, causal, dtype
+    (1, 8, 2, 2048, 2048, False, torch.bfloat16),   # every query block for every key block
+    (1, 8, 4, 2048, 2048, True, torch.float16),
+    (1, 4, 1, 1000, 3000, True, torch.bfloat16),     # bottom-right mask, Nq < Nk
+    (1, 4, 2, 2500, 700, True, torch.bfloat16),      # Nq > Nk: early rows see no key
+]
+
+
+@pytest.mark.parametrize("shape", LONG_256, ids=[f"{s[:6]}-{'fp16' if s[6] == torch.float16 else 'bf16'}"
+                                                 for s in LONG_256])
+def test_large_headdim_long_variants(shape):
+    """d = 256 forward and backward at multi-wave sizes beyond the causal,
+    square bf16 cases: non-causal (every step slot and both feature halves
+    over all query blocks), fp16, and Nq != Nk with the bottom-right mask.
+    Sampled query rows (O, LSE, dQ) and the heaviest and last keys (dK, dV)."""
+    B, Hq, Hkv, Nq, Nk, causal, dtype = shape
+    w = synth.Workload("headdim_long_v", B, Hq, Hkv, Nq, Nk, 256, causal, 6460 + Nq + Nk)
+    x = synth.make_inputs(w, dtype=dtype)
+    xd = G.to_gpu(x)
+    o, lse = G.gpu_forward(xd, w)
+    rows = G.sample_rows(w, n_random=12)
+    o_ref, lse_ref = oracle.fwd(x["q"], x["k"], x["v"], w.scale, causal, rows=rows)
+    G.assert_o(G.f64(o).reshape(-1, w.d)[rows], o_ref,
+               o_abs=G.o_abs_ref(x["q"], x["k"], x["v"], w.scale, causal, rows=rows))
+    G.assert_lse(G.f64(lse).reshape(-1)[rows], lse_ref)
+    dq, dk, dv = G.gpu_backward(xd, o, lse, w)
+    rq = oracle.bwd_dq_rows(x["q"], x["k"], x["v"], x["dout"], w.scale, causal, rows)
+    G.assert_grad(G.f64(dq).reshape(-1, w.d)[rows], rq, "dQ (sampled rows)")
+    keys = np.concatenate([G.sample_keys_heavy(w, kv_heads=(0, w.Hkv - 1)),
+                           G.sample_keys_cheap(w, kv_heads=(0, w.Hkv - 1))])
+    rk, rv = oracle.bwd_dkv_rows(x["q"], x["k"], x["v"], x["dout"], w.scale, causal, keys)
+    G.assert_grad(G.f64(dk).reshape(-1, w.d)[keys], rk, "dK (sampled keys)")
+    G.assert_grad(G.f64(dv).reshape(-1, w.d)[keys], rv, "dV (sampled keys)")
