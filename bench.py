@@ -492,9 +492,11 @@ def run_libfa(args, rank, world, local):
     # long MHA one (B=2, H=32, N=4096, d=128, causal, every 64th query row x8) held
     # to the same bar, and the d = 64 MHA one (B=4, H=16, N=1024), causal and not
     other = {}
-    # the step workload's shape at head size 256 (the feature-split backward)
-    extra = {"gqa_8k_d256": synth.WORKLOADS[STEP_WORKLOAD].with_(name="gqa_8k_d256", d=256)}
-    for name in ("mha_4k_long", "mha_1k", "mha_1k_noncausal", "gqa_8k_d256"):
+    # the step workload's shape at head size 256 (the feature-split backward), and
+    # without the causal mask (the backward shares each unit between two CTAs there)
+    extra = {"gqa_8k_d256": synth.WORKLOADS[STEP_WORKLOAD].with_(name="gqa_8k_d256", d=256),
+             "gqa_8k_noncausal": synth.WORKLOADS[STEP_WORKLOAD].with_(name="gqa_8k_noncausal", causal=False)}
+    for name in ("mha_4k_long", "mha_1k", "mha_1k_noncausal", "gqa_8k_d256", "gqa_8k_noncausal"):
         base = extra.get(name) or synth.WORKLOADS[name]
         wo = base.with_(seed=rank_seed(base.seed, rank))
         xo = {k_: v_.to(dev) for k_, v_ in synth.make_inputs(wo).items()}
@@ -519,6 +521,8 @@ def run_libfa(args, rank, world, local):
         b_ms = statistics.median(timed(bo, max(10, args.steps)))
         other[name] = {"workload": f"B={wo.B}, Hq={wo.Hq}, Hkv={wo.Hkv}, N={wo.Nq}, d={wo.d}, "
                                    f"{'causal' if wo.causal else 'non-causal'}",
+                       "bwd_query_split": fa.fa_bwd_query_split(wo.B, wo.Hq, wo.Hkv, wo.Nq, wo.Nk, wo.d,
+                                                                wo.causal),
                        "fwd_ms": f_ms, "fwd_tflops": wo.fwd_flops() / (f_ms * 1e-3) / 1e12,
                        "bwd_ms": b_ms, "bwd_tflops": wo.bwd_flops() / (b_ms * 1e-3) / 1e12}
         del xo, oo, lo, go, wso

@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
             L.fa_fwd_paged_ex.restype = ip
             L.fa_bwd_workspace_size.argtypes = [ip, ip, ip, ip, ip, ip]
             L.fa_bwd_workspace_size.restype = sz
+            L.fa_bwd_query_split.argtypes = [ip, ip, ip, ip, ip, ip, ip]
+            L.fa_bwd_query_split.restype = ip
             L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, fl, ip,
                                  vp, sz, vp]
             L.fa_bwd.restype = ip
@@ -331,6 +333,12 @@ def fa_fwd_splitkv_noalloc(q, k, v, o, lse, *, causal=False, scale=None, num_spl
 
 def fa_bwd_workspace_size(B, Hq, Hkv, Nq, Nk, d) -> int:
     return int(lib().fa_bwd_workspace_size(B, Hq, Hkv, Nq, Nk, d))
+
+
+def fa_bwd_query_split(B, Hq, Hkv, Nq, Nk, d, causal) -> int:
+    """CTAs that fa_bwd shares each (key block, kv head) unit between on the
+    current device, given a full-size workspace (1: no split; 0: bad sizes)."""
+    return int(lib().fa_bwd_query_split(B, Hq, Hkv, Nq, Nk, d, int(bool(causal))))
 
 
 def fa_bwd(q, k, v, o, dout, lse, dq=None, dk=None, dv=None, *, causal=False, scale=None,

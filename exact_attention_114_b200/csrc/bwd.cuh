@@ -15,6 +15,15 @@
 //             reduction over query heads needs no atomics.
 //   bwd_post  dQ = bf16(scale * accumulator).
 //
+// Query split: when there are too few (key block, kv head) units to fill the SMs, or
+// their count leaves a last round of CTAs with most SMs idle, q_split CTAs share a
+// unit, each walking a contiguous share of its (query head, query block) steps.  Their
+// dK / dV sums meet in an fp32 workspace: each takes a ticket when its steps are done;
+// all but the last store their sums (16-byte columns, lane after lane) and count
+// themselves; the last waits for that count (bounded), adds the partials in a fixed
+// order and writes dK / dV.  The last waits only for CTAs that have finished their
+// steps, so the wait cannot depend on a CTA that is not yet running.
+//
 // bwd_main roles (384 threads = 3 warpgroups):
 //   warps 0-3  thread r = key r = TMEM lane r: read S^T and dP^T rows from TMEM,
 //              write P^T (bf16) back over S^T in TMEM and dS^T (bf16) into
@@ -102,6 +111,11 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdParams p)
     const T* po = static_cast<const T*>(p.o);
     const T* pd = static_cast<const T*>(p.dout);
     float s[2] = {0.f, 0.f};
+    if (p.q_split > 1) {
+        for (int i = (int)(blockIdx.x * blockDim.x + threadIdx.x); i < 2 * p.n_split_units;
+             i += (int)(gridDim.x * blockDim.x))
+            p.split_cnt[i] = 0;
+    }
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
         const int row = row0 + r;
@@ -270,7 +284,9 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int chunk)
     return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-template <int D, bool CAUSAL, typename T = __nv_bfloat16>
+// SPLIT: the launch shares units between CTAs (q_split > 1); without it the kernel
+// carries none of the split's code
+template <int D, bool CAUSAL, typename T = __nv_bfloat16, bool SPLIT = false>
 __global__ void __launch_bounds__(384, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -305,13 +321,16 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* bar_qfree = bars + 19;   // [2]
     uint64_t* bar_dofree = bars + 21;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* split_word = reinterpret_cast<int*>(bars + 22);   // query split: the ticket, to the compute warps
 
     const int warp = warp_id(), lane = lane_id();
-    const int n_kb = (p.Nk + 127) / 128;
-    const int units = p.B * p.Hkv * C::kFeatSplit;
-    const int kb = (int)blockIdx.x / units;   // small key blocks (most work) first
-    const int kvh = ((int)blockIdx.x % units) / C::kFeatSplit;
-    const int fh = ((int)blockIdx.x % units) % C::kFeatSplit;   // feature half (head size 256)
+    const int nsp = SPLIT ? p.q_split : 1;                         // CTAs per unit
+    const int units = p.B * p.Hkv * C::kFeatSplit;                 // units per key block
+    const int kb = (int)blockIdx.x / (units * nsp);   // small key blocks (most work) first
+    const int ui = ((int)blockIdx.x % (units * nsp)) / nsp;
+    const int sp = (int)blockIdx.x % nsp;                          // share of the unit's steps
+    const int kvh = ui / C::kFeatSplit;
+    const int fh = ui % C::kFeatSplit;   // feature half (head size 256)
     const int b = kvh / p.Hkv, hk = kvh % p.Hkv;
     int qb0, nqb;
     bwd_q_range(p, kb, qb0, nqb);
@@ -319,8 +338,10 @@ __global__ void __launch_bounds__(384, 1)
         qb0 = 0;
         nqb = p.Nq_pad / 64;
     }
-    const int n_it = p.G * nqb;
-    (void)n_kb;
+    // steps it_lo .. it_lo + n_it - 1 of the unit's G * nqb (query head, query block) steps
+    const int n_all = p.G * nqb;
+    const int it_lo = (int)(((long long)sp * n_all) / nsp);
+    const int n_it = (int)(((long long)(sp + 1) * n_all) / nsp) - it_lo;
 
     if (threadIdx.x == 0) {
         mbar_init(bar_kv, 1);
@@ -358,8 +379,9 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tmem = *tmem_slot;
 
     auto step_coords = [&](int it, int& h, int& qb) {
-        h = hk * p.G + it / nqb;
-        qb = qb0 + it % nqb;
+        const int g = it_lo + it;
+        h = hk * p.G + g / nqb;
+        qb = qb0 + g % nqb;
     };
 
     // Each role runs inside the branch that sets its register budget.
@@ -746,15 +768,53 @@ __global__ void __launch_bounds__(384, 1)
             if (lane == 0)
                 mbar_arrive(&bar_ds[it & 1]);
         }
-        // ---- epilogue: dK = scale * acc, dV = acc  (bf16)
+        // ---- epilogue: dK = scale * acc, dV = acc  (bf16).  With q_split > 1 each CTA
+        // of the unit holds the sums over its own steps: the first q_split - 1 to get
+        // here leave theirs in fp32 in the workspace, and the last adds them in.
         if (ok) {
             ok = mbar_wait(bar_final, 0, abort_flag);
             ok = __all_sync(0xffffffffu, ok);
+        }
+        int ticket = nsp - 1;   // the last CTA of the unit (the only one without a split)
+        // the unit's counters, from the block index again (nothing kept live over the steps)
+        const int unit_e = SPLIT ? (int)(ctaid_x() / (uint32_t)nsp) : 0;
+        int* n_written = SPLIT ? p.split_cnt + p.n_split_units + unit_e : nullptr;
+        if (SPLIT && nsp > 1) {
+            ok = named_bar_and(3, 128, ok);   // the four warps go on together
+            if (threadIdx.x == 0)
+                *split_word = atomicAdd(&p.split_cnt[unit_e], 1);
+            named_bar_sync(3, 128);
+            ticket = *split_word;
+            if (ok && ticket == nsp - 1) {
+                // the others took their tickets after their last step and only store
+                // and count from there, so this wait ends unless one of them gave up
+                bool got = true;
+                if (threadIdx.x == 0) {
+                    const long long t0 = clock64();
+                    while (ld_acquire_gpu(n_written) < nsp - 1) {
+                        if (clock64() - t0 > FA_WAIT_LIMIT_CYCLES) {
+                            atomicOr(&g_status, kStatusTimeout);
+                            got = false;
+                            break;
+                        }
+                        __nanosleep(128);
+                    }
+                }
+                ok = named_bar_and(3, 128, got);
+                __threadfence();
+            }
         }
         if (ok) {
             tc_fence_after();
             const bool key_ok = key < p.Nk;
             const int d_io = p.d_io;
+            constexpr int kPart4 = 2 * C::kDO / 4 * 128;   // float4 per partial
+            // partial slots: one per unit for two shares (the last CTA adds the other's to
+            // its own, and a + b = b + a); one per share for more, all stored and added in
+            // share order, so that dK / dV do not depend on which CTA finishes last
+            const int nslot = nsp == 2 ? 1 : nsp;
+            const int my_slot = (!SPLIT || nsp == 2) ? 0 : (int)(ctaid_x() % (uint32_t)nsp);
+            float4* part = SPLIT ? p.dkv_part + (size_t)unit_e * (size_t)nslot * kPart4 + r : nullptr;
 #pragma unroll 1
             for (int c0 = 0; c0 < C::kDO; c0 += 32) {
                 const int col = fh * C::kDO + c0;   // feature of the tensors in memory
@@ -769,6 +829,53 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
                     for (int c = 0; c < 32; ++c)
                         a[c] = v[c] = 0u;
+                }
+                // a partial is [dK chunks | dV chunks][128 keys] of 4 floats: lane r of a
+                // warp stores or loads the 16 bytes after lane r - 1's (each thread reads
+                // back only what it or another CTA's thread r stored)
+                const int ck = c0 / 4, cv = C::kDO / 4 + c0 / 4;
+                if (SPLIT && nsp > 1) {
+                    if (ticket < nsp - 1 || nsp > 2) {
+                        float4* out = part + (size_t)my_slot * kPart4;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            __stcg(out + (ck + j) * 128, make_float4(__uint_as_float(a[4 * j]), __uint_as_float(a[4 * j + 1]),
+                                                                     __uint_as_float(a[4 * j + 2]), __uint_as_float(a[4 * j + 3])));
+                            __stcg(out + (cv + j) * 128, make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                                     __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
+                        }
+                    }
+                    if (ticket < nsp - 1)
+                        continue;
+                    // the last: two shares add the other's partial to this one; more start
+                    // from share 0's and add the rest in order (this CTA's own included)
+#pragma unroll 1
+                    for (int o = (nsp == 2 ? 0 : 1); o < nslot; ++o) {
+                        const float4* in = part + (size_t)o * kPart4;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const float4 x = __ldcg(in + (ck + j) * 128), y = __ldcg(in + (cv + j) * 128);
+                            if (nsp > 2 && o == 1) {
+                                const float4 x0 = __ldcg(part + (ck + j) * 128), y0 = __ldcg(part + (cv + j) * 128);
+                                a[4 * j] = __float_as_uint(x0.x);
+                                a[4 * j + 1] = __float_as_uint(x0.y);
+                                a[4 * j + 2] = __float_as_uint(x0.z);
+                                a[4 * j + 3] = __float_as_uint(x0.w);
+                                v[4 * j] = __float_as_uint(y0.x);
+                                v[4 * j + 1] = __float_as_uint(y0.y);
+                                v[4 * j + 2] = __float_as_uint(y0.z);
+                                v[4 * j + 3] = __float_as_uint(y0.w);
+                            }
+                            a[4 * j] = __float_as_uint(__uint_as_float(a[4 * j]) + x.x);
+                            a[4 * j + 1] = __float_as_uint(__uint_as_float(a[4 * j + 1]) + x.y);
+                            a[4 * j + 2] = __float_as_uint(__uint_as_float(a[4 * j + 2]) + x.z);
+                            a[4 * j + 3] = __float_as_uint(__uint_as_float(a[4 * j + 3]) + x.w);
+                            v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + y.x);
+                            v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + y.y);
+                            v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + y.z);
+                            v[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) + y.w);
+                        }
+                    }
                 }
                 if (key_ok) {
                     uint32_t wk[16], wv[16];
@@ -786,6 +893,14 @@ __global__ void __launch_bounds__(384, 1)
                     }
                 }
             }
+        }
+        if (SPLIT && nsp > 1 && ticket < nsp - 1) {
+            // publish the partial: every thread's stores, then the count (also after a
+            // give-up, so that the last CTA does not wait out its limit)
+            __threadfence();
+            named_bar_sync(3, 128);
+            if (threadIdx.x == 0)
+                atomicAdd(n_written, 1);
         }
     } else {
         regs_dec<C::kRegsDQ>();

@@ -563,10 +563,58 @@ fa_status_t noalloc_scratch(void** out)
 // ---------------------------------------------------------------------------
 struct BwdPlan {
     int Nq_pad;
-    size_t delta_off, lse_off, acc_off, total;
+    size_t delta_off, lse_off, acc_off, total;   // total: without a query split
+    // query split (q_split[causal] CTAs per unit): fp32 dK / dV partials and the two
+    // counters per unit, after the accumulator, sized for the larger of the two splits
+    int q_split[2], n_units;
+    size_t part_off, cnt_off, total_split;
 };
 
-BwdPlan bwd_plan(int B, int Hq, int Nq, int d)
+// CTAs that share each (key block, kv head[, feature half]) unit's query steps.  A unit of
+// key block kb has G * (visible 64-row query blocks) steps; a CTA costs its steps plus a
+// fixed part (set-up, pipeline fill, dK / dV epilogue: about 8.5 step times) and, when
+// split, about 0.8 step times per fp32 partial it stores or adds.  Without a causal mask
+// all units are alike and the launch takes ceil(CTAs / SMs) rounds of one CTA; with it
+// the estimate is the larger of the total work over the SMs and the longest CTA.  The
+// split of least estimated time is taken if it saves at least 3% (each CTA keeps at
+// least 16 steps): it fills the SMs when there are few units, and evens out a last
+// round that would leave most of them idle.
+int bwd_q_split(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, int sms)
+{
+    const int kd = kernel_d(d);
+    const int n_kb = (Nk + 127) / 128;
+    const double per_kb = (double)B * Hkv * (kd == 256 ? 2 : 1);
+    const int G = Hq / Hkv, nqb_all = (Nq + 63) / 64;
+    double total = 0, longest = 0;
+    for (int kb = 0; kb < n_kb; ++kb) {
+        int qb0 = 0;
+        if (causal) {
+            const int first_row = kb * 128 - (Nk - Nq);
+            qb0 = first_row <= 0 ? 0 : first_row / 64;
+        }
+        const double steps = (double)G * std::max(0, nqb_all - qb0);
+        total += steps * per_kb;
+        longest = std::max(longest, steps);
+    }
+    static const int kSplits[] = {1, 2, 3, 4, 6, 8};
+    int best = 1;
+    double best_cost = 0;
+    for (int s : kSplits) {
+        if (s > 1 && longest < 16.0 * s)
+            break;
+        const double fixed = 8.5 + (s > 1 ? 0.8 * (s - 1) : 0.0);
+        const double ctas = n_kb * per_kb * s;
+        const double cost = causal ? std::max((total + ctas * fixed) / sms, longest / s + fixed)
+                                   : std::ceil(ctas / sms) * (longest / s + fixed);
+        if (s == 1 || cost < 0.97 * best_cost) {
+            best = s;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
+
+BwdPlan bwd_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d)
 {
     BwdPlan pl;
     pl.Nq_pad = (Nq + 63) / 64 * 64;
@@ -575,6 +623,18 @@ BwdPlan bwd_plan(int B, int Hq, int Nq, int d)
     pl.lse_off = align256(rows * 4);
     pl.acc_off = pl.lse_off + align256(rows * 4);
     pl.total = pl.acc_off + align256(rows * kernel_d(d) * 4);   // accumulator rows of the kernel width
+    const int kd = kernel_d(d);
+    pl.n_units = ((Nk + 127) / 128) * B * Hkv * (kd == 256 ? 2 : 1);
+    const int sms = sm_count();
+    pl.q_split[0] = bwd_q_split(B, Hq, Hkv, Nq, Nk, d, 0, sms);
+    pl.q_split[1] = bwd_q_split(B, Hq, Hkv, Nq, Nk, d, 1, sms);
+    const int most = std::max(pl.q_split[0], pl.q_split[1]);
+    // partial slots per unit: one for two shares, one per share for more
+    const int slots = most == 1 ? 0 : most == 2 ? 1 : most;
+    const size_t part_bytes = (size_t)pl.n_units * slots * 2 * std::min(kd, 128) * 128 * 4;
+    pl.part_off = pl.total;
+    pl.cnt_off = pl.part_off + align256(part_bytes);
+    pl.total_split = most > 1 ? pl.cnt_off + align256((size_t)pl.n_units * 2 * 4) : pl.total;
     return pl;
 }
 
@@ -594,9 +654,9 @@ fa_status_t launch_bwd(const fa::BwdParams& p, const void* q, const void* k, con
     if ((st = make_map(&mdo, dout, p.d_io, p.Nq, (uint64_t)p.B * p.Hq, 64, dt)) != FA_OK) return st;
     if ((st = make_map(&mk, k, p.d_io, p.Nk, (uint64_t)p.B * p.Hkv, 128, dt)) != FA_OK) return st;
     if ((st = make_map(&mv, v, p.d_io, p.Nk, (uint64_t)p.B * p.Hkv, 128, dt)) != FA_OK) return st;
-    auto kern = fa::bwd_main_kernel<D, CAUSAL, T>;
+    auto kern = p.q_split > 1 ? fa::bwd_main_kernel<D, CAUSAL, T, true> : fa::bwd_main_kernel<D, CAUSAL, T, false>;
     if ((st = ensure_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes)) != FA_OK) return st;
-    const long long grid = (long long)((p.Nk + 127) / 128) * p.B * p.Hkv * C::kFeatSplit;
+    const long long grid = (long long)((p.Nk + 127) / 128) * p.B * p.Hkv * C::kFeatSplit * p.q_split;
     kern<<<(unsigned)grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mdo, p);
     if ((st = check_launch("bwd_main_kernel launch")) != FA_OK) return st;
 
@@ -982,7 +1042,15 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d)
 {
     if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || Hq % Hkv != 0 || d < 1 || d > 256)
         return 0;
-    return bwd_plan(B, Hq, Nq, d).total;
+    return bwd_plan(B, Hq, Hkv, Nq, Nk, d).total_split;
+}
+
+int fa_bwd_query_split(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || Hq % Hkv != 0 || d < 1 || d > 256 ||
+        (causal != 0 && causal != 1))
+        return 0;
+    return bwd_plan(B, Hq, Hkv, Nq, Nk, d).q_split[causal];
 }
 
 static fa_status_t bwd_entry(int dtype, const void* q, const void* k, const void* v, const void* o,
@@ -1006,16 +1074,18 @@ static fa_status_t bwd_entry(int dtype, const void* q, const void* k, const void
         set_error("workspace is not 256-byte aligned");
         return FA_ERR_INVALID_ARGUMENT;
     }
-    const BwdPlan pl = bwd_plan(B, Hq, Nq, d);
+    const BwdPlan pl = bwd_plan(B, Hq, Hkv, Nq, Nk, d);
     if (workspace && workspace_bytes < pl.total) {
         set_error("workspace has %zu bytes, %zu needed", workspace_bytes, pl.total);
         return FA_ERR_WORKSPACE;
     }
+    // the query split needs the partials' room too: a smaller workspace runs without it
+    const int q_split = (!workspace || workspace_bytes >= pl.total_split) ? pl.q_split[causal ? 1 : 0] : 1;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     void* ws = workspace;
     bool owned = false;
     if (!ws) {
-        cudaError_t e = cudaMallocAsync(&ws, pl.total, s);
+        cudaError_t e = cudaMallocAsync(&ws, q_split > 1 ? pl.total_split : pl.total, s);
         if (e != cudaSuccess)
             return cuda_fail(e, "cudaMallocAsync (backward workspace)");
         owned = true;
@@ -1045,6 +1115,10 @@ static fa_status_t bwd_entry(int dtype, const void* q, const void* k, const void
     p.causal = causal;
     p.scale = scale;
     p.scale_log2 = scale * kLog2e;
+    p.q_split = q_split;
+    p.n_split_units = pl.n_units;
+    p.dkv_part = q_split > 1 ? reinterpret_cast<float4*>(w + pl.part_off) : nullptr;
+    p.split_cnt = q_split > 1 ? reinterpret_cast<int*>(w + pl.cnt_off) : nullptr;
     st = dtype == FA_DTYPE_FP16 ? bwd_dispatch<__half>(p, q, k, v, dout, kernel_d(d), causal, s)
                                 : bwd_dispatch<__nv_bfloat16>(p, q, k, v, dout, kernel_d(d), causal, s);
     if (owned) {

@@ -68,6 +68,13 @@ struct BwdParams {
     int causal;
     float scale;
     float scale_log2;
+    // q_split CTAs share each (key block, kv head[, feature half]) unit, each walking
+    // its own share of the unit's query steps; all but the last to finish leave their
+    // fp32 dK / dV sums in dkv_part, and the last adds them up (q_split = 1: no split)
+    int q_split;
+    int n_split_units;          // units of the launch (q_split > 1)
+    float4* dkv_part;           // [n_split_units][q_split == 2 ? 1 : q_split][2 * dK/dV features / 4][128]
+    int* split_cnt;             // [2][n_split_units]: tickets taken, partials written
 };
 
 }  // namespace fa

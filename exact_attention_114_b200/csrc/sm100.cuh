@@ -563,6 +563,23 @@ __device__ __forceinline__ void regs_dec()
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// the block index, read where it is used (a volatile read is not merged with an
+// earlier one, so the value need not stay live in a register up to here)
+__device__ __forceinline__ uint32_t ctaid_x()
+{
+    uint32_t v;
+    asm volatile("mov.u32 %0, %%ctaid.x;" : "=r"(v));
+    return v;
+}
+
+// load with acquire semantics at GPU scope (pairs with a writer's fence + atomic)
+__device__ __forceinline__ int ld_acquire_gpu(const int* ptr)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
 // barrier over a subset of the block's warps (ids 1..15; 0 is __syncthreads)
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads)
 {

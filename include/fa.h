@@ -242,14 +242,30 @@ fa_status_t fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, 
  *   scale and causal flag.
  *   dq [B,Hq,Nq,d], dk/dv [B,Hkv,Nk,d] (bf16, written).  dk/dv are summed over
  *   the Hq / Hkv query heads of each kv group.
- *   workspace: device scratch of at least fa_bwd_workspace_size(...) bytes,
- *   256-byte aligned (it holds D = rowsum(dout * o) and the fp32 dq
- *   accumulator); NULL makes the call allocate it stream-ordered.
+ *   workspace: device scratch of fa_bwd_workspace_size(...) bytes, 256-byte
+ *   aligned (it holds D = rowsum(dout * o), the fp32 dq accumulator and, for
+ *   the query split below, fp32 dk / dv partials); NULL makes the call
+ *   allocate it stream-ordered.  A workspace smaller than that but large
+ *   enough without the partials (D, LSE and the accumulator) runs unsplit.
+ *   Query split: where there are too few (key block, kv head) units to fill
+ *   the GPU, or their count would leave a last round of CTAs with most SMs
+ *   idle, fa_bwd_query_split(...) CTAs share each unit's query steps and the
+ *   last of them adds the others' partials in a fixed order, so dk / dv still
+ *   repeat bitwise from call to call.
  *   For d > 128 the features are split in two halves: each key block is
  *   handled by two CTAs that both recompute S and dP over all d features and
  *   each accumulate their half of dk, dv and dq.
  */
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d);
+
+/*
+ * The number of CTAs that fa_bwd / fa_bwd_ex share each (key block, kv head)
+ * unit between on the current device, given fa_bwd_workspace_size(...) bytes
+ * of workspace (or none, so that the call allocates it): 1 (no split), 2, 3,
+ * 4, 6 or 8.  The choice depends only on the sizes, the causal flag and the
+ * device's SM count.  0 for sizes that fa_bwd would refuse.
+ */
+int fa_bwd_query_split(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal);
 fa_status_t fa_bwd(const void* q, const void* k, const void* v, const void* o,
                    const void* dout, const float* lse, void* dq, void* dk, void* dv,
                    int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,

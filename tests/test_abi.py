@@ -139,11 +139,22 @@ def test_splitkv_noalloc_rejects_before_touching_cuda():
     assert m and int(m[1]) * int(m[2]) * int(m[3]) == fa.NOALLOC_SCRATCH_BYTES
 
 
+def _sm_count():
+    import torch
+    return torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
+
+
 def test_workspace_sizes():
     # backward: D and LSE rows (fp32) + fp32 dQ accumulator, rows padded to 64
     n = fa.fa_bwd_workspace_size(1, 32, 8, 8192, 8192, 128)
     rows = 32 * 8192
-    assert n == rows * 4 * 2 + rows * 128 * 4
+    base = rows * 4 * 2 + rows * 128 * 4
+    if _sm_count() == 148:
+        # without a causal mask the 512 (key block, kv head) units split in two: one
+        # fp32 dK | dV partial per unit (2 x 128 keys x 128 x 4 B) and two counters
+        assert n == base + 512 * 2 * 128 * 128 * 4 + 512 * 2 * 4
+    else:
+        assert n >= base
     assert fa.fa_bwd_workspace_size(1, 1, 1, 65, 65, 64) == 512 * 2 + 128 * 64 * 4  # 65 -> 128 rows
     assert fa.fa_bwd_workspace_size(0, 1, 1, 1, 1, 64) == 0
     # split-KV: one partial (O_s, lse_s) per (b, kv head, split, row); one split needs none
@@ -236,3 +247,28 @@ def test_tile_slot_hook_checks_its_slot_before_any_cuda_call():
         assert "slot" in fa.last_error_message()
     assert L.fa_testhook_tile_slot(3, 0) == fa.FA_OK
     assert L.fa_testhook_tile_slot(-1, 0) == fa.FA_OK
+
+
+def test_backward_query_split_rule():
+    """The split fa_bwd takes on a 148-SM device: none where the units fill
+    the SMs in whole rounds (the causal step workloads), two where 512 equal
+    units would leave a last round of 68 CTAs, and up to eight where a few
+    units would leave most SMs idle; 0 for sizes fa_bwd refuses."""
+    if _sm_count() != 148:
+        pytest.skip("the expected splits are for 148 SMs")
+    qs = fa.fa_bwd_query_split
+    assert qs(1, 32, 8, 8192, 8192, 128, 1) == 1      # gqa_8k causal
+    assert qs(1, 32, 8, 8192, 8192, 128, 0) == 2      # gqa_8k without the mask
+    assert qs(2, 32, 32, 4096, 4096, 128, 1) == 1     # mha_4k_long
+    assert qs(4, 16, 16, 1024, 1024, 64, 0) == 1      # mha_1k: 16 steps per unit
+    assert qs(1, 32, 8, 8192, 8192, 256, 1) == 1
+    assert qs(1, 4, 1, 2048, 2048, 128, 1) == 8       # 16 units
+    assert qs(1, 4, 1, 2048, 2048, 128, 0) == 8
+    assert qs(1, 2, 1, 1536, 1536, 128, 1) == 3
+    assert qs(1, 2, 1, 2048, 2048, 128, 0) == 4
+    assert qs(1, 4, 1, 1536, 1536, 128, 0) == 6
+    assert qs(1, 4, 1, 1000, 3000, 128, 1) == 4       # bottom-right mask, Nq < Nk
+    assert qs(1, 1, 1, 64, 64, 64, 0) == 1
+    assert qs(1, 3, 2, 64, 64, 64, 0) == 0            # Hq not a multiple of Hkv
+    assert qs(1, 2, 1, 64, 64, 288, 0) == 0
+    assert fa.lib().fa_bwd_query_split(1, 2, 1, 64, 64, 64, 2) == 0   # causal flag not 0 / 1
