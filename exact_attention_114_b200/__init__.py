@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
             L.fa_bwd_workspace_size.restype = sz
             L.fa_bwd_query_split.argtypes = [ip, ip, ip, ip, ip, ip, ip]
             L.fa_bwd_query_split.restype = ip
+            L.fa_fwd_kv_split.argtypes = [ip, ip, ip, ip, ip, ip, ip]
+            L.fa_fwd_kv_split.restype = ip
             L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, fl, ip,
                                  vp, sz, vp]
             L.fa_bwd.restype = ip
@@ -333,6 +335,12 @@ def fa_fwd_splitkv_noalloc(q, k, v, o, lse, *, causal=False, scale=None, num_spl
 
 def fa_bwd_workspace_size(B, Hq, Hkv, Nq, Nk, d) -> int:
     return int(lib().fa_bwd_workspace_size(B, Hq, Hkv, Nq, Nk, d))
+
+
+def fa_fwd_kv_split(B, Hq, Hkv, Nq, Nk, d, causal) -> int:
+    """Key shares per work tile of fa_fwd on the current device (1: no split;
+    0: bad sizes)."""
+    return int(lib().fa_fwd_kv_split(B, Hq, Hkv, Nq, Nk, d, int(bool(causal))))
 
 
 def fa_bwd_query_split(B, Hq, Hkv, Nq, Nk, d, causal) -> int:

@@ -234,11 +234,65 @@ int sm_count()
 int kernel_d(int d) { return d <= 64 ? 64 : d <= 128 ? 128 : 256; }
 
 // The forward is persistent: one block per SM (its shared memory allows no
-// second), together working through the n_pairs * B * Hq tiles.
+// second), together working through the n_pairs * B * Hq (* kv_split) tiles.
 unsigned fwd_grid(const fa::FwdParams& p)
 {
-    const long long tiles = (long long)p.n_pairs * p.B * p.Hq;
+    const long long tiles = (long long)p.n_pairs * p.B * p.Hq * p.kv_split;
     return (unsigned)std::max<long long>(1, std::min<long long>(tiles, sm_count()));
+}
+
+// stream-ordered scratch from the library's memory pool (defined below)
+cudaError_t scratch_alloc(void** out, size_t bytes, cudaStream_t s);
+
+// 128-key blocks seen by the 128-row query tile starting at row qt (as the kernel's
+// fwd_blocks_for_tile)
+int host_blocks_for_tile(int qt, int Nq, int Nk, int causal)
+{
+    const int nkb = (Nk + 127) / 128;
+    if (qt >= Nq)
+        return 0;
+    if (!causal)
+        return nkb;
+    const long long last_key = (long long)std::min(qt + 127, Nq - 1) + (Nk - Nq);
+    return last_key < 0 ? 0 : (int)std::min<long long>(nkb, last_key / 128 + 1);
+}
+
+// Key shares per (query tile pair, head) of the tiled forward.  Unsplit, the launch has
+// n_pairs * B * Hq work tiles, each costing its key blocks plus about 2 block times of
+// fixed work (Q load, first S, epilogue).  With fewer tiles than SMs the longest tile
+// bounds the launch, so each is cut into s contiguous shares of its key blocks (at least
+// 2 blocks each), all of them in one round (tiles * s <= SMs), and a second kernel merges
+// them (with the extra launch, about 8 block times more, as measured on small launches).
+// The estimate is max(total / SMs, longest / s + fixed) (+ 8 with a split); the cheapest
+// split that saves 10% on no split is taken, with the fp32 partials held under 256 MB.
+int fwd_kv_split(int B, int Hq, int Nq, int Nk, int d, int causal, int sms)
+{
+    const int kt = kernel_d(d) == 256 ? 1 : 2;
+    const int n_pairs = (Nq + 128 * kt - 1) / (128 * kt);
+    const double bh = (double)B * Hq;
+    double total = 0, longest = 0;
+    for (int pr = 0; pr < n_pairs; ++pr) {
+        int n = 0;
+        for (int t = 0; t < kt; ++t)
+            n = std::max(n, host_blocks_for_tile(pr * 128 * kt + 128 * t, Nq, Nk, causal));
+        total += n * bh;
+        longest = std::max(longest, (double)n);
+    }
+    const double tiles = n_pairs * bh, fixed = 2.0;
+    const double c1 = std::max((total + tiles * fixed) / sms, longest + fixed);
+    static const int kShares[] = {2, 3, 4, 6, 8, 12, 16};
+    int best = 1;
+    double best_cost = c1;
+    for (int sh : kShares) {
+        if (longest < 2.0 * sh || tiles * sh > sms || bh * sh * Nq * d * 4.0 > 256.0 * (1 << 20))
+            break;
+        const double c = std::max((total + tiles * sh * fixed) / sms, longest / sh + fixed) + 8.0;
+        if (c < best_cost && c < 0.9 * c1) {
+            best = sh;
+            best_cost = c;
+        }
+    }
+    return best;
 }
 
 // Test hook state: a slot every tiled forward launch is pinned to (-1: rotate).
@@ -274,7 +328,8 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     if ((st = make_map(&mq, q, d, Nq, (uint64_t)B * Hq, 128, tma_type<T>())) != FA_OK) return st;
     if ((st = make_map(&mk, k, d, Nk, (uint64_t)B * Hkv, 128, tma_type<T>())) != FA_OK) return st;
     if ((st = make_map(&mv, v, d, Nk, (uint64_t)B * Hkv, 128, tma_type<T>())) != FA_OK) return st;
-    auto kern = fa::fwd_kernel<D, CAUSAL, T>;
+    const int kv_split = fwd_kv_split(B, Hq, Nq, Nk, d, CAUSAL, sm_count());
+    auto kern = kv_split > 1 ? fa::fwd_kernel<D, CAUSAL, T, false, true> : fa::fwd_kernel<D, CAUSAL, T, false, false>;
     if ((st = ensure_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes)) != FA_OK) return st;
     fa::FwdParams p;
     p.o = o;
@@ -289,10 +344,35 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     p.d_io = d;
     p.scale_log2 = scale * kLog2e;
     p.o_scale = 1.f;
+    p.kv_split = kv_split;
+    p.part_o = nullptr;
+    p.part_lse = nullptr;
     if ((st = fwd_tile_counter(&p.tile_ctr, &p.tile_tag)) != FA_OK)
         return st;
+    void* ws = nullptr;
+    if (kv_split > 1) {
+        // the shares' partials, stream-ordered scratch
+        const size_t rows = (size_t)B * Hq * kv_split * Nq;
+        const size_t o_bytes = align256(rows * d * 4);
+        cudaError_t e = scratch_alloc(&ws, o_bytes + align256(rows * 4), stream);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "scratch allocation (forward key-split partials)");
+        p.part_o = static_cast<float*>(ws);
+        p.part_lse = reinterpret_cast<float*>(static_cast<char*>(ws) + o_bytes);
+    }
     kern<<<fwd_grid(p), C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
-    return check_launch("fwd_kernel launch");
+    st = check_launch("fwd_kernel launch");
+    if (kv_split > 1) {
+        if (st == FA_OK) {
+            const long long rows = (long long)B * Hq * Nq;
+            fa::fwd_combine_kernel<T><<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(p);
+            st = check_launch("fwd_combine_kernel launch");
+        }
+        cudaError_t e = cudaFreeAsync(ws, stream);
+        if (e != cudaSuccess && st == FA_OK)
+            st = cuda_fail(e, "cudaFreeAsync");
+    }
+    return st;
 }
 
 // ---------------------------------------------------------------------------
@@ -337,6 +417,9 @@ fa_status_t launch_fwd_fp8(const void* q, const void* k, const void* v, void* vt
     p.d_io = kF8D;
     p.scale_log2 = scale_log2;
     p.o_scale = o_scale;
+    p.kv_split = 1;   // no key split for e4m3 inputs
+    p.part_o = nullptr;
+    p.part_lse = nullptr;
     if ((st = fwd_tile_counter(&p.tile_ctr, &p.tile_tag)) != FA_OK)
         return st;
     kern<<<fwd_grid(p), C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
@@ -520,6 +603,54 @@ CtxGetCurrentFn get_ctx_current()
 // on the current CUDA context as well as the device: after cudaDeviceReset the
 // runtime makes a new context, the module (and the array) is loaded again, and
 // the address is looked up again instead of reusing the old one.
+// Stream-ordered scratch of the calls that allocate their own: a memory pool of the
+// library per device (per context: a new one after cudaDeviceReset) that keeps up to
+// kScratchKeepBytes between calls.  The device's default pool gives its free memory back
+// at every synchronisation, so each call after one would map fresh pages again (about
+// 0.2 ms per call measured).  While the stream is being captured into a graph the
+// allocation is left to cudaMallocAsync, whose graph memory nodes are the documented path.
+constexpr uint64_t kScratchKeepBytes = 1ull << 30;
+
+cudaError_t scratch_alloc(void** out, size_t bytes, cudaStream_t s)
+{
+    static std::mutex mu;
+    static cudaMemPool_t pool_of[64] = {};
+    static CUcontext ctx_of[64] = {};
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) {
+        cudaGetLastError();
+        cap = cudaStreamCaptureStatusActive;
+    }
+    int dev = 0;
+    CtxGetCurrentFn get_ctx = get_ctx_current();
+    CUcontext ctx = nullptr;
+    if (cap != cudaStreamCaptureStatusNone || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 ||
+        !get_ctx || get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+        return cudaMallocAsync(out, bytes, s);
+    cudaMemPool_t pool = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (pool_of[dev] == nullptr || ctx_of[dev] != ctx) {
+            cudaMemPoolProps props = {};
+            props.allocType = cudaMemAllocationTypePinned;
+            props.handleTypes = cudaMemHandleTypeNone;
+            props.location.type = cudaMemLocationTypeDevice;
+            props.location.id = dev;
+            cudaMemPool_t p = nullptr;
+            if (cudaMemPoolCreate(&p, &props) != cudaSuccess) {
+                cudaGetLastError();
+                return cudaMallocAsync(out, bytes, s);
+            }
+            uint64_t keep = kScratchKeepBytes;
+            cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
+            pool_of[dev] = p;
+            ctx_of[dev] = ctx;
+        }
+        pool = pool_of[dev];
+    }
+    return cudaMallocFromPoolAsync(out, bytes, pool, s);
+}
+
 fa_status_t noalloc_scratch(void** out)
 {
     static std::mutex mu;
@@ -745,9 +876,9 @@ static fa_status_t fwd_entry(int dtype, const void* q, const void* k, const void
     const DecodePlan pl = decode_plan(B, Hq, Hkv, Nq, Nk, d, 0);
     void* ws = nullptr;
     if (pl.total() > 0) {
-        cudaError_t e = cudaMallocAsync(&ws, pl.total(), s);
+        cudaError_t e = scratch_alloc(&ws, pl.total(), s);
         if (e != cudaSuccess)
-            return cuda_fail(e, "cudaMallocAsync (split-KV partials)");
+            return cuda_fail(e, "scratch allocation (split-KV partials)");
     }
     st = launch_decode(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, pl, ws, s, nullptr, dtype);
     if (ws) {
@@ -823,9 +954,9 @@ fa_status_t fa_fwd_fp8(const void* q, const void* k, const void* v, float descal
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     void* ws = workspace;
     if (!ws) {
-        cudaError_t e = cudaMallocAsync(&ws, need, s);
+        cudaError_t e = scratch_alloc(&ws, need, s);
         if (e != cudaSuccess)
-            return cuda_fail(e, "cudaMallocAsync (V^T workspace)");
+            return cuda_fail(e, "scratch allocation (V^T workspace)");
     }
     st = causal ? launch_fwd_fp8<true>(q, k, v, ws, o, lse, B, Hq, Hkv, Nq, Nk, scale_log2, descale_v, s)
                 : launch_fwd_fp8<false>(q, k, v, ws, o, lse, B, Hq, Hkv, Nq, Nk, scale_log2, descale_v, s);
@@ -877,9 +1008,9 @@ fa_status_t fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o,
     bool owned = false;
     if (pl.total() > 0) {
         if (ws == nullptr) {
-            cudaError_t e = cudaMallocAsync(&ws, pl.total(), s);
+            cudaError_t e = scratch_alloc(&ws, pl.total(), s);
             if (e != cudaSuccess)
-                return cuda_fail(e, "cudaMallocAsync (split-KV partials)");
+                return cuda_fail(e, "scratch allocation (split-KV partials)");
             owned = true;
         } else if (workspace_bytes < pl.total()) {
             set_error("workspace has %zu bytes, %zu needed", workspace_bytes, pl.total());
@@ -997,9 +1128,9 @@ static fa_status_t paged_entry(int dtype, const void* q, const void* k_cache, co
     bool owned = false;
     if (pl.total() > 0) {
         if (ws == nullptr) {
-            cudaError_t e = cudaMallocAsync(&ws, pl.total(), s);
+            cudaError_t e = scratch_alloc(&ws, pl.total(), s);
             if (e != cudaSuccess)
-                return cuda_fail(e, "cudaMallocAsync (paged split-KV partials)");
+                return cuda_fail(e, "scratch allocation (paged split-KV partials)");
             owned = true;
         } else if (workspace_bytes < pl.total()) {
             set_error("workspace has %zu bytes, %zu needed", workspace_bytes, pl.total());
@@ -1045,6 +1176,16 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d)
     return bwd_plan(B, Hq, Hkv, Nq, Nk, d).total_split;
 }
 
+int fa_fwd_kv_split(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || Hq % Hkv != 0 || d < 1 || d > 256 || d % 32 != 0 ||
+        (causal != 0 && causal != 1))
+        return 0;
+    if (decode_shape(Hq, Hkv, Nq, d))
+        return 1;
+    return fwd_kv_split(B, Hq, Nq, Nk, d, causal, sm_count());
+}
+
 int fa_bwd_query_split(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal)
 {
     if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || Hq % Hkv != 0 || d < 1 || d > 256 ||
@@ -1085,9 +1226,9 @@ static fa_status_t bwd_entry(int dtype, const void* q, const void* k, const void
     void* ws = workspace;
     bool owned = false;
     if (!ws) {
-        cudaError_t e = cudaMallocAsync(&ws, q_split > 1 ? pl.total_split : pl.total, s);
+        cudaError_t e = scratch_alloc(&ws, q_split > 1 ? pl.total_split : pl.total, s);
         if (e != cudaSuccess)
-            return cuda_fail(e, "cudaMallocAsync (backward workspace)");
+            return cuda_fail(e, "scratch allocation (backward workspace)");
         owned = true;
     }
     fa::BwdParams p;

@@ -20,6 +20,12 @@ struct FwdParams {
     unsigned* tile_ctr; // [4]: tiles claimed beyond each block's first, blocks done claiming,
                         // owner tag (zero when free; the last block resets all three), padding
     unsigned tile_tag;  // this launch's owner tag (nonzero)
+    // key split (fwd_kernel<..., SPLIT = true>): each (query tile pair, head) is kv_split work
+    // tiles, share s taking the pair's key blocks [s * n / kv_split, (s + 1) * n / kv_split)
+    // of its n; the shares' partial results are merged by fwd_combine_kernel
+    int kv_split;
+    float* part_o;      // [B * Hq, kv_split, Nq, d_io] fp32: O_s = U_s / l_s of share s
+    float* part_lse;    // [B * Hq, kv_split, Nq] fp32: m_s + log2(l_s), -inf where share s sees no key
 };
 
 struct DecodeParams {

@@ -39,6 +39,12 @@
 // in the order the MMAs free them, and a softmax that rescales O first waits for
 // the previous block's P.V (S(j) no longer follows it).
 //
+// Key split (SPLIT): where the launch has fewer work tiles than SMs, each tile's
+// key blocks are cut into kv_split contiguous shares that run as tiles of their
+// own; a share ends with O_s = U_s / l_s in fp32 and lse_s = m_s + log2(l_s), and
+// fwd_combine_kernel merges the shares by their lse (the same rescale-and-add as
+// between blocks).
+//
 // Scores are kept in the log2 domain: x = s * scale * log2(e), p = 2^(x - m).
 // Rescaling is lazy: the reference max m moves (and U, l are multiplied by
 // 2^(m_old - m_new)) only when the block max exceeds it by more than
@@ -122,25 +128,39 @@ struct FwdTile {
     int bh;        // batch * Hq + head
     int kvh;       // batch * Hkv + kv head
     int q0;        // first query row
-    int nb0, nb1;  // 128-key blocks seen by query tile 0 / 1
+    int nb0, nb1;  // 128-key blocks seen by query tile 0 / 1 (in this tile's key share)
     int n_iter;    // max of the two
+    int kb0;       // first key block of the share (0 without a key split)
+    int share;     // key share (0 without a key split)
 };
 
 // The launch has at most one block per SM.  Block c starts with tile c; each
 // further tile is the next unclaimed one (the launch's tile counter), so like a
 // hardware block scheduler the blocks take the heavy causal tiles first and
-// whichever block is free takes the next.
-template <int kTiles, bool CAUSAL>
+// whichever block is free takes the next.  With a key split (SPLIT) tile i is
+// share (i / (B*Hq)) % kv_split of its pair's key blocks.
+template <int kTiles, bool CAUSAL, bool SPLIT = false>
 __device__ __forceinline__ void fwd_tile(const FwdParams& p, int i, FwdTile& w)
 {
     const int n_bh = p.B * p.Hq;
-    const int pair = p.n_pairs - 1 - i / n_bh;
+    const int ns = SPLIT ? p.kv_split : 1;
+    const int pair = p.n_pairs - 1 - i / (n_bh * ns);
     w.bh = i % n_bh;
+    w.share = SPLIT ? (i / n_bh) % ns : 0;
     const int b = w.bh / p.Hq, h = w.bh % p.Hq;
     w.kvh = b * p.Hkv + h / p.G;
     w.q0 = pair * 128 * kTiles;
     w.nb0 = fwd_blocks_for_tile(w.q0, p.Nq, p.Nk, CAUSAL);
     w.nb1 = (kTiles == 2) ? fwd_blocks_for_tile(w.q0 + 128, p.Nq, p.Nk, CAUSAL) : 0;
+    w.kb0 = 0;
+    if constexpr (SPLIT) {
+        // blocks [lo, hi) of the pair's n; a tile sees the part of them below its own count
+        const int n = max(w.nb0, w.nb1);
+        const int lo = (int)(((long long)w.share * n) / ns), hi = (int)(((long long)(w.share + 1) * n) / ns);
+        w.kb0 = lo;
+        w.nb0 = max(0, min(hi, w.nb0) - lo);
+        w.nb1 = max(0, min(hi, w.nb1) - lo);
+    }
     w.n_iter = max(w.nb0, w.nb1);
 }
 
@@ -159,7 +179,9 @@ __device__ __forceinline__ int fwd_take_tile(uint64_t* bar_tfull, uint64_t* bar_
     return tile;
 }
 
-template <int D, bool CAUSAL, typename T = __nv_bfloat16, bool F8 = false>
+// SPLIT: key split (kv_split shares per pair, partial results to part_o / part_lse);
+// without it the kernel carries none of the split's code
+template <int D, bool CAUSAL, typename T = __nv_bfloat16, bool F8 = false, bool SPLIT = false>
 __global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, FwdParams p)
@@ -189,7 +211,7 @@ __global__ void __launch_bounds__(384, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* tile_ring = abort_flag + 1;          // [2]  tile indices (>= n_tiles: no more)
     static_assert((17 + 2 * C::kStages) * 8 + 16 <= C::kBarBytes, "barrier area too small");
-    const int n_tiles = p.n_pairs * p.B * p.Hq;
+    const int n_tiles = p.n_pairs * p.B * p.Hq * (SPLIT ? p.kv_split : 1);
 
     const int warp = warp_id(), lane = lane_id();
     const int delta = p.Nk - p.Nq;
@@ -254,7 +276,7 @@ __global__ void __launch_bounds__(384, 1)
                 mbar_arrive(&bar_tfull[u & 1]);
                 if (tile >= n_tiles)
                     break;
-                fwd_tile<C::kTiles, CAUSAL>(p, tile, w);
+                fwd_tile<C::kTiles, CAUSAL, SPLIT>(p, tile, w);
                 for (int t = 0; t < 2 && ok; ++t) {
                     if ((t ? w.nb1 : w.nb0) == 0)
                         continue;
@@ -284,7 +306,7 @@ __global__ void __launch_bounds__(384, 1)
                         mbar_arrive_expect_tx(&bar_full[kv], C::kTileBytes);
                         for (int pn = 0; pn < C::kPanels; ++pn)
                             tma_load_3d(dst + pn * C::kPanelBytes, kv ? &tmV : &tmK, &bar_full[kv],
-                                        pn * C::kPanelElems, j * 128, w.kvh);
+                                        pn * C::kPanelElems, (w.kb0 + j) * 128, w.kvh);
                         ++cnt;
                         return true;
                     };
@@ -307,11 +329,11 @@ __global__ void __launch_bounds__(384, 1)
                         uint8_t* dst = sKV + slot * C::kTileBytes;
                         mbar_arrive_expect_tx(&bar_full[slot], C::kTileBytes);
                         if (F8 && kv)   // V^T: d rows of keys j*128 .. j*128+127
-                            tma_load_3d(dst, &tmV, &bar_full[slot], j * 128, 0, w.kvh);
+                            tma_load_3d(dst, &tmV, &bar_full[slot], (w.kb0 + j) * 128, 0, w.kvh);
                         else
                             for (int pn = 0; pn < C::kPanels; ++pn)
                                 tma_load_3d(dst + pn * C::kPanelBytes, kv ? &tmV : &tmK, &bar_full[slot],
-                                            pn * C::kPanelElems, j * 128, w.kvh);
+                                            pn * C::kPanelElems, (w.kb0 + j) * 128, w.kvh);
                         ++kvi;
                     }
                 }
@@ -419,7 +441,7 @@ __global__ void __launch_bounds__(384, 1)
                 const int tile = fwd_take_tile(bar_tfull, bar_tfree, tile_ring, u, lane, abort_flag, ok);
                 if (!ok || tile >= n_tiles)
                     break;
-                fwd_tile<C::kTiles, CAUSAL>(p, tile, w);
+                fwd_tile<C::kTiles, CAUSAL, SPLIT>(p, tile, w);
                 for (int t = 0; t < 2 && ok; ++t) {
                     if ((t ? w.nb1 : w.nb0) == 0)
                         continue;
@@ -565,7 +587,7 @@ __global__ void __launch_bounds__(384, 1)
             const int tile = fwd_take_tile(bar_tfull, bar_tfree, tile_ring, u, lane, abort_flag, ok);
             if (!ok || tile >= n_tiles)
                 break;
-            fwd_tile<C::kTiles, CAUSAL>(p, tile, w);
+            fwd_tile<C::kTiles, CAUSAL, SPLIT>(p, tile, w);
             const int qi = w.q0 + 128 * t + r;
             const int nb = t ? w.nb1 : w.nb0;
             const int qlim = qi + delta;
@@ -588,7 +610,7 @@ __global__ void __launch_bounds__(384, 1)
                 for (int c = 0; c < 128; ++c)
                     s[c] = __uint_as_float(sr[c]);
 
-                const int kb = j * 128;
+                const int kb = (w.kb0 + j) * 128;
                 const bool need_mask = (kb + 128 > p.Nk) || (CAUSAL && kb + 127 > qlim);
                 if (need_mask) {
                     const int lim = CAUSAL ? min(p.Nk - 1, qlim) : p.Nk - 1;
@@ -720,6 +742,18 @@ __global__ void __launch_bounds__(384, 1)
                 for (int c0 = 0; c0 < p.d_io; c0 += 32) {
                     uint32_t o[32];
                     tmem_ld32(tO + (uint32_t)c0, o);
+                    if constexpr (SPLIT) {
+                        // this share's normalised partial O_s in fp32
+                        if (row_valid) {
+                            const size_t prow = ((size_t)w.bh * p.kv_split + w.share) * p.Nq + qi;
+                            float4* dst = reinterpret_cast<float4*>(p.part_o + prow * p.d_io + c0);
+#pragma unroll
+                            for (int c = 0; c < 8; ++c)
+                                dst[c] = make_float4(__uint_as_float(o[4 * c]) * inv_l, __uint_as_float(o[4 * c + 1]) * inv_l,
+                                                     __uint_as_float(o[4 * c + 2]) * inv_l, __uint_as_float(o[4 * c + 3]) * inv_l);
+                        }
+                        continue;
+                    }
                     if (row_valid) {
                         uint32_t wv[16];
 #pragma unroll
@@ -735,8 +769,16 @@ __global__ void __launch_bounds__(384, 1)
                 // O(t) is read out: the next tile's first P.V may overwrite it once this
                 // warpgroup's P of that tile is signalled (after the fence in the P write)
                 tc_fence_before();
-                if (row_valid && p.lse)
+                if constexpr (SPLIT) {
+                    if (row_valid)
+                        p.part_lse[((size_t)w.bh * p.kv_split + w.share) * p.Nq + qi] =
+                            (l > 0.f) ? m_ref + __log2f(l) : -INFINITY;
+                } else if (row_valid && p.lse) {
                     p.lse[row] = (l > 0.f) ? (m_ref + __log2f(l)) * kLn2 : -INFINITY;
+                }
+            } else if (SPLIT && row_valid) {
+                // no key of this share for any row of the tile: its partial carries no weight
+                p.part_lse[((size_t)w.bh * p.kv_split + w.share) * p.Nq + qi] = -INFINITY;
             } else if (row_valid) {
                 // no visible key for any row of this tile
                 uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(p.o) + row * p.d_io);
@@ -758,6 +800,59 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }
+}
+
+// Merge of the key shares of a split forward (one warp per query row): with
+// w_s = 2^(lse_s - M), M = max_s lse_s, O = sum_s w_s O_s / sum_s w_s and
+// LSE = (M + log2 sum_s w_s) ln 2 -- the rescale-and-add of the online softmax
+// (page "FlashAttention：为什么少搬数据，反而算得更快", §04) applied to whole
+// shares.  Shares with lse_s = -inf (no key) are skipped; a row no share sees
+// gets O = 0 and LSE = -inf.
+template <typename T = __nv_bfloat16>
+__global__ void __launch_bounds__(128) fwd_combine_kernel(FwdParams p)
+{
+    const long long row = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= (long long)p.B * p.Hq * p.Nq)
+        return;
+    const long long bh = row / p.Nq, i = row % p.Nq;
+    const int ns = p.kv_split;
+    const float* lse_s = p.part_lse + (size_t)bh * ns * p.Nq + i;
+    float M = -INFINITY;
+    for (int s = lane; s < ns; s += 32)
+        M = fmaxf(M, lse_s[(size_t)s * p.Nq]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    constexpr int kMaxPerLane = 8;   // d_io <= 256
+    float acc[kMaxPerLane];
+#pragma unroll
+    for (int k = 0; k < kMaxPerLane; ++k)
+        acc[k] = 0.f;
+    float L = 0.f;
+    const int per_lane = p.d_io / 32;
+    if (M != -INFINITY) {
+        for (int s = 0; s < ns; ++s) {
+            const float ls = lse_s[(size_t)s * p.Nq];
+            if (ls == -INFINITY)
+                continue;
+            const float wgt = ex2_approx(ls - M);
+            L += wgt;
+            const float* os = p.part_o + (((size_t)bh * ns + s) * p.Nq + i) * p.d_io + lane;
+#pragma unroll
+            for (int k = 0; k < kMaxPerLane; ++k)
+                if (k < per_lane)
+                    acc[k] = fmaf(wgt, os[32 * k], acc[k]);
+        }
+    }
+    const float inv = (L > 0.f) ? 1.f / L : 0.f;
+    T* o = static_cast<T*>(p.o) + (size_t)row * p.d_io + lane;
+#pragma unroll
+    for (int k = 0; k < kMaxPerLane; ++k)
+        if (k < per_lane)
+            o[32 * k] = Elt<T>::from_float(acc[k] * inv);
+    if (lane == 0 && p.lse)
+        p.lse[row] = (L > 0.f) ? (M + __log2f(L)) * kLn2 : -INFINITY;
 }
 
 }  // namespace fa

@@ -36,6 +36,13 @@
  *    enqueued on it; no call synchronises the stream or the device.
  *  - Ownership: the caller owns every buffer; the library keeps no pointer
  *    after a call returns and frees nothing it did not allocate.
+ *  - Scratch: a call that allocates its own scratch (workspace NULL, or the
+ *    split-KV / key-split partials of fa_fwd) takes it stream-ordered from a
+ *    memory pool of the library (one per device and context) and frees it
+ *    stream-ordered on the same stream.  The pool keeps up to 1 GiB of freed
+ *    memory for later calls (the device's default pool returns its memory at
+ *    every synchronisation, and mapping it again cost about 0.2 ms per call);
+ *    during stream capture the allocation uses cudaMallocAsync instead.
  *  - Errors: arguments are checked before anything is enqueued; a bad argument
  *    returns FA_ERR_INVALID_ARGUMENT or FA_ERR_UNSUPPORTED with nothing launched.
  *    A CUDA launch or allocation failure returns FA_ERR_CUDA;
@@ -90,9 +97,14 @@ const char* fa_last_error_message(void);
  *   scale multiplies q.k (usually 1/sqrt(d)); it must be finite and > 0.
  * Shapes with few query rows per kv head (Nq * Hq / Hkv <= 16, the decode shape
  * of §09) run the split-KV kernels; their partial results need scratch, which
- * this call allocates stream-ordered with cudaMallocAsync and frees with
- * cudaFreeAsync on `stream`.  Use fa_fwd_splitkv() to pass the scratch instead.
- * Other shapes run one persistent block per SM.  The blocks share a tile
+ * this call allocates and frees stream-ordered on `stream` (see Scratch
+ * above).  Use fa_fwd_splitkv() to pass the scratch instead.
+ * Other shapes run one persistent block per SM.  Where they have fewer work
+ * tiles (pairs of 128-row query tiles of one head) than the GPU has SMs, each
+ * tile's key blocks are cut into fa_fwd_kv_split(...) contiguous shares that
+ * run as separate tiles; their partial results (fp32 O and LSE per share, in
+ * scratch this call allocates and frees stream-ordered on `stream`) are merged
+ * by a second kernel as the online softmax merges blocks (§04).  The blocks share a tile
  * counter, one of 256 slots in the library's device memory that launches take
  * in turn; the launch's last block resets it.  So at most 256 tiled forward
  * launches (this call, fa_fwd_ex, fa_fwd_fp8) may be in flight on one device
@@ -257,6 +269,14 @@ fa_status_t fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, 
  *   each accumulate their half of dk, dv and dq.
  */
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d);
+
+/*
+ * Key shares per work tile that fa_fwd / fa_fwd_ex use on the current device
+ * (1: no key split, also for the decode shapes, which run the split-KV decode
+ * kernels; 2 to 16 where the work tiles are fewer than the SMs and the split
+ * is estimated to save at least 10%).  0 for sizes fa_fwd would refuse.
+ */
+int fa_fwd_kv_split(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal);
 
 /*
  * The number of CTAs that fa_bwd / fa_bwd_ex share each (key block, kv head)

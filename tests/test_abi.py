@@ -272,3 +272,28 @@ def test_backward_query_split_rule():
     assert qs(1, 3, 2, 64, 64, 64, 0) == 0            # Hq not a multiple of Hkv
     assert qs(1, 2, 1, 64, 64, 288, 0) == 0
     assert fa.lib().fa_bwd_query_split(1, 2, 1, 64, 64, 64, 2) == 0   # causal flag not 0 / 1
+
+
+def test_forward_key_split_rule():
+    """The key shares fa_fwd takes on a 148-SM device: none where the work tiles
+    fill the SMs (the step workloads) or for the decode shapes (split-KV decode
+    kernels), up to 16 where a few long tiles would leave most SMs idle (a short
+    chunk appended to a long context); 0 for sizes fa_fwd refuses."""
+    if _sm_count() != 148:
+        pytest.skip("the expected shares are for 148 SMs")
+    ks = fa.fa_fwd_kv_split
+    assert ks(1, 32, 8, 8192, 8192, 128, 1) == 1      # gqa_8k: 1024 work tiles
+    assert ks(2, 32, 32, 4096, 4096, 128, 1) == 1     # mha_4k_long
+    assert ks(4, 16, 16, 1024, 1024, 64, 0) == 1      # mha_1k: 256 work tiles
+    assert ks(1, 32, 8, 8192, 8192, 256, 1) == 1
+    assert ks(64, 32, 8, 1, 8192, 128, 0) == 1        # decode shape
+    assert ks(1, 32, 8, 512, 32768, 128, 1) == 2      # 64 work tiles of 254-256 key blocks
+    assert ks(1, 32, 8, 64, 32768, 128, 1) == 4       # 32 work tiles: four shares fill one round
+    assert ks(1, 4, 1, 2048, 2048, 128, 1) == 4
+    assert ks(1, 4, 1, 2048, 2048, 128, 0) == 4
+    assert ks(1, 2, 1, 300, 5000, 64, 1) == 16
+    assert ks(1, 2, 1, 1000, 2000, 256, 0) == 8
+    assert ks(1, 4, 1, 1000, 1000, 128, 1) == 1       # 16 tiles of at most 8 blocks: too little to gain
+    assert ks(1, 3, 2, 64, 64, 64, 0) == 0            # Hq not a multiple of Hkv
+    assert ks(1, 2, 1, 64, 64, 80, 0) == 0            # head size not a multiple of 32
+    assert fa.lib().fa_fwd_kv_split(1, 2, 1, 64, 64, 64, 2) == 0

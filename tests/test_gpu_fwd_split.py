@@ -1,0 +1,101 @@
+"""GPU parity of the forward's key split against the oracle.  Where a tiled
+forward has fewer work tiles (pairs of 128-row query tiles of one head) than the
+GPU has SMs, each tile's key blocks are cut into contiguous shares that run as
+separate tiles, and a second kernel merges their fp32 partials by their LSE.
+Each case checks O and LSE (every row, or sampled rows at the long append
+shapes) and that O repeats bitwise from call to call."""
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_114_b200 as fa
+import oracle
+import synth
+from tests import gpu_parity as G
+
+pytestmark = pytest.mark.gpu
+
+# B, Hq, Hkv, Nq, Nk, d, causal, the key shares a 148-SM device takes
+FWD_SPLIT_SHAPES = [
+    (1, 4, 1, 2048, 2048, 128, True, 4),
+    (1, 4, 1, 2048, 2048, 128, False, 4),
+    (1, 8, 2, 1000, 3000, 128, True, 4),     # bottom-right mask, Nq < Nk
+    (1, 2, 1, 3000, 2000, 128, True, 6),     # Nq > Nk: the first rows see no key
+    (2, 2, 1, 600, 4000, 128, True, 12),
+    (1, 2, 1, 1000, 2000, 256, False, 8),    # one query tile per work tile
+    (1, 2, 1, 1024, 8192, 256, True, 8),
+    (1, 2, 1, 300, 5000, 64, True, 16),
+    (1, 4, 1, 200, 4096, 128, False, 16),
+]
+
+
+def _sms():
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
+def _forward_twice(w, xd):
+    o1, l1 = fa.fa_fwd(xd["q"], xd["k"], xd["v"], causal=w.causal, scale=w.scale)
+    o2, l2 = fa.fa_fwd(xd["q"], xd["k"], xd["v"], causal=w.causal, scale=w.scale)
+    torch.cuda.synchronize()
+    fa.fa_check_device_status()
+    return o1, l1, o2, l2
+
+
+@pytest.mark.parametrize("shape", FWD_SPLIT_SHAPES, ids=[str(s) for s in FWD_SPLIT_SHAPES])
+def test_fwd_split_full(shape):
+    B, Hq, Hkv, Nq, Nk, d, causal, shares = shape
+    got = fa.fa_fwd_kv_split(B, Hq, Hkv, Nq, Nk, d, causal)
+    if _sms() == 148:
+        assert got == shares
+    w = synth.Workload("fwd_split", B, Hq, Hkv, Nq, Nk, d, causal, 9800 + FWD_SPLIT_SHAPES.index(shape))
+    x = synth.make_inputs(w, dout=False)
+    xd = {k: v.cuda() for k, v in x.items()}
+    o, lse, o2, l2 = _forward_twice(w, xd)
+    o_ref, lse_ref = oracle.fwd(x["q"], x["k"], x["v"], w.scale, w.causal)
+    G.assert_o(G.f64(o), o_ref, o_abs=G.o_abs_ref(x["q"], x["k"], x["v"], w.scale, w.causal))
+    G.assert_lse(G.f64(lse), lse_ref)
+    assert torch.equal(o, o2) and torch.equal(lse, l2), "O / LSE not repeatable"
+
+
+def test_fwd_split_fp16_with_backward():
+    """fp16 inputs through the split forward, and the backward on its O / LSE."""
+    w = synth.Workload("fwd_split16", 1, 4, 1, 2048, 2048, 128, True, 9900)
+    x = synth.make_inputs(w, dtype=torch.float16)
+    xd = {k: v.cuda() for k, v in x.items()}
+    o, lse, _, _ = _forward_twice(w, xd)
+    assert o.dtype == torch.float16
+    xr = {k: v.double() for k, v in x.items()}
+    o_ref, lse_ref = oracle.fwd(xr["q"], xr["k"], xr["v"], w.scale, w.causal)
+    G.assert_o(G.f64(o), o_ref, o_abs=G.o_abs_ref(xr["q"], xr["k"], xr["v"], w.scale, w.causal))
+    G.assert_lse(G.f64(lse), lse_ref)
+    dq, dk, dv = fa.fa_bwd(xd["q"], xd["k"], xd["v"], o, xd["dout"], lse, causal=w.causal, scale=w.scale)
+    torch.cuda.synchronize()
+    fa.fa_check_device_status()
+    rq, rk, rv = oracle.bwd(xr["q"], xr["k"], xr["v"], xr["dout"], w.scale, w.causal)
+    G.assert_grad(G.f64(dq), rq, "dQ")
+    G.assert_grad(G.f64(dk), rk, "dK")
+    G.assert_grad(G.f64(dv), rv, "dV")
+
+
+APPEND_SHAPES = [
+    # a 512-row chunk appended to a 32K context, and a 64-row one (GQA 32 / 8)
+    (1, 32, 8, 512, 32768, 128, True, 2),
+    (1, 32, 8, 64, 32768, 128, True, 4),
+]
+
+
+@pytest.mark.parametrize("shape", APPEND_SHAPES, ids=[str(s) for s in APPEND_SHAPES])
+def test_fwd_split_append_sampled(shape):
+    B, Hq, Hkv, Nq, Nk, d, causal, shares = shape
+    if _sms() == 148:
+        assert fa.fa_fwd_kv_split(B, Hq, Hkv, Nq, Nk, d, causal) == shares
+    w = synth.Workload("append", B, Hq, Hkv, Nq, Nk, d, causal, 9950 + APPEND_SHAPES.index(shape))
+    x = synth.make_inputs(w, dout=False)
+    xd = {k: v.cuda() for k, v in x.items()}
+    o, lse, o2, _ = _forward_twice(w, xd)
+    assert torch.equal(o, o2)
+    rows = G.sample_rows(w, n_random=24)
+    o_ref, lse_ref = oracle.fwd(x["q"], x["k"], x["v"], w.scale, w.causal, rows=rows)
+    G.assert_o(G.f64(o).reshape(-1, d)[rows], o_ref,
+               o_abs=G.o_abs_ref(x["q"], x["k"], x["v"], w.scale, w.causal, rows=rows))
+    G.assert_lse(G.f64(lse).reshape(-1)[rows], lse_ref)

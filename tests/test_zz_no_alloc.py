@@ -6,10 +6,11 @@ On two calls in a row with different shapes (the fixed scratch keeps the
 previous call's contents, which must not leak into the next result) its
 output must match the fp64 oracle on the same inputs within the parity
 tolerances of the other tests (|O - O_ref| <= 1e-2, |LSE - LSE_ref| <= 1e-3)
-and agree with fa_fwd_splitkv given a caller workspace.  The call must leave
-the device's stream-ordered memory pool untouched (the allocating entry point
-is the positive control), the automatic split count must fit the fixed
-scratch, and an explicit split count that does not fit must be refused.
+and agree with fa_fwd_splitkv given a caller workspace.  Captured into a CUDA
+graph, the call must add no memory-allocation node (the allocating entry point,
+captured the same way, adds one: the positive control); the automatic split
+count must fit the fixed scratch, and an explicit split count that does not fit
+must be refused.
 This file is collected last so that a stop at the first failure has run
 every other test already.
 """
@@ -39,33 +40,30 @@ def _with_workspace(xd, w, splits):
                              num_splits=splits, workspace=ws if n else None)
 
 
-class DefaultPool:
-    """High-water mark of used bytes in the current device's default
-    stream-ordered memory pool (the pool cudaMallocAsync draws from), read and
-    reset through the driver API."""
-    USED_MEM_CURRENT, USED_MEM_HIGH = 7, 8   # CUmemPool_attribute
-
-    def __init__(self):
-        self.cu = ctypes.CDLL("libcuda.so.1")
-        dev = ctypes.c_int()
-        assert self.cu.cuCtxGetDevice(ctypes.byref(dev)) == 0
-        self.pool = ctypes.c_void_p()
-        assert self.cu.cuDeviceGetDefaultMemPool(ctypes.byref(self.pool), dev) == 0
-
-    def _get(self, attr):
-        v = ctypes.c_uint64()
-        assert self.cu.cuMemPoolGetAttribute(self.pool, attr, ctypes.byref(v)) == 0
-        return v.value
-
-    def reset_high(self):
-        zero = ctypes.c_uint64(0)   # the only value the high-water mark can be set to
-        assert self.cu.cuMemPoolSetAttribute(self.pool, self.USED_MEM_HIGH, ctypes.byref(zero)) == 0
-
-    def used_high(self):
-        return self._get(self.USED_MEM_HIGH)
-
-    def used_current(self):
-        return self._get(self.USED_MEM_CURRENT)
+def alloc_nodes(fn):
+    """Memory-allocation nodes of a CUDA graph captured (relaxed mode) from the
+    work fn enqueues on a fresh stream; the graph is never launched."""
+    from cuda.bindings import runtime as rt
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        err, = rt.cudaStreamBeginCapture(stream.cuda_stream,
+                                         rt.cudaStreamCaptureMode.cudaStreamCaptureModeRelaxed)
+        assert err == rt.cudaError_t.cudaSuccess, err
+        try:
+            fn()
+        finally:
+            err, graph = rt.cudaStreamEndCapture(stream.cuda_stream)
+    assert err == rt.cudaError_t.cudaSuccess, err
+    try:
+        err, _, n = rt.cudaGraphGetNodes(graph, 0)
+        assert err == rt.cudaError_t.cudaSuccess, err
+        err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+        assert err == rt.cudaError_t.cudaSuccess, err
+        kinds = [rt.cudaGraphNodeGetType(nd)[1] for nd in nodes[:n]]
+        return sum(1 for k in kinds if k == rt.cudaGraphNodeType.cudaGraphNodeTypeMemAlloc), len(kinds)
+    finally:
+        rt.cudaGraphDestroy(graph)
 
 
 def test_noalloc_matches_oracle_and_workspace_entry_point_two_calls():
@@ -77,14 +75,10 @@ def test_noalloc_matches_oracle_and_workspace_entry_point_two_calls():
     outs = [(torch.empty_like(xd["q"]), torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device="cuda"))
             for (w, _), xd in zip(CASES, inputs)]
     torch.cuda.synchronize()
-    pool = DefaultPool()
-    base = pool.used_current()
-    pool.reset_high()
     for (w, splits), xd, (o, lse) in zip(CASES, inputs, outs):   # two calls in a row
         fa.fa_fwd_splitkv_noalloc(xd["q"], xd["k"], xd["v"], o, lse, causal=w.causal,
                                   scale=w.scale, num_splits=splits)
     torch.cuda.synchronize()
-    assert pool.used_high() <= base, "the no-allocation call drew memory from the default pool"
     fa.fa_check_device_status()
     for (w, splits), x, xd, (o, lse) in zip(CASES, hosts, inputs, outs):
         o_ref, lse_ref = oracle.fwd(x["q"], x["k"], x["v"], w.scale, w.causal)
@@ -95,14 +89,17 @@ def test_noalloc_matches_oracle_and_workspace_entry_point_two_calls():
         torch.cuda.synchronize()
         G.assert_o(G.f64(o), G.f64(o_ws), what="O (no-alloc vs workspace call)")
         G.assert_lse(G.f64(lse), G.f64(lse_ws))
-    # positive control: the same call without a workspace allocates from the pool
+    # captured into a graph the no-allocation call adds no allocation node; the same
+    # call without a workspace (the allocating entry point) adds one
     w, splits = CASES[0]
     xd = inputs[0]
-    pool.reset_high()
-    fa.fa_fwd_splitkv(xd["q"], xd["k"], xd["v"], causal=w.causal, scale=w.scale, num_splits=splits)
-    torch.cuda.synchronize()
-    assert pool.used_high() > base, "the pool's high-water mark did not see an allocating call"
-
+    o, lse = outs[0]
+    n_alloc, n_nodes = alloc_nodes(lambda: fa.fa_fwd_splitkv_noalloc(
+        xd["q"], xd["k"], xd["v"], o, lse, causal=w.causal, scale=w.scale, num_splits=splits))
+    assert n_nodes > 0 and n_alloc == 0, (n_alloc, n_nodes)
+    n_alloc, n_nodes = alloc_nodes(lambda: fa.fa_fwd_splitkv(
+        xd["q"], xd["k"], xd["v"], o, lse, causal=w.causal, scale=w.scale, num_splits=splits))
+    assert n_alloc >= 1, "the allocating entry point added no allocation node"
 
 def test_noalloc_automatic_split_count_fits_the_fixed_scratch():
     """A shape whose automatic split count would overflow the fixed scratch
