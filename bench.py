@@ -275,11 +275,11 @@ def run_reference(args, rank, world):
 # ----------------------------------------------------------------------------
 # GPU arm
 # ----------------------------------------------------------------------------
-# DRAM bytes (read + write) of one bwd_main launch on this workload, from a one-pass
-# ncu capture of this bench command on the current kernel (dram__bytes_read.sum +
-# dram__bytes_write.sum, the first timed-step launch); to be taken again whenever the
-# kernel changes.
-BWD_MAIN_DRAM_BYTES = 699.24e6 + 321.14e6
+# DRAM bytes (read + write) of one bwd_main launch on this workload, from the ncu
+# launch list of this bench command on the current kernel (dram__bytes_read.sum +
+# dram__bytes_write.sum, mean of the six warm-up and timed-step launches); to be
+# taken again whenever the kernel changes.
+BWD_MAIN_DRAM_BYTES = 706.00e6 + 319.01e6
 
 
 def run_libfa(args, rank, world, local):
@@ -494,9 +494,13 @@ def run_libfa(args, rank, world, local):
     other = {}
     # the step workload's shape at head size 256 (the feature-split backward), and
     # without the causal mask (the backward shares each unit between two CTAs there)
+    # without the causal mask (the backward shares each unit between two CTAs there), and a
+    # 512-row chunk appended to a 32K-key context (the forward cuts each work tile's keys into shares)
     extra = {"gqa_8k_d256": synth.WORKLOADS[STEP_WORKLOAD].with_(name="gqa_8k_d256", d=256),
-             "gqa_8k_noncausal": synth.WORKLOADS[STEP_WORKLOAD].with_(name="gqa_8k_noncausal", causal=False)}
-    for name in ("mha_4k_long", "mha_1k", "mha_1k_noncausal", "gqa_8k_d256", "gqa_8k_noncausal"):
+             "gqa_8k_noncausal": synth.WORKLOADS[STEP_WORKLOAD].with_(name="gqa_8k_noncausal", causal=False),
+             "append_512_32k": synth.WORKLOADS[STEP_WORKLOAD].with_(name="append_512_32k", Nq=512, Nk=32768)}
+    for name in ("mha_4k_long", "mha_1k", "mha_1k_noncausal", "gqa_8k_d256", "gqa_8k_noncausal",
+                 "append_512_32k"):
         base = extra.get(name) or synth.WORKLOADS[name]
         wo = base.with_(seed=rank_seed(base.seed, rank))
         xo = {k_: v_.to(dev) for k_, v_ in synth.make_inputs(wo).items()}
@@ -519,12 +523,24 @@ def run_libfa(args, rank, world, local):
         torch.cuda.synchronize()
         f_ms = statistics.median(timed(fo, max(10, args.steps)))
         b_ms = statistics.median(timed(bo, max(10, args.steps)))
-        other[name] = {"workload": f"B={wo.B}, Hq={wo.Hq}, Hkv={wo.Hkv}, N={wo.Nq}, d={wo.d}, "
+        if wo.Nq == wo.Nk:
+            shape, f_fl, b_fl, rule = f"N={wo.Nq}", wo.fwd_flops(), wo.bwd_flops(), "FLOP rule"
+        else:
+            # bottom-right mask with Nq << Nk: almost every (query, key) pair is visible, so
+            # the rule's causal half would understate the work; count the visible pairs
+            vis = sum(min(max(i + wo.Nk - wo.Nq + 1, 0), wo.Nk) for i in range(wo.Nq)) if wo.causal \
+                else wo.Nq * wo.Nk
+            shape = f"Nq={wo.Nq}, Nk={wo.Nk}"
+            f_fl = 4.0 * wo.B * wo.Hq * vis * wo.d
+            b_fl, rule = 2.5 * f_fl, "4 d per visible (query, key) pair and head, x2.5 for the backward"
+        other[name] = {"workload": f"B={wo.B}, Hq={wo.Hq}, Hkv={wo.Hkv}, {shape}, d={wo.d}, "
                                    f"{'causal' if wo.causal else 'non-causal'}",
+                       "fwd_kv_split": fa.fa_fwd_kv_split(wo.B, wo.Hq, wo.Hkv, wo.Nq, wo.Nk, wo.d, wo.causal),
                        "bwd_query_split": fa.fa_bwd_query_split(wo.B, wo.Hq, wo.Hkv, wo.Nq, wo.Nk, wo.d,
                                                                 wo.causal),
-                       "fwd_ms": f_ms, "fwd_tflops": wo.fwd_flops() / (f_ms * 1e-3) / 1e12,
-                       "bwd_ms": b_ms, "bwd_tflops": wo.bwd_flops() / (b_ms * 1e-3) / 1e12}
+                       "flops": rule,
+                       "fwd_ms": f_ms, "fwd_tflops": f_fl / (f_ms * 1e-3) / 1e12,
+                       "bwd_ms": b_ms, "bwd_tflops": b_fl / (b_ms * 1e-3) / 1e12}
         del xo, oo, lo, go, wso
     fa.fa_check_device_status()
 
