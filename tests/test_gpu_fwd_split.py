@@ -26,6 +26,9 @@ FWD_SPLIT_SHAPES = [
     (1, 2, 1, 1024, 8192, 256, True, 8),
     (1, 2, 1, 300, 5000, 64, True, 16),
     (1, 4, 1, 200, 4096, 128, False, 16),
+    # decode shapes at d = 256 (beyond the split-KV decode kernels' 128) take the tiled path
+    (1, 8, 2, 1, 8192, 256, True, 16),
+    (2, 16, 4, 4, 16384, 256, True, 4),
 ]
 
 
