@@ -234,57 +234,79 @@ int sm_count()
 int kernel_d(int d) { return d <= 64 ? 64 : d <= 128 ? 128 : 256; }
 
 // The forward is persistent: one block per SM (its shared memory allows no
-// second), together working through the n_pairs * B * Hq (* kv_split) tiles.
+// second), together working through the n_pairs * n_bh (* kv_split) tiles.
 unsigned fwd_grid(const fa::FwdParams& p)
 {
-    const long long tiles = (long long)p.n_pairs * p.B * p.Hq * p.kv_split;
+    const long long tiles = (long long)p.n_pairs * p.n_bh * p.kv_split;
     return (unsigned)std::max<long long>(1, std::min<long long>(tiles, sm_count()));
 }
 
 // stream-ordered scratch from the library's memory pool (defined below)
 cudaError_t scratch_alloc(void** out, size_t bytes, cudaStream_t s);
 
-// 128-key blocks seen by the 128-row query tile starting at row qt (as the kernel's
-// fwd_blocks_for_tile)
-int host_blocks_for_tile(int qt, int Nq, int Nk, int causal)
+// Tile heads of the tiled forward.  A query head with fewer rows than a work tile
+// (Nq < 128 * tiles per CTA) would leave most of its tiles' rows idle and read its kv
+// head's K/V once per query head; so where a kv head serves several query heads (G > 1)
+// their G * Nq rows, consecutive in q / o / lse, share the kv head's tiles ("group rows").
+struct FwdGeom {
+    int group_rows, n_bh, rows, n_pairs;
+};
+
+FwdGeom fwd_geom(int B, int Hq, int Hkv, int Nq, int d)
+{
+    const int kt = kernel_d(d) == 256 ? 1 : 2;
+    const int G = Hq / Hkv;
+    FwdGeom g;
+    g.group_rows = (G > 1 && Nq < 128 * kt) ? 1 : 0;
+    g.n_bh = g.group_rows ? B * Hkv : B * Hq;
+    g.rows = g.group_rows ? G * Nq : Nq;
+    g.n_pairs = (g.rows + 128 * kt - 1) / (128 * kt);
+    return g;
+}
+
+// 128-key blocks seen by the 128-row query tile at row qt of a tile head with `rows`
+// rows, row r at query position r % Nq (as the kernel's fwd_blocks_for_tile)
+int host_blocks_for_tile(int qt, int rows, int Nq, int Nk, int causal)
 {
     const int nkb = (Nk + 127) / 128;
-    if (qt >= Nq)
+    if (qt >= rows)
         return 0;
     if (!causal)
         return nkb;
-    const long long last_key = (long long)std::min(qt + 127, Nq - 1) + (Nk - Nq);
+    const int last_row = std::min(qt + 127, rows - 1);
+    const int last_pos = (qt / Nq == last_row / Nq) ? last_row % Nq : Nq - 1;
+    const long long last_key = (long long)last_pos + (Nk - Nq);
     return last_key < 0 ? 0 : (int)std::min<long long>(nkb, last_key / 128 + 1);
 }
 
-// Key shares per (query tile pair, head) of the tiled forward.  Unsplit, the launch has
-// n_pairs * B * Hq work tiles, each costing its key blocks plus about 2 block times of
-// fixed work (Q load, first S, epilogue).  With fewer tiles than SMs the longest tile
-// bounds the launch, so each is cut into s contiguous shares of its key blocks (at least
-// 2 blocks each), all of them in one round (tiles * s <= SMs), and a second kernel merges
-// them (with the extra launch, about 8 block times more, as measured on small launches).
-// The estimate is max(total / SMs, longest / s + fixed) (+ 8 with a split); the cheapest
-// split that saves 10% on no split is taken, with the fp32 partials held under 256 MB.
-int fwd_kv_split(int B, int Hq, int Nq, int Nk, int d, int causal, int sms)
+// Key shares per work tile (query tile pair of a tile head) of the tiled forward.
+// Unsplit, the launch has n_pairs * n_bh work tiles, each costing its key blocks plus
+// about 2 block times of fixed work (Q load, first S, epilogue).  With fewer tiles than
+// SMs the longest tile bounds the launch, so each is cut into s contiguous shares of its
+// key blocks (at least 2 blocks each), all of them in one round (tiles * s <= SMs), and
+// a second kernel merges them (with the extra launch, about 8 block times more, as
+// measured on small launches).  The estimate is max(total / SMs, longest / s + fixed)
+// (+ 8 with a split); the cheapest split that saves 10% on no split is taken, with the
+// fp32 partials held under 256 MB.
+int fwd_kv_split(const FwdGeom& g, int Nq, int Nk, int d, int causal, int sms)
 {
     const int kt = kernel_d(d) == 256 ? 1 : 2;
-    const int n_pairs = (Nq + 128 * kt - 1) / (128 * kt);
-    const double bh = (double)B * Hq;
+    const double bh = (double)g.n_bh;
     double total = 0, longest = 0;
-    for (int pr = 0; pr < n_pairs; ++pr) {
+    for (int pr = 0; pr < g.n_pairs; ++pr) {
         int n = 0;
         for (int t = 0; t < kt; ++t)
-            n = std::max(n, host_blocks_for_tile(pr * 128 * kt + 128 * t, Nq, Nk, causal));
+            n = std::max(n, host_blocks_for_tile(pr * 128 * kt + 128 * t, g.rows, Nq, Nk, causal));
         total += n * bh;
         longest = std::max(longest, (double)n);
     }
-    const double tiles = n_pairs * bh, fixed = 2.0;
+    const double tiles = g.n_pairs * bh, fixed = 2.0;
     const double c1 = std::max((total + tiles * fixed) / sms, longest + fixed);
     static const int kShares[] = {2, 3, 4, 6, 8, 12, 16};
     int best = 1;
     double best_cost = c1;
     for (int sh : kShares) {
-        if (longest < 2.0 * sh || tiles * sh > sms || bh * sh * Nq * d * 4.0 > 256.0 * (1 << 20))
+        if (longest < 2.0 * sh || tiles * sh > sms || bh * sh * g.rows * d * 4.0 > 256.0 * (1 << 20))
             break;
         const double c = std::max((total + tiles * sh * fixed) / sms, longest / sh + fixed) + 8.0;
         if (c < best_cost && c < 0.9 * c1) {
@@ -325,10 +347,12 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     using C = fa::FwdCfg<D>;
     CUtensorMap mq, mk, mv;
     fa_status_t st;
-    if ((st = make_map(&mq, q, d, Nq, (uint64_t)B * Hq, 128, tma_type<T>())) != FA_OK) return st;
+    const FwdGeom g = fwd_geom(B, Hq, Hkv, Nq, d);
+    // q as [tile heads][rows][d]: with group rows a kv head's G query heads are one run of rows
+    if ((st = make_map(&mq, q, d, g.rows, (uint64_t)g.n_bh, 128, tma_type<T>())) != FA_OK) return st;
     if ((st = make_map(&mk, k, d, Nk, (uint64_t)B * Hkv, 128, tma_type<T>())) != FA_OK) return st;
     if ((st = make_map(&mv, v, d, Nk, (uint64_t)B * Hkv, 128, tma_type<T>())) != FA_OK) return st;
-    const int kv_split = fwd_kv_split(B, Hq, Nq, Nk, d, CAUSAL, sm_count());
+    const int kv_split = fwd_kv_split(g, Nq, Nk, d, CAUSAL, sm_count());
     auto kern = kv_split > 1 ? fa::fwd_kernel<D, CAUSAL, T, false, true> : fa::fwd_kernel<D, CAUSAL, T, false, false>;
     if ((st = ensure_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes)) != FA_OK) return st;
     fa::FwdParams p;
@@ -340,7 +364,10 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     p.Nq = Nq;
     p.Nk = Nk;
     p.G = Hq / Hkv;
-    p.n_pairs = (Nq + 128 * C::kTiles - 1) / (128 * C::kTiles);
+    p.group_rows = g.group_rows;
+    p.n_bh = g.n_bh;
+    p.rows = g.rows;
+    p.n_pairs = g.n_pairs;
     p.d_io = d;
     p.scale_log2 = scale * kLog2e;
     p.o_scale = 1.f;
@@ -352,7 +379,7 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     void* ws = nullptr;
     if (kv_split > 1) {
         // the shares' partials, stream-ordered scratch
-        const size_t rows = (size_t)B * Hq * kv_split * Nq;
+        const size_t rows = (size_t)g.n_bh * kv_split * g.rows;
         const size_t o_bytes = align256(rows * d * 4);
         cudaError_t e = scratch_alloc(&ws, o_bytes + align256(rows * 4), stream);
         if (e != cudaSuccess)
@@ -364,7 +391,7 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     st = check_launch("fwd_kernel launch");
     if (kv_split > 1) {
         if (st == FA_OK) {
-            const long long rows = (long long)B * Hq * Nq;
+            const long long rows = (long long)g.n_bh * g.rows;
             fa::fwd_combine_kernel<T><<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(p);
             st = check_launch("fwd_combine_kernel launch");
         }
@@ -414,6 +441,9 @@ fa_status_t launch_fwd_fp8(const void* q, const void* k, const void* v, void* vt
     p.Nk = Nk;
     p.G = Hq / Hkv;
     p.n_pairs = (Nq + 255) / 256;
+    p.group_rows = 0;   // one tile head per query head
+    p.n_bh = B * Hq;
+    p.rows = Nq;
     p.d_io = kF8D;
     p.scale_log2 = scale_log2;
     p.o_scale = o_scale;
@@ -1183,7 +1213,7 @@ int fa_fwd_kv_split(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal)
         return 0;
     if (decode_shape(Hq, Hkv, Nq, d))
         return 1;
-    return fwd_kv_split(B, Hq, Nq, Nk, d, causal, sm_count());
+    return fwd_kv_split(fwd_geom(B, Hq, Hkv, Nq, d), Nq, Nk, d, causal, sm_count());
 }
 
 int fa_bwd_query_split(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal)

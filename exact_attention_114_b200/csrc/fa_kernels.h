@@ -12,7 +12,13 @@ struct FwdParams {
     float* lse;         // [B, Hq, Nq] or nullptr
     int B, Hq, Hkv, Nq, Nk;
     int G;              // Hq / Hkv
-    int n_pairs;        // query tile pairs per head: ceil(Nq / 256) (ceil(Nq / 128) at d = 256)
+    int n_pairs;        // query tile pairs per tile head: ceil(rows / 256) (ceil(rows / 128) at d = 256)
+    // tile heads: with group_rows = 0 each (batch, query head), whose rows are its Nq query
+    // positions; with group_rows = 1 each (batch, kv head), whose rows are the G * Nq rows of its
+    // G query heads (consecutive in q / o / lse), row r at query position r % Nq
+    int group_rows;
+    int n_bh;           // B * Hq, or B * Hkv with group rows
+    int rows;           // Nq, or G * Nq with group rows
     int d_io;           // head dim of the tensors in memory (<= kernel D, multiple of 32); the
                         // columns d_io..D-1 of the tiles are TMA zero fill and are never stored
     float scale_log2;   // scale * log2(e) (times the Q and K descales for e4m3 inputs)
@@ -24,8 +30,8 @@ struct FwdParams {
     // tiles, share s taking the pair's key blocks [s * n / kv_split, (s + 1) * n / kv_split)
     // of its n; the shares' partial results are merged by fwd_combine_kernel
     int kv_split;
-    float* part_o;      // [B * Hq, kv_split, Nq, d_io] fp32: O_s = U_s / l_s of share s
-    float* part_lse;    // [B * Hq, kv_split, Nq] fp32: m_s + log2(l_s), -inf where share s sees no key
+    float* part_o;      // [n_bh, kv_split, rows, d_io] fp32: O_s = U_s / l_s of share s
+    float* part_lse;    // [n_bh, kv_split, rows] fp32: m_s + log2(l_s), -inf where share s sees no key
 };
 
 struct DecodeParams {

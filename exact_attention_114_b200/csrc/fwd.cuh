@@ -93,15 +93,19 @@ struct FwdCfg {
     static_assert(kTiles == 2 || 2 * 128 + D <= (int)kTmemCols, "one tile: two S buffers and O must fit in TMEM");
 };
 
-__device__ __forceinline__ int fwd_blocks_for_tile(int qt, int Nq, int Nk, bool causal)
+// 128-key blocks seen by the 128-row query tile at row qt of a tile head with `rows`
+// rows, row r at query position r % Nq (rows = Nq: position r)
+__device__ __forceinline__ int fwd_blocks_for_tile(int qt, int rows, int Nq, int Nk, bool causal)
 {
     const int nkb = (Nk + 127) / 128;
-    if (qt >= Nq)
+    if (qt >= rows)
         return 0;
     if (!causal)
         return nkb;
-    const int last_row = min(qt + 127, Nq - 1);
-    const int last_key = last_row + (Nk - Nq);
+    const int last_row = min(qt + 127, rows - 1);
+    // the largest query position among the tile's rows
+    const int last_pos = (qt / Nq == last_row / Nq) ? last_row % Nq : Nq - 1;
+    const int last_key = last_pos + (Nk - Nq);
     if (last_key < 0)
         return 0;
     return min(nkb, last_key / 128 + 1);
@@ -142,16 +146,20 @@ struct FwdTile {
 template <int kTiles, bool CAUSAL, bool SPLIT = false>
 __device__ __forceinline__ void fwd_tile(const FwdParams& p, int i, FwdTile& w)
 {
-    const int n_bh = p.B * p.Hq;
+    const int n_bh = p.n_bh;
     const int ns = SPLIT ? p.kv_split : 1;
     const int pair = p.n_pairs - 1 - i / (n_bh * ns);
     w.bh = i % n_bh;
     w.share = SPLIT ? (i / n_bh) % ns : 0;
-    const int b = w.bh / p.Hq, h = w.bh % p.Hq;
-    w.kvh = b * p.Hkv + h / p.G;
+    if (p.group_rows) {
+        w.kvh = w.bh;
+    } else {
+        const int b = w.bh / p.Hq, h = w.bh % p.Hq;
+        w.kvh = b * p.Hkv + h / p.G;
+    }
     w.q0 = pair * 128 * kTiles;
-    w.nb0 = fwd_blocks_for_tile(w.q0, p.Nq, p.Nk, CAUSAL);
-    w.nb1 = (kTiles == 2) ? fwd_blocks_for_tile(w.q0 + 128, p.Nq, p.Nk, CAUSAL) : 0;
+    w.nb0 = fwd_blocks_for_tile(w.q0, p.rows, p.Nq, p.Nk, CAUSAL);
+    w.nb1 = (kTiles == 2) ? fwd_blocks_for_tile(w.q0 + 128, p.rows, p.Nq, p.Nk, CAUSAL) : 0;
     w.kb0 = 0;
     if constexpr (SPLIT) {
         // blocks [lo, hi) of the pair's n; a tile sees the part of them below its own count
@@ -211,7 +219,7 @@ __global__ void __launch_bounds__(384, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* tile_ring = abort_flag + 1;          // [2]  tile indices (>= n_tiles: no more)
     static_assert((17 + 2 * C::kStages) * 8 + 16 <= C::kBarBytes, "barrier area too small");
-    const int n_tiles = p.n_pairs * p.B * p.Hq * (SPLIT ? p.kv_split : 1);
+    const int n_tiles = p.n_pairs * p.n_bh * (SPLIT ? p.kv_split : 1);
 
     const int warp = warp_id(), lane = lane_id();
     const int delta = p.Nk - p.Nq;
@@ -588,9 +596,9 @@ __global__ void __launch_bounds__(384, 1)
             if (!ok || tile >= n_tiles)
                 break;
             fwd_tile<C::kTiles, CAUSAL, SPLIT>(p, tile, w);
-            const int qi = w.q0 + 128 * t + r;
+            const int qi = w.q0 + 128 * t + r;   // row of the tile head
             const int nb = t ? w.nb1 : w.nb0;
-            const int qlim = qi + delta;
+            const int qlim = (p.group_rows ? qi % p.Nq : qi) + delta;   // last key its query position sees
             float m_ref = -INFINITY, l = 0.f;
 
             for (int j = 0; j < nb; ++j) {
@@ -728,8 +736,8 @@ __global__ void __launch_bounds__(384, 1)
                 break;
 
             // ---- epilogue: O = U / l (bf16), LSE = (m + log2 l) ln 2
-            const bool row_valid = (C::kTiles == 2 || t == 0) && qi < p.Nq;   // one-tile blocks: warps 4-7 idle
-            const size_t row = (size_t)w.bh * (size_t)p.Nq + (size_t)qi;
+            const bool row_valid = (C::kTiles == 2 || t == 0) && qi < p.rows;   // one-tile blocks: warps 4-7 idle
+            const size_t row = (size_t)w.bh * (size_t)p.rows + (size_t)qi;   // the same flat row either way
             if (nb > 0) {
                 ok = mbar_wait(&bar_o[t], (uint32_t)(no & 1), abort_flag);
                 ok = __all_sync(0xffffffffu, ok);
@@ -745,7 +753,7 @@ __global__ void __launch_bounds__(384, 1)
                     if constexpr (SPLIT) {
                         // this share's normalised partial O_s in fp32
                         if (row_valid) {
-                            const size_t prow = ((size_t)w.bh * p.kv_split + w.share) * p.Nq + qi;
+                            const size_t prow = ((size_t)w.bh * p.kv_split + w.share) * p.rows + qi;
                             float4* dst = reinterpret_cast<float4*>(p.part_o + prow * p.d_io + c0);
 #pragma unroll
                             for (int c = 0; c < 8; ++c)
@@ -771,14 +779,14 @@ __global__ void __launch_bounds__(384, 1)
                 tc_fence_before();
                 if constexpr (SPLIT) {
                     if (row_valid)
-                        p.part_lse[((size_t)w.bh * p.kv_split + w.share) * p.Nq + qi] =
+                        p.part_lse[((size_t)w.bh * p.kv_split + w.share) * p.rows + qi] =
                             (l > 0.f) ? m_ref + __log2f(l) : -INFINITY;
                 } else if (row_valid && p.lse) {
                     p.lse[row] = (l > 0.f) ? (m_ref + __log2f(l)) * kLn2 : -INFINITY;
                 }
             } else if (SPLIT && row_valid) {
                 // no key of this share for any row of the tile: its partial carries no weight
-                p.part_lse[((size_t)w.bh * p.kv_split + w.share) * p.Nq + qi] = -INFINITY;
+                p.part_lse[((size_t)w.bh * p.kv_split + w.share) * p.rows + qi] = -INFINITY;
             } else if (row_valid) {
                 // no visible key for any row of this tile
                 uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(p.o) + row * p.d_io);
@@ -813,44 +821,74 @@ __global__ void __launch_bounds__(128) fwd_combine_kernel(FwdParams p)
 {
     const long long row = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (row >= (long long)p.B * p.Hq * p.Nq)
+    if (row >= (long long)p.n_bh * p.rows)
         return;
-    const long long bh = row / p.Nq, i = row % p.Nq;
-    const int ns = p.kv_split;
-    const float* lse_s = p.part_lse + (size_t)bh * ns * p.Nq + i;
-    float M = -INFINITY;
-    for (int s = lane; s < ns; s += 32)
-        M = fmaxf(M, lse_s[(size_t)s * p.Nq]);
+    const long long bh = row / p.rows, i = row % p.rows;
+    const int ns = p.kv_split;   // <= 32: lane s holds share s's lse and weight
+    const float ls = lane < ns ? p.part_lse[((size_t)bh * ns + lane) * p.rows + i] : -INFINITY;
+    float M = ls;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1)
         M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    constexpr int kMaxPerLane = 8;   // d_io <= 256
-    float acc[kMaxPerLane];
+    const float wl = (M != -INFINITY && ls != -INFINITY) ? ex2_approx(ls - M) : 0.f;
+    float L = wl;
 #pragma unroll
-    for (int k = 0; k < kMaxPerLane; ++k)
+    for (int off = 16; off > 0; off >>= 1)
+        L += __shfl_xor_sync(0xffffffffu, L, off);
+    // lane l merges columns [n*l, n*l + n) of the row, n = d_io / 32 (<= 8): one or
+    // two 16-byte loads per share and lane where n is 4 or 8
+    const int n = p.d_io / 32;
+    float acc[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
         acc[k] = 0.f;
-    float L = 0.f;
-    const int per_lane = p.d_io / 32;
-    if (M != -INFINITY) {
-        for (int s = 0; s < ns; ++s) {
-            const float ls = lse_s[(size_t)s * p.Nq];
-            if (ls == -INFINITY)
-                continue;
-            const float wgt = ex2_approx(ls - M);
-            L += wgt;
-            const float* os = p.part_o + (((size_t)bh * ns + s) * p.Nq + i) * p.d_io + lane;
+    const float* o0 = p.part_o + (((size_t)bh * ns) * p.rows + i) * p.d_io + (size_t)n * lane;
+    const size_t share_stride = (size_t)p.rows * p.d_io;
+#pragma unroll 4
+    for (int s = 0; s < ns; ++s) {
+        const float w = __shfl_sync(0xffffffffu, wl, s);
+        if (w == 0.f)   // no key in this share (its O_s was never written) or a negligible one
+            continue;
+        const float* os = o0 + (size_t)s * share_stride;
+        if (n == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(os);
+            acc[0] = fmaf(w, v.x, acc[0]);
+            acc[1] = fmaf(w, v.y, acc[1]);
+            acc[2] = fmaf(w, v.z, acc[2]);
+            acc[3] = fmaf(w, v.w, acc[3]);
+        } else if (n == 8) {
+            const float4 v = *reinterpret_cast<const float4*>(os), u = *reinterpret_cast<const float4*>(os + 4);
+            acc[0] = fmaf(w, v.x, acc[0]);
+            acc[1] = fmaf(w, v.y, acc[1]);
+            acc[2] = fmaf(w, v.z, acc[2]);
+            acc[3] = fmaf(w, v.w, acc[3]);
+            acc[4] = fmaf(w, u.x, acc[4]);
+            acc[5] = fmaf(w, u.y, acc[5]);
+            acc[6] = fmaf(w, u.z, acc[6]);
+            acc[7] = fmaf(w, u.w, acc[7]);
+        } else {
 #pragma unroll
-            for (int k = 0; k < kMaxPerLane; ++k)
-                if (k < per_lane)
-                    acc[k] = fmaf(wgt, os[32 * k], acc[k]);
+            for (int k = 0; k < 8; ++k)
+                if (k < n)
+                    acc[k] = fmaf(w, os[k], acc[k]);
         }
     }
     const float inv = (L > 0.f) ? 1.f / L : 0.f;
-    T* o = static_cast<T*>(p.o) + (size_t)row * p.d_io + lane;
+    T* o = static_cast<T*>(p.o) + (size_t)row * p.d_io + (size_t)n * lane;
+    if (n == 4) {
+        *reinterpret_cast<uint2*>(o) = make_uint2(Elt<T>::pack(acc[0] * inv, acc[1] * inv),
+                                                  Elt<T>::pack(acc[2] * inv, acc[3] * inv));
+    } else if (n == 8) {
+        *reinterpret_cast<uint4*>(o) = make_uint4(Elt<T>::pack(acc[0] * inv, acc[1] * inv),
+                                                  Elt<T>::pack(acc[2] * inv, acc[3] * inv),
+                                                  Elt<T>::pack(acc[4] * inv, acc[5] * inv),
+                                                  Elt<T>::pack(acc[6] * inv, acc[7] * inv));
+    } else {
 #pragma unroll
-    for (int k = 0; k < kMaxPerLane; ++k)
-        if (k < per_lane)
-            o[32 * k] = Elt<T>::from_float(acc[k] * inv);
+        for (int k = 0; k < 8; ++k)
+            if (k < n)
+                o[k] = Elt<T>::from_float(acc[k] * inv);
+    }
     if (lane == 0 && p.lse)
         p.lse[row] = (L > 0.f) ? (M + __log2f(L)) * kLn2 : -INFINITY;
 }

@@ -288,7 +288,7 @@ def test_forward_key_split_rule():
     assert ks(1, 32, 8, 8192, 8192, 256, 1) == 1
     assert ks(64, 32, 8, 1, 8192, 128, 0) == 1        # decode shape
     assert ks(1, 32, 8, 512, 32768, 128, 1) == 2      # 64 work tiles of 254-256 key blocks
-    assert ks(1, 32, 8, 64, 32768, 128, 1) == 4       # 32 work tiles: four shares fill one round
+    assert ks(1, 32, 8, 64, 32768, 128, 1) == 16      # group rows: 8 work tiles (one per kv head)
     assert ks(1, 4, 1, 2048, 2048, 128, 1) == 4
     assert ks(1, 4, 1, 2048, 2048, 128, 0) == 4
     assert ks(1, 2, 1, 300, 5000, 64, 1) == 16

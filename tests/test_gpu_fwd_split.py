@@ -28,7 +28,7 @@ FWD_SPLIT_SHAPES = [
     (1, 4, 1, 200, 4096, 128, False, 16),
     # decode shapes at d = 256 (beyond the split-KV decode kernels' 128) take the tiled path
     (1, 8, 2, 1, 8192, 256, True, 16),
-    (2, 16, 4, 4, 16384, 256, True, 4),
+    (2, 16, 4, 4, 16384, 256, True, 16),
 ]
 
 
@@ -83,7 +83,7 @@ def test_fwd_split_fp16_with_backward():
 APPEND_SHAPES = [
     # a 512-row chunk appended to a 32K context, and a 64-row one (GQA 32 / 8)
     (1, 32, 8, 512, 32768, 128, True, 2),
-    (1, 32, 8, 64, 32768, 128, True, 4),
+    (1, 32, 8, 64, 32768, 128, True, 16),
 ]
 
 
@@ -102,3 +102,38 @@ def test_fwd_split_append_sampled(shape):
     G.assert_o(G.f64(o).reshape(-1, d)[rows], o_ref,
                o_abs=G.o_abs_ref(x["q"], x["k"], x["v"], w.scale, w.causal, rows=rows))
     G.assert_lse(G.f64(lse).reshape(-1)[rows], lse_ref)
+
+
+# Group rows: where a query head has fewer rows than a work tile (Nq < 256, or < 128 at
+# d = 256) and a kv head serves G > 1 query heads, the G * Nq rows of its heads share
+# the kv head's tiles (row r at query position r % Nq).  B, Hq, Hkv, Nq, Nk, d, causal
+GROUP_ROW_SHAPES = [
+    (64, 32, 8, 1, 8192, 256, False),    # d = 256 decode: 512 tiles, one per (batch, kv head)
+    (2, 12, 4, 37, 500, 128, True),      # G = 3, bottom-right mask with Nq < Nk
+    (1, 8, 2, 100, 100, 64, True),       # causal Nq = Nk: one tile mixes every query position
+    (2, 6, 2, 90, 260, 256, True),
+]
+
+
+@pytest.mark.parametrize("shape", GROUP_ROW_SHAPES, ids=[str(s) for s in GROUP_ROW_SHAPES])
+def test_group_rows_full(shape):
+    B, Hq, Hkv, Nq, Nk, d, causal = shape
+    w = synth.Workload("group_rows", B, Hq, Hkv, Nq, Nk, d, causal, 9700 + GROUP_ROW_SHAPES.index(shape))
+    x = synth.make_inputs(w, dout=False)
+    xd = {k: v.cuda() for k, v in x.items()}
+    o, lse, o2, _ = _forward_twice(w, xd)
+    assert torch.equal(o, o2)
+    o_ref, lse_ref = oracle.fwd(x["q"], x["k"], x["v"], w.scale, w.causal)
+    G.assert_o(G.f64(o), o_ref, o_abs=G.o_abs_ref(x["q"], x["k"], x["v"], w.scale, w.causal))
+    G.assert_lse(G.f64(lse), lse_ref)
+
+
+def test_group_rows_fp16():
+    w = synth.Workload("group_rows16", 1, 8, 2, 33, 2000, 128, False, 9790)
+    x = synth.make_inputs(w, dout=False, dtype=torch.float16)
+    xd = {k: v.cuda() for k, v in x.items()}
+    o, lse, _, _ = _forward_twice(w, xd)
+    xr = {k: v.double() for k, v in x.items()}
+    o_ref, lse_ref = oracle.fwd(xr["q"], xr["k"], xr["v"], w.scale, w.causal)
+    G.assert_o(G.f64(o), o_ref, o_abs=G.o_abs_ref(xr["q"], xr["k"], xr["v"], w.scale, w.causal))
+    G.assert_lse(G.f64(lse), lse_ref)
