@@ -96,11 +96,14 @@ const char* fa_last_error_message(void);
  *   the caller does not need it).
  *   scale multiplies q.k (usually 1/sqrt(d)); it must be finite and > 0.
  * Shapes with few query rows per kv head (Nq * Hq / Hkv <= 16, the decode shape
- * of §09) run the split-KV kernels; their partial results need scratch, which
+ * of §09) and d <= 128 run the split-KV kernels; their partial results need scratch, which
  * this call allocates and frees stream-ordered on `stream` (see Scratch
  * above).  Use fa_fwd_splitkv() to pass the scratch instead.
- * Other shapes run one persistent block per SM.  Where they have fewer work
- * tiles (pairs of 128-row query tiles of one head) than the GPU has SMs, each
+ * Other shapes run one persistent block per SM over work tiles of 256 query
+ * rows (128 at d > 128).  Where a kv head serves several query heads and each
+ * has fewer rows than a tile, the G * Nq rows of the kv head's query heads
+ * share its tiles (row r at query position r % Nq), so K/V are read once per
+ * kv head.  Where the launch has fewer work tiles than the GPU has SMs, each
  * tile's key blocks are cut into fa_fwd_kv_split(...) contiguous shares that
  * run as separate tiles; their partial results (fp32 O and LSE per share, in
  * scratch this call allocates and frees stream-ordered on `stream`) are merged
