@@ -112,6 +112,9 @@ GROUP_ROW_SHAPES = [
     (2, 12, 4, 37, 500, 128, True),      # G = 3, bottom-right mask with Nq < Nk
     (1, 8, 2, 100, 100, 64, True),       # causal Nq = Nk: one tile mixes every query position
     (2, 6, 2, 90, 260, 256, True),
+    (1, 4, 2, 200, 100, 128, True),      # Nq > Nk: positions below Nq - Nk see no key
+    (2, 8, 4, 130, 60, 64, True),
+    (3, 6, 2, 6, 700, 128, False),       # 18 rows per kv head: just past the decode kernels' 16
 ]
 
 
