@@ -340,6 +340,37 @@ fa_status_t fwd_tile_counter(unsigned** ctr, unsigned* tag)
     return FA_OK;
 }
 
+// The tiled forward's launch: with a key split (p.kv_split > 1) the shares' fp32 partials
+// go to stream-ordered scratch and fwd_combine_kernel merges them into o / lse.
+template <typename T, typename Kern>
+fa_status_t launch_fwd_tiles(Kern kern, int threads, int smem, const CUtensorMap& mq, const CUtensorMap& mk,
+                             const CUtensorMap& mv, fa::FwdParams& p, cudaStream_t stream)
+{
+    void* ws = nullptr;
+    if (p.kv_split > 1) {
+        const size_t rows = (size_t)p.n_bh * p.kv_split * p.rows;
+        const size_t o_bytes = align256(rows * p.d_io * 4);
+        cudaError_t e = scratch_alloc(&ws, o_bytes + align256(rows * 4), stream);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "scratch allocation (forward key-split partials)");
+        p.part_o = static_cast<float*>(ws);
+        p.part_lse = reinterpret_cast<float*>(static_cast<char*>(ws) + o_bytes);
+    }
+    kern<<<fwd_grid(p), threads, smem, stream>>>(mq, mk, mv, p);
+    fa_status_t st = check_launch("fwd_kernel launch");
+    if (p.kv_split > 1) {
+        if (st == FA_OK) {
+            const long long rows = (long long)p.n_bh * p.rows;
+            fa::fwd_combine_kernel<T><<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(p);
+            st = check_launch("fwd_combine_kernel launch");
+        }
+        cudaError_t e = cudaFreeAsync(ws, stream);
+        if (e != cudaSuccess && st == FA_OK)
+            st = cuda_fail(e, "cudaFreeAsync");
+    }
+    return st;
+}
+
 template <int D, bool CAUSAL, typename T>
 fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                        int Nq, int Nk, int d, float scale, cudaStream_t stream)
@@ -376,30 +407,7 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     p.part_lse = nullptr;
     if ((st = fwd_tile_counter(&p.tile_ctr, &p.tile_tag)) != FA_OK)
         return st;
-    void* ws = nullptr;
-    if (kv_split > 1) {
-        // the shares' partials, stream-ordered scratch
-        const size_t rows = (size_t)g.n_bh * kv_split * g.rows;
-        const size_t o_bytes = align256(rows * d * 4);
-        cudaError_t e = scratch_alloc(&ws, o_bytes + align256(rows * 4), stream);
-        if (e != cudaSuccess)
-            return cuda_fail(e, "scratch allocation (forward key-split partials)");
-        p.part_o = static_cast<float*>(ws);
-        p.part_lse = reinterpret_cast<float*>(static_cast<char*>(ws) + o_bytes);
-    }
-    kern<<<fwd_grid(p), C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
-    st = check_launch("fwd_kernel launch");
-    if (kv_split > 1) {
-        if (st == FA_OK) {
-            const long long rows = (long long)g.n_bh * g.rows;
-            fa::fwd_combine_kernel<T><<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(p);
-            st = check_launch("fwd_combine_kernel launch");
-        }
-        cudaError_t e = cudaFreeAsync(ws, stream);
-        if (e != cudaSuccess && st == FA_OK)
-            st = cuda_fail(e, "cudaFreeAsync");
-    }
-    return st;
+    return launch_fwd_tiles<T>(kern, C::kThreads, C::kSmemBytes, mq, mk, mv, p, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -424,12 +432,15 @@ fa_status_t launch_fwd_fp8(const void* q, const void* k, const void* v, void* vt
     fa_status_t st;
     if ((st = check_launch("fp8_vt_kernel launch")) != FA_OK) return st;
     constexpr CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    const FwdGeom g = fwd_geom(B, Hq, Hkv, Nq, kF8D);
     CUtensorMap mq, mk, mv;
-    if ((st = make_map_box(&mq, q, kF8D, Nq, (uint64_t)B * Hq, 1, 128, 128, u8)) != FA_OK) return st;
+    if ((st = make_map_box(&mq, q, kF8D, g.rows, (uint64_t)g.n_bh, 1, 128, 128, u8)) != FA_OK) return st;
     if ((st = make_map_box(&mk, k, kF8D, Nk, (uint64_t)B * Hkv, 1, 128, 128, u8)) != FA_OK) return st;
     // V^T [B * Hkv][d][nk_pad]: box of 128 keys x d rows
     if ((st = make_map_box(&mv, vt, nk_pad, kF8D, (uint64_t)B * Hkv, 1, 128, kF8D, u8)) != FA_OK) return st;
-    auto kern = fa::fwd_kernel<kF8D, CAUSAL, __nv_bfloat16, true>;
+    const int kv_split = fwd_kv_split(g, Nq, Nk, kF8D, CAUSAL, sm_count());
+    auto kern = kv_split > 1 ? fa::fwd_kernel<kF8D, CAUSAL, __nv_bfloat16, true, true>
+                             : fa::fwd_kernel<kF8D, CAUSAL, __nv_bfloat16, true, false>;
     if ((st = ensure_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes)) != FA_OK) return st;
     fa::FwdParams p;
     p.o = o;
@@ -440,20 +451,19 @@ fa_status_t launch_fwd_fp8(const void* q, const void* k, const void* v, void* vt
     p.Nq = Nq;
     p.Nk = Nk;
     p.G = Hq / Hkv;
-    p.n_pairs = (Nq + 255) / 256;
-    p.group_rows = 0;   // one tile head per query head
-    p.n_bh = B * Hq;
-    p.rows = Nq;
+    p.group_rows = g.group_rows;
+    p.n_bh = g.n_bh;
+    p.rows = g.rows;
+    p.n_pairs = g.n_pairs;
     p.d_io = kF8D;
     p.scale_log2 = scale_log2;
     p.o_scale = o_scale;
-    p.kv_split = 1;   // no key split for e4m3 inputs
+    p.kv_split = kv_split;
     p.part_o = nullptr;
     p.part_lse = nullptr;
     if ((st = fwd_tile_counter(&p.tile_ctr, &p.tile_tag)) != FA_OK)
         return st;
-    kern<<<fwd_grid(p), C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
-    return check_launch("fwd_kernel (e4m3) launch");
+    return launch_fwd_tiles<__nv_bfloat16>(kern, C::kThreads, C::kSmemBytes, mq, mk, mv, p, stream);
 }
 
 template <typename T>

@@ -143,7 +143,9 @@ fa_status_t fa_fwd_ex(fa_dtype_t dtype, const void* q, const void* k, const void
  *   to e4m3 for the P.V product (fp32 accumulation); the row sum l uses the
  *   fp32 P.  o [B,Hq,Nq,d] is bf16 (written); lse [B,Hq,Nq] fp32 (or NULL).
  *   d must be 128 (else FA_ERR_UNSUPPORTED).  Masking and shapes as fa_fwd,
- *   always on the tiled kernel.
+ *   always on the tiled kernel (decode shapes too), with fa_fwd's group rows
+ *   and key split (whose partials are fp32 scratch allocated and freed
+ *   stream-ordered, outside `workspace`).
  *   workspace: device scratch of fa_fwd_fp8_workspace_size(B, Hkv, Nk, d)
  *   bytes, 256-byte aligned, for V transposed to [B,Hkv,d,Nk rounded up to
  *   16]; NULL makes the call allocate it stream-ordered.  A smaller one returns

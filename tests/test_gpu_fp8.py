@@ -39,6 +39,8 @@ SHAPES = [
     (1, 2, 2, 513, 513, 128, False),
     (1, 4, 1, 1, 1000, 128, False),     # one query row: still the tiled kernel
     (2, 4, 2, 1000, 1000, 128, True),
+    (1, 32, 8, 64, 4096, 128, True),    # group rows (a kv head's 4 query heads share tiles), key split
+    (4, 32, 8, 1, 4096, 128, False),    # decode shape on the tiled kernel: group rows, key split
 ]
 
 
