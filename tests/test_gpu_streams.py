@@ -20,6 +20,8 @@ CASES = [
     ("d64", 2, 12, 4, 2048, 2048, 64, True, torch.bfloat16),
     ("d256", 1, 4, 4, 777, 777, 256, True, torch.bfloat16),
     ("fp16", 1, 16, 16, 1024, 1024, 128, True, torch.float16),
+    ("group_rows", 2, 16, 4, 40, 3000, 128, True, torch.bfloat16),    # kv heads' rows share tiles, key split
+    ("decode_d256", 4, 16, 4, 1, 4096, 256, False, torch.bfloat16),
 ]
 
 
@@ -104,3 +106,43 @@ def test_slot_held_by_another_launch_is_reported_not_silent():
     torch.cuda.synchronize()
     fa.fa_check_device_status()
     assert torch.equal(o2, o_ref) and torch.equal(l2, l_ref)
+
+
+# backward shapes whose units are shared by several CTAs (query split): each call's
+# counters and fp32 partials live in its own workspace
+BWD_CASES = [
+    ("split8", 1, 4, 1, 2048, 2048, 128, True),
+    ("split4_d256", 1, 2, 1, 2048, 2048, 256, True),
+    ("split2_noncausal", 1, 1, 1, 2048, 2048, 64, False),
+]
+
+
+def test_concurrent_backward_streams_match_serial():
+    probs = []
+    for i, (name, B, Hq, Hkv, Nq, Nk, d, causal) in enumerate(BWD_CASES):
+        w = synth.Workload(name, B, Hq, Hkv, Nq, Nk, d, causal, 7400 + i)
+        x = {k: v.cuda() for k, v in synth.make_inputs(w).items()}
+        o, lse = fa.fa_fwd(x["q"], x["k"], x["v"], causal=causal)
+        probs.append((w, x, o, lse))
+    ref = []
+    for w, x, o, lse in probs:
+        g = fa.fa_bwd(x["q"], x["k"], x["v"], o, x["dout"], lse, causal=w.causal)
+        torch.cuda.synchronize()
+        ref.append([t.clone() for t in g])
+    streams = [torch.cuda.Stream() for _ in range(3)]
+    rounds = 2
+    outs = [[[torch.empty_like(t) for t in ref[j]] for j in range(len(probs))] for _ in range(rounds)]
+    torch.cuda.synchronize()
+    for r in range(rounds):
+        for j, (w, x, o, lse) in enumerate(probs):
+            fa.fa_bwd(x["q"], x["k"], x["v"], o, x["dout"], lse, *outs[r][j], causal=w.causal,
+                      stream=streams[(r + j) % len(streams)])
+    torch.cuda.synchronize()
+    fa.fa_check_device_status()
+    for r in range(rounds):
+        for j, (w, *_rest) in enumerate(probs):
+            dq, dk, dv = outs[r][j]
+            # dK / dV: fixed-order sums, bitwise; dQ: fp32 reductions in any order
+            assert torch.equal(dk, ref[j][1]) and torch.equal(dv, ref[j][2]), (w.name, r)
+            err = (dq.float() - ref[j][0].float()).abs().max().item()
+            assert err <= 1e-2 * ref[j][0].float().abs().max().item(), (w.name, r, err)
