@@ -5,8 +5,10 @@
 // numerator and denominator together by exp(m_old - m_new), add the block).
 //
 // Layout of one CTA (384 threads = 3 warpgroups, one CTA per SM):
-//   * per work tile, two 128-row query tiles of one (batch, head), Q0 and Q1,
-//     staged in shared memory by TMA (128-byte swizzle, 64-column panels);
+//   * per work tile, two 128-row query tiles of one tile head, Q0 and Q1, staged
+//     in shared memory by TMA (128-byte swizzle, 64-column panels); a tile head is
+//     a (batch, query head), or a (batch, kv head) whose G query heads' rows
+//     share its tiles when each has fewer rows than a tile (group rows);
 //   * K and V blocks of 128 keys stream through one ring of NSTAGE tile slots
 //     (order K0, V0, K1, V1, ...), each slot guarded by a full / empty mbarrier;
 //   * tensor memory (512 columns): S0 | S1 (128 fp32 columns each) | O0 | O1
@@ -21,7 +23,7 @@
 //     third warpgroup, which hands most of its registers to the softmax ones.
 //
 // The launch is persistent: one CTA per SM works through the (query tile pair,
-// batch, head) tiles, heaviest causal tiles first, each CTA claiming its next
+// tile head) tiles, heaviest causal tiles first, each CTA claiming its next
 // tile from an atomic counter (fwd_tile).  The TMA warp claims it and hands it
 // to the other roles through a two-entry ring in shared memory.  TMEM,
 // barriers and the K/V ring carry over from tile to tile.  The producer reloads a
@@ -125,11 +127,12 @@ constexpr int kFwdCtrSlots = 256;
 constexpr int kFwdCtrWords = 4;
 __device__ unsigned g_fwd_tile_ctr[kFwdCtrSlots][kFwdCtrWords];
 
-// One work tile: a pair of 128-row query tiles (one at d = 256) of one
-// (batch, head).  Tile i of the launch: pair n_pairs-1 - i / (B*Hq) (heaviest
-// causal pairs first), (batch, head) i % (B*Hq).
+// One work tile: a pair of 128-row query tiles (one at d = 256) of one tile head
+// (see FwdParams::group_rows).  Tile i of the launch: pair n_pairs-1 - i / n_bh
+// (heaviest causal pairs first; with a key split, i / (n_bh * kv_split)), tile head
+// i % n_bh.
 struct FwdTile {
-    int bh;        // batch * Hq + head
+    int bh;        // tile head: batch * Hq + head, or batch * Hkv + kv head with group rows
     int kvh;       // batch * Hkv + kv head
     int q0;        // first query row
     int nb0, nb1;  // 128-key blocks seen by query tile 0 / 1 (in this tile's key share)
