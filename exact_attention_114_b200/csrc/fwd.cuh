@@ -82,6 +82,10 @@ struct FwdCfg {
     static constexpr int kKSteps = D * kElt / 32;        // Q.K^T instructions (32 bytes of d each)
     static constexpr int kStages = F8 ? 10 : (D == 256) ? 2 : (D == 128) ? 5 : 8;
     static constexpr int kBarBytes = 512;
+    // part of the exponentials on the FMA pipe (exp2_poly2): pays at d = 128 and for
+    // e4m3, where the MUFU unit is the busier one; at d = 64 and 256 all of them on the
+    // MUFU measured faster (the FMA-pipe work slows the co-running MMA issue more)
+    static constexpr bool kPoly = F8 || D == 128;
     static constexpr int kOffQ = 0;
     static constexpr int kOffKV = kTiles * kTileBytes;
     static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
@@ -669,10 +673,10 @@ __global__ void __launch_bounds__(384, 1)
                 const float2 sl22 = make_float2(sl2, sl2), nm2 = make_float2(neg_m, neg_m);
                 float2 acc = make_float2(0.f, 0.f);
                 // One exp2 per score: the MUFU unit would be as busy as the tensor
-                // core at d = 128, so in blocks without masked scores one pair in
-                // four goes to the FMA-pipe exp2 instead (masked -inf scores always
-                // take ex2.approx, which returns exactly 0 for them).
-                const bool soft = !__any_sync(0xffffffffu, need_mask);
+                // core at d = 128, so there (kPoly) in blocks without masked scores
+                // one pair in four goes to the FMA-pipe exp2 instead (masked -inf
+                // scores always take ex2.approx, which returns exactly 0 for them).
+                const bool soft = C::kPoly && !__any_sync(0xffffffffu, need_mask);
                 auto half_block_f8 = [&](int hf, auto use_poly) {
                     uint32_t pk[16];
 #pragma unroll
