@@ -730,6 +730,8 @@ PROFILE_CASES = {
     # head size 256: Q and O 64 MiB each, K and V 16 MiB each
     "fwd_d256": ("gqa_8k", dict(Nq=4096, Nk=4096, d=256)),
     "bwd_d256": ("gqa_8k", dict(Nq=4096, Nk=4096, d=256)),
+    # a 512-row chunk appended to 32K keys: the forward's key split (K and V 64 MiB each)
+    "fwd_append": ("gqa_8k", dict(Nq=512, Nk=32768)),
 }
 
 
