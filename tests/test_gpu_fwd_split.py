@@ -29,6 +29,7 @@ FWD_SPLIT_SHAPES = [
     # decode shapes at d = 256 (beyond the split-KV decode kernels' 128) take the tiled path
     (1, 8, 2, 1, 8192, 256, True, 16),
     (2, 16, 4, 4, 16384, 256, True, 16),
+    (2, 4, 4, 1, 5000, 256, False, 16),     # MHA decode at d = 256: one row per tile head, key split only
 ]
 
 
