@@ -15,6 +15,8 @@
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <queue>
+#include <vector>
 #include <string>
 #include <type_traits>
 
@@ -237,7 +239,8 @@ int kernel_d(int d) { return d <= 64 ? 64 : d <= 128 ? 128 : 256; }
 // second), together working through the n_pairs * n_bh (* kv_split) tiles.
 unsigned fwd_grid(const fa::FwdParams& p)
 {
-    const long long tiles = (long long)p.n_pairs * p.n_bh * p.kv_split;
+    const long long units = (long long)p.n_pairs * p.n_bh;
+    const long long tiles = p.kv_split > 1 ? p.full_tiles + (units - p.full_tiles) * p.kv_split : units;
     return (unsigned)std::max<long long>(1, std::min<long long>(tiles, sm_count()));
 }
 
@@ -279,41 +282,98 @@ int host_blocks_for_tile(int qt, int rows, int Nq, int Nk, int causal)
     return last_key < 0 ? 0 : (int)std::min<long long>(nkb, last_key / 128 + 1);
 }
 
-// Key shares per work tile (query tile pair of a tile head) of the tiled forward.
-// Unsplit, the launch has n_pairs * n_bh work tiles, each costing its key blocks plus
-// about 2 block times of fixed work (Q load, first S, epilogue).  With fewer tiles than
-// SMs the longest tile bounds the launch, so each is cut into s contiguous shares of its
-// key blocks (at least 2 blocks each), all of them in one round (tiles * s <= SMs), and
-// a second kernel merges them (with the extra launch, about 8 block times more, as
-// measured on small launches).  The estimate is max(total / SMs, longest / s + fixed)
-// (+ 8 with a split); the cheapest split that saves 10% on no split is taken, with the
-// fp32 partials held under 256 MB.
-int fwd_kv_split(const FwdGeom& g, int Nq, int Nk, int d, int causal, int sms)
+// Key split of the tiled forward.  The persistent launch claims its work units (query tile
+// pair, tile head) heaviest first; a unit costs its key blocks plus about 2 block times of
+// fixed work (Q load, first S, epilogue).  With few units, or a last round that fills few
+// SMs, units are cut into s contiguous shares of their key blocks (each share a work tile of
+// its own, writing an fp32 partial that fwd_combine_kernel merges): either every unit, or only
+// the units after the last full round of whole units (full_tiles of them stay whole and write
+// o / lse directly).  Each choice is scored by simulating the greedy claiming on the SMs, plus
+// the merge: about 8 block times of launch and fixed work and the partials' traffic (written
+// and read, 13 MB per block time at the copy bandwidth).  A split is taken where it saves at
+// least 5%; launches with more than 8 units per SM are balanced enough by the claiming alone.
+// A tail split keeps to 2 shares when K and V take more than 64 MB: the whole units of a kv
+// head stream its keys together and mostly hit in L2, while the shares of one unit read
+// different key ranges at once (4 shares on a 2048-row chunk against 32K keys: no gain, with
+// 8% in the simulation).  The choice depends only on the sizes and the SM count, and is cached.
+struct FwdSplit {
+    int shares, full;
+};
+
+FwdSplit fwd_split_plan(const FwdGeom& g, int B, int Hkv, int Nq, int Nk, int d, int causal, int sms)
 {
+    const long long n_units = (long long)g.n_pairs * g.n_bh;
+    if (n_units > 8LL * sms || n_units < 1)
+        return {1, (int)n_units};
+    static std::mutex mu;
+    static std::map<std::vector<long long>, FwdSplit> cache;
+    const std::vector<long long> key{g.n_pairs, g.n_bh, g.rows, B, Hkv, Nq, Nk, d, causal, sms};
+    const double kv_bytes = 4.0 * B * Hkv * (double)Nk * d;   // K and V, 16-bit
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        auto it = cache.find(key);
+        if (it != cache.end())
+            return it->second;
+    }
     const int kt = kernel_d(d) == 256 ? 1 : 2;
-    const double bh = (double)g.n_bh;
-    double total = 0, longest = 0;
+    std::vector<int> pair_len((size_t)g.n_pairs);
     for (int pr = 0; pr < g.n_pairs; ++pr) {
         int n = 0;
         for (int t = 0; t < kt; ++t)
             n = std::max(n, host_blocks_for_tile(pr * 128 * kt + 128 * t, g.rows, Nq, Nk, causal));
-        total += n * bh;
-        longest = std::max(longest, (double)n);
+        pair_len[(size_t)pr] = n;
     }
-    const double tiles = g.n_pairs * bh, fixed = 2.0;
-    const double c1 = std::max((total + tiles * fixed) / sms, longest + fixed);
+    auto unit_len = [&](long long u) { return pair_len[(size_t)(g.n_pairs - 1 - u / g.n_bh)]; };
+    const double fixed = 2.0, merge_fixed = 8.0, bytes_per_block = 13.0e6;
+    // greedy claiming of the work tiles in order on `sms` CTAs: the last finish
+    auto simulate = [&](long long full, int sh) {
+        std::priority_queue<double, std::vector<double>, std::greater<double>> done;
+        double last = 0;
+        auto take = [&](double len) {
+            double start = 0;
+            if ((int)done.size() == sms) {
+                start = done.top();
+                done.pop();
+            }
+            done.push(start + len + fixed);
+            last = std::max(last, start + len + fixed);
+        };
+        for (long long u = 0; u < n_units; ++u) {
+            const int n = unit_len(u);
+            if (u < full || sh == 1) {
+                take(n);
+            } else {
+                for (int k = 0; k < sh; ++k)
+                    take((double)(((long long)(k + 1) * n) / sh - ((long long)k * n) / sh));
+            }
+        }
+        return last;
+    };
+    const double base = simulate(n_units, 1);
+    FwdSplit best{1, (int)n_units};
+    double best_cost = base;
     static const int kShares[] = {2, 3, 4, 6, 8, 12, 16};
-    int best = 1;
-    double best_cost = c1;
-    for (int sh : kShares) {
-        if (longest < 2.0 * sh || tiles * sh > sms || bh * sh * g.rows * d * 4.0 > 256.0 * (1 << 20))
-            break;
-        const double c = std::max((total + tiles * sh * fixed) / sms, longest / sh + fixed) + 8.0;
-        if (c < best_cost && c < 0.9 * c1) {
-            best = sh;
-            best_cost = c;
+    const long long fulls[2] = {0, (n_units / sms) * sms};
+    for (long long full : fulls) {
+        if (full >= n_units || (full > 0 && full == fulls[0]))
+            continue;
+        int longest = 0;
+        for (long long u = full; u < n_units; ++u)
+            longest = std::max(longest, unit_len(u));
+        for (int sh : kShares) {
+            const double part_bytes = (double)(n_units - full) * sh * 128 * kt * d * 4.0;
+            if (longest < 2 * sh || part_bytes > 256.0 * (1 << 20) ||
+                (full > 0 && sh > 2 && kv_bytes > 64.0 * (1 << 20)))
+                break;
+            const double cost = simulate(full, sh) + merge_fixed + 2.0 * part_bytes / bytes_per_block;
+            if (cost < best_cost && cost < 0.95 * base) {
+                best = {sh, (int)full};
+                best_cost = cost;
+            }
         }
     }
+    std::lock_guard<std::mutex> lk(mu);
+    cache[key] = best;
     return best;
 }
 
@@ -348,6 +408,7 @@ fa_status_t launch_fwd_tiles(Kern kern, int threads, int smem, const CUtensorMap
 {
     void* ws = nullptr;
     if (p.kv_split > 1) {
+        // indexed by tile head and share: [n_bh][kv_split][rows] (only split units' rows used)
         const size_t rows = (size_t)p.n_bh * p.kv_split * p.rows;
         const size_t o_bytes = align256(rows * p.d_io * 4);
         cudaError_t e = scratch_alloc(&ws, o_bytes + align256(rows * 4), stream);
@@ -383,7 +444,8 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     if ((st = make_map(&mq, q, d, g.rows, (uint64_t)g.n_bh, 128, tma_type<T>())) != FA_OK) return st;
     if ((st = make_map(&mk, k, d, Nk, (uint64_t)B * Hkv, 128, tma_type<T>())) != FA_OK) return st;
     if ((st = make_map(&mv, v, d, Nk, (uint64_t)B * Hkv, 128, tma_type<T>())) != FA_OK) return st;
-    const int kv_split = fwd_kv_split(g, Nq, Nk, d, CAUSAL, sm_count());
+    const FwdSplit sp = fwd_split_plan(g, B, Hkv, Nq, Nk, d, CAUSAL, sm_count());
+    const int kv_split = sp.shares;
     auto kern = kv_split > 1 ? fa::fwd_kernel<D, CAUSAL, T, false, true> : fa::fwd_kernel<D, CAUSAL, T, false, false>;
     if ((st = ensure_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes)) != FA_OK) return st;
     fa::FwdParams p;
@@ -403,6 +465,8 @@ fa_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     p.scale_log2 = scale * kLog2e;
     p.o_scale = 1.f;
     p.kv_split = kv_split;
+    p.full_tiles = sp.full;
+    p.pair_rows = 128 * C::kTiles;
     p.part_o = nullptr;
     p.part_lse = nullptr;
     if ((st = fwd_tile_counter(&p.tile_ctr, &p.tile_tag)) != FA_OK)
@@ -438,7 +502,8 @@ fa_status_t launch_fwd_fp8(const void* q, const void* k, const void* v, void* vt
     if ((st = make_map_box(&mk, k, kF8D, Nk, (uint64_t)B * Hkv, 1, 128, 128, u8)) != FA_OK) return st;
     // V^T [B * Hkv][d][nk_pad]: box of 128 keys x d rows
     if ((st = make_map_box(&mv, vt, nk_pad, kF8D, (uint64_t)B * Hkv, 1, 128, kF8D, u8)) != FA_OK) return st;
-    const int kv_split = fwd_kv_split(g, Nq, Nk, kF8D, CAUSAL, sm_count());
+    const FwdSplit sp = fwd_split_plan(g, B, Hkv, Nq, Nk, kF8D, CAUSAL, sm_count());
+    const int kv_split = sp.shares;
     auto kern = kv_split > 1 ? fa::fwd_kernel<kF8D, CAUSAL, __nv_bfloat16, true, true>
                              : fa::fwd_kernel<kF8D, CAUSAL, __nv_bfloat16, true, false>;
     if ((st = ensure_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes)) != FA_OK) return st;
@@ -459,6 +524,8 @@ fa_status_t launch_fwd_fp8(const void* q, const void* k, const void* v, void* vt
     p.scale_log2 = scale_log2;
     p.o_scale = o_scale;
     p.kv_split = kv_split;
+    p.full_tiles = sp.full;
+    p.pair_rows = 256;
     p.part_o = nullptr;
     p.part_lse = nullptr;
     if ((st = fwd_tile_counter(&p.tile_ctr, &p.tile_tag)) != FA_OK)
@@ -1223,7 +1290,7 @@ int fa_fwd_kv_split(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal)
         return 0;
     if (decode_shape(Hq, Hkv, Nq, d))
         return 1;
-    return fwd_kv_split(fwd_geom(B, Hq, Hkv, Nq, d), Nq, Nk, d, causal, sm_count());
+    return fwd_split_plan(fwd_geom(B, Hq, Hkv, Nq, d), B, Hkv, Nq, Nk, d, causal, sm_count()).shares;
 }
 
 int fa_bwd_query_split(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal)

@@ -26,10 +26,14 @@ struct FwdParams {
     unsigned* tile_ctr; // [4]: tiles claimed beyond each block's first, blocks done claiming,
                         // owner tag (zero when free; the last block resets all three), padding
     unsigned tile_tag;  // this launch's owner tag (nonzero)
-    // key split (fwd_kernel<..., SPLIT = true>): each (query tile pair, head) is kv_split work
-    // tiles, share s taking the pair's key blocks [s * n / kv_split, (s + 1) * n / kv_split)
-    // of its n; the shares' partial results are merged by fwd_combine_kernel
+    // key split (fwd_kernel<..., SPLIT = true>): the work units (query tile pair, tile head) in
+    // claim order u = 0, 1, ...; units u < full_tiles are one work tile each, every later unit is
+    // kv_split work tiles, share s taking the pair's key blocks [s * n / kv_split,
+    // (s + 1) * n / kv_split) of its n; the shares' partial results are merged by
+    // fwd_combine_kernel (full_tiles = 0: every unit is split)
     int kv_split;
+    int full_tiles;
+    int pair_rows;      // query rows of a work unit: 256 (128 at d = 256)
     float* part_o;      // [n_bh, kv_split, rows, d_io] fp32: O_s = U_s / l_s of share s
     float* part_lse;    // [n_bh, kv_split, rows] fp32: m_s + log2(l_s), -inf where share s sees no key
 };

@@ -143,6 +143,7 @@ struct FwdTile {
     int n_iter;    // max of the two
     int kb0;       // first key block of the share (0 without a key split)
     int share;     // key share (0 without a key split)
+    int nshares;   // key shares of the tile's unit (1: the whole unit, written straight to o / lse)
 };
 
 // The launch has at most one block per SM.  Block c starts with tile c; each
@@ -154,10 +155,19 @@ template <int kTiles, bool CAUSAL, bool SPLIT = false>
 __device__ __forceinline__ void fwd_tile(const FwdParams& p, int i, FwdTile& w)
 {
     const int n_bh = p.n_bh;
-    const int ns = SPLIT ? p.kv_split : 1;
-    const int pair = p.n_pairs - 1 - i / (n_bh * ns);
-    w.bh = i % n_bh;
-    w.share = SPLIT ? (i / n_bh) % ns : 0;
+    // unit u = (pair n_pairs - 1 - u / n_bh, tile head u % n_bh); units below full_tiles whole
+    int u = i, ns = 1;
+    w.share = 0;
+    if constexpr (SPLIT) {
+        if (i >= p.full_tiles) {
+            ns = p.kv_split;
+            u = p.full_tiles + (i - p.full_tiles) / ns;
+            w.share = (i - p.full_tiles) % ns;
+        }
+    }
+    w.nshares = ns;
+    const int pair = p.n_pairs - 1 - u / n_bh;
+    w.bh = u % n_bh;
     if (p.group_rows) {
         w.kvh = w.bh;
     } else {
@@ -168,7 +178,7 @@ __device__ __forceinline__ void fwd_tile(const FwdParams& p, int i, FwdTile& w)
     w.nb0 = fwd_blocks_for_tile(w.q0, p.rows, p.Nq, p.Nk, CAUSAL);
     w.nb1 = (kTiles == 2) ? fwd_blocks_for_tile(w.q0 + 128, p.rows, p.Nq, p.Nk, CAUSAL) : 0;
     w.kb0 = 0;
-    if constexpr (SPLIT) {
+    if (SPLIT && ns > 1) {
         // blocks [lo, hi) of the pair's n; a tile sees the part of them below its own count
         const int n = max(w.nb0, w.nb1);
         const int lo = (int)(((long long)w.share * n) / ns), hi = (int)(((long long)(w.share + 1) * n) / ns);
@@ -226,7 +236,8 @@ __global__ void __launch_bounds__(384, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* tile_ring = abort_flag + 1;          // [2]  tile indices (>= n_tiles: no more)
     static_assert((17 + 2 * C::kStages) * 8 + 16 <= C::kBarBytes, "barrier area too small");
-    const int n_tiles = p.n_pairs * p.n_bh * (SPLIT ? p.kv_split : 1);
+    const int n_units = p.n_pairs * p.n_bh;
+    const int n_tiles = SPLIT ? p.full_tiles + (n_units - p.full_tiles) * p.kv_split : n_units;
 
     const int warp = warp_id(), lane = lane_id();
     const int delta = p.Nk - p.Nq;
@@ -757,7 +768,7 @@ __global__ void __launch_bounds__(384, 1)
                 for (int c0 = 0; c0 < p.d_io; c0 += 32) {
                     uint32_t o[32];
                     tmem_ld32(tO + (uint32_t)c0, o);
-                    if constexpr (SPLIT) {
+                    if (SPLIT && w.nshares > 1) {
                         // this share's normalised partial O_s in fp32
                         if (row_valid) {
                             const size_t prow = ((size_t)w.bh * p.kv_split + w.share) * p.rows + qi;
@@ -784,14 +795,14 @@ __global__ void __launch_bounds__(384, 1)
                 // O(t) is read out: the next tile's first P.V may overwrite it once this
                 // warpgroup's P of that tile is signalled (after the fence in the P write)
                 tc_fence_before();
-                if constexpr (SPLIT) {
+                if (SPLIT && w.nshares > 1) {
                     if (row_valid)
                         p.part_lse[((size_t)w.bh * p.kv_split + w.share) * p.rows + qi] =
                             (l > 0.f) ? m_ref + __log2f(l) : -INFINITY;
                 } else if (row_valid && p.lse) {
                     p.lse[row] = (l > 0.f) ? (m_ref + __log2f(l)) * kLn2 : -INFINITY;
                 }
-            } else if (SPLIT && row_valid) {
+            } else if (SPLIT && w.nshares > 1 && row_valid) {
                 // no key of this share for any row of the tile: its partial carries no weight
                 p.part_lse[((size_t)w.bh * p.kv_split + w.share) * p.rows + qi] = -INFINITY;
             } else if (row_valid) {
@@ -831,6 +842,10 @@ __global__ void __launch_bounds__(128) fwd_combine_kernel(FwdParams p)
     if (row >= (long long)p.n_bh * p.rows)
         return;
     const long long bh = row / p.rows, i = row % p.rows;
+    // rows of the whole units (written straight to o / lse by the forward) are final
+    const long long unit = (long long)(p.n_pairs - 1 - (int)(i / p.pair_rows)) * p.n_bh + bh;
+    if (unit < p.full_tiles)
+        return;
     const int ns = p.kv_split;   // <= 32: lane s holds share s's lse and weight
     const float ls = lane < ns ? p.part_lse[((size_t)bh * ns + lane) * p.rows + i] : -INFINITY;
     float M = ls;

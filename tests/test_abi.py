@@ -295,6 +295,9 @@ def test_forward_key_split_rule():
     assert ks(1, 2, 1, 1000, 2000, 256, 0) == 8
     assert ks(1, 4, 1, 1000, 1000, 128, 1) == 1       # 16 tiles of at most 8 blocks: too little to gain
     assert ks(1, 8, 2, 1, 8192, 256, 1) == 16         # a d = 256 decode shape runs the tiled kernel
+    assert ks(1, 32, 8, 1024, 32768, 128, 1) == 1     # 128 equal units: one round, splitting costs more
+    assert ks(1, 32, 8, 2048, 32768, 128, 1) == 1     # 256 units: 4-share tail, but K / V beyond L2 (no gain)
+    assert ks(1, 32, 8, 4096, 32768, 128, 1) == 2     # 512 units: the last 68 in 2 shares
     assert ks(1, 3, 2, 64, 64, 64, 0) == 0            # Hq not a multiple of Hkv
     assert ks(1, 2, 1, 64, 64, 80, 0) == 0            # head size not a multiple of 32
     assert fa.lib().fa_fwd_kv_split(1, 2, 1, 64, 64, 64, 2) == 0

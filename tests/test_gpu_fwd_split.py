@@ -85,6 +85,11 @@ APPEND_SHAPES = [
     # a 512-row chunk appended to a 32K context, and a 64-row one (GQA 32 / 8)
     (1, 32, 8, 512, 32768, 128, True, 2),
     (1, 32, 8, 64, 32768, 128, True, 16),
+    # a 4096-row chunk: 512 equal units; the 68 after the last full round of 148 run in two
+    # shares (a tail split), the others whole.  (A 2048-row one stays whole: with K and V
+    # beyond L2 its 4-share tail gained nothing.)
+    (1, 32, 8, 2048, 32768, 128, True, 1),
+    (1, 32, 8, 4096, 32768, 128, True, 2),
 ]
 
 
@@ -103,6 +108,34 @@ def test_fwd_split_append_sampled(shape):
     G.assert_o(G.f64(o).reshape(-1, d)[rows], o_ref,
                o_abs=G.o_abs_ref(x["q"], x["k"], x["v"], w.scale, w.causal, rows=rows))
     G.assert_lse(G.f64(lse).reshape(-1)[rows], lse_ref)
+
+
+# Tail split: more units than SMs, with a last round that would leave most SMs idle; the
+# first 148 units (claimed first, heaviest first) run whole and write o / lse directly, the
+# rest run in shares merged by the merge kernel, which leaves the whole units' rows alone.
+TAIL_SHAPES = [
+    (1, 20, 4, 2048, 2048, 64, False, 8),
+    (1, 40, 8, 1024, 3000, 64, True, 4),
+    (2, 40, 8, 512, 3000, 64, True, 8),
+    (1, 20, 4, 2048, 2048, 128, False, 8),
+    (2, 20, 4, 1024, 3000, 128, True, 4),
+    (1, 20, 4, 1024, 3000, 256, False, 12),
+]
+
+
+@pytest.mark.parametrize("shape", TAIL_SHAPES, ids=[str(s) for s in TAIL_SHAPES])
+def test_fwd_tail_split_full(shape):
+    B, Hq, Hkv, Nq, Nk, d, causal, shares = shape
+    if _sms() == 148:
+        assert fa.fa_fwd_kv_split(B, Hq, Hkv, Nq, Nk, d, causal) == shares
+    w = synth.Workload("tail_split", B, Hq, Hkv, Nq, Nk, d, causal, 9850 + TAIL_SHAPES.index(shape))
+    x = synth.make_inputs(w, dout=False)
+    xd = {k: v.cuda() for k, v in x.items()}
+    o, lse, o2, l2 = _forward_twice(w, xd)
+    assert torch.equal(o, o2) and torch.equal(lse, l2)
+    o_ref, lse_ref = oracle.fwd(x["q"], x["k"], x["v"], w.scale, w.causal)
+    G.assert_o(G.f64(o), o_ref, o_abs=G.o_abs_ref(x["q"], x["k"], x["v"], w.scale, w.causal))
+    G.assert_lse(G.f64(lse), lse_ref)
 
 
 # Group rows: where a query head has fewer rows than a work tile (Nq < 256, or < 128 at
