@@ -103,11 +103,13 @@ const char* fa_last_error_message(void);
  * rows (128 at d > 128).  Where a kv head serves several query heads and each
  * has fewer rows than a tile, the G * Nq rows of the kv head's query heads
  * share its tiles (row r at query position r % Nq), so K/V are read once per
- * kv head.  Where the launch has fewer work tiles than the GPU has SMs, each
- * tile's key blocks are cut into fa_fwd_kv_split(...) contiguous shares that
- * run as separate tiles; their partial results (fp32 O and LSE per share, in
- * scratch this call allocates and frees stream-ordered on `stream`) are merged
- * by a second kernel as the online softmax merges blocks (§04).  The blocks share a tile
+ * kv head.  Where the work tiles would leave SMs idle (fewer tiles than SMs,
+ * or a last round that fills few of them), the key blocks of every tile, or
+ * of the tiles after the last full round, are cut into fa_fwd_kv_split(...)
+ * contiguous shares that run as separate tiles; their partial results (fp32 O
+ * and LSE per share, in scratch this call allocates and frees stream-ordered
+ * on `stream`) are merged by a second kernel as the online softmax merges
+ * blocks (§04).  The blocks share a tile
  * counter, one of 256 slots in the library's device memory that launches take
  * in turn; the launch's last block resets it.  So at most 256 tiled forward
  * launches (this call, fa_fwd_ex, fa_fwd_fp8) may be in flight on one device
@@ -276,10 +278,11 @@ fa_status_t fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, 
 size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d);
 
 /*
- * Key shares per work tile that fa_fwd / fa_fwd_ex use on the current device
- * (1: no key split, also for the decode shapes, which run the split-KV decode
- * kernels; 2 to 16 where the work tiles are fewer than the SMs and the split
- * is estimated to save at least 10%).  0 for sizes fa_fwd would refuse.
+ * Key shares per split work tile that fa_fwd / fa_fwd_ex use on the current
+ * device: 1 for no key split (also for the decode shapes, which run the
+ * split-KV decode kernels), 2 to 16 where a split of every tile, or of the
+ * tiles after the last full round, is estimated (by simulating the persistent
+ * launch's claiming) to save at least 5%.  0 for sizes fa_fwd would refuse.
  */
 int fa_fwd_kv_split(int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal);
 
