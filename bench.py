@@ -275,6 +275,42 @@ def run_reference(args, rank, world):
 # ----------------------------------------------------------------------------
 # GPU arm
 # ----------------------------------------------------------------------------
+# Shared-memory bytes of one 64-row query step of bwd_main at d = 128 (the kernel's
+# dataflow): MMA operand reads (S^T: K 32 KB + Q 16 KB, dP^T: V 32 KB + dO 16 KB, dV: dO
+# 16 KB and dK: Q 16 KB with A in tensor memory, dQ^T: K 32 KB + dS^T 16 KB), TMA writes
+# (Q, dO 16 KB each, -LSE / -D 512 B), dS^T stores 16 KB, and the fp32 dQ staging tile
+# (32 KB stored by the drain warps, 32 KB read by the bulk reduce)
+BWD_MAIN_SMEM_BYTES_PER_STEP = 180224 + 33280 + 16384 + 65536
+SMEM_BYTES_PER_CLK_PER_SM = 128
+
+
+def smem_roofline(w, bwd_ms, clocks):
+    """bwd_main's shared-memory traffic by its dataflow (bytes per step x steps) over the
+    fa_bwd call's mean time, against 148 SMs x 128 B/clk at the sampled SM clock."""
+    steps = bwd_main_steps(w)
+    mhz = clocks.get("sm_mhz") or 1965.0
+    peak = 148 * SMEM_BYTES_PER_CLK_PER_SM * mhz * 1e6 / 1e12
+    achieved = steps * BWD_MAIN_SMEM_BYTES_PER_STEP / (bwd_ms * 1e-3) / 1e12
+    return {"unit": "TB/s", "achieved": achieved, "peak": peak, "frac": achieved / peak,
+            "steps": steps, "bytes_per_step": BWD_MAIN_SMEM_BYTES_PER_STEP,
+            "rule": "bytes per 64-row step of the kernel's dataflow x steps / mean fa_bwd call time "
+                    "(pre / post included); peak 148 SMs x 128 B/clk at the sampled SM clock"}
+
+
+def bwd_main_steps(w) -> int:
+    """64-row query steps of one bwd_main launch: every (key block, kv head) unit walks
+    G heads x the 64-row query blocks that can see its keys."""
+    nqb_all = (w.Nq + 63) // 64
+    total = 0
+    for kb in range((w.Nk + 127) // 128):
+        qb0 = 0
+        if w.causal:
+            first = kb * 128 - (w.Nk - w.Nq)
+            qb0 = 0 if first <= 0 else first // 64
+        total += max(0, nqb_all - qb0)
+    return total * w.B * w.Hkv * (w.Hq // w.Hkv)
+
+
 # DRAM bytes (read + write) of one bwd_main launch on this workload, from the ncu
 # launch list of this bench command on the current kernel (dram__bytes_read.sum +
 # dram__bytes_write.sum, mean of the six warm-up and timed-step launches); to be
@@ -693,7 +729,9 @@ def run_libfa(args, rank, world, local):
                                       f"CUDA-event duration of the {args.steps} timed calls",
                      "traffic": BWD_MAIN_DRAM_BYTES, "traffic_kernel": "bwd_main (one launch at this workload, one-pass ncu)",
                      "peak_source": peaks["source"] + " burst bf16 cuBLAS (each call timed alone after an "
-                                                      "L2 flush)"},
+                                                      "L2 flush)",
+                     # the resource that binds bwd_main: shared-memory bandwidth
+                     "smem": smem_roofline(w, bwd_mean, clocks)},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "mode": "double-buffered: step i+1 inputs copied in and step i-1 gradients copied out "
