@@ -799,6 +799,64 @@ def run_profile(which: str, launches: int = 3) -> int:
     return 0
 
 
+# (B, Hq, Hkv, Nq, Nk, d, causal): sequence lengths, masks and head sizes around the step
+# workload, short-query shapes (chunked prefill against a long context) and small launches
+SWEEP_SHAPES = [
+    (1, 32, 8, n, n, 128, c) for n in (1024, 2048, 4096, 8192, 16384) for c in (True, False)
+] + [
+    (1, 32, 8, 8192, 8192, 64, True), (1, 32, 8, 8192, 8192, 256, True),
+    (4, 16, 16, 1024, 1024, 64, True), (2, 32, 32, 4096, 4096, 128, True),
+    (1, 32, 8, 512, 32768, 128, True), (1, 32, 8, 2048, 32768, 128, True),
+    (1, 32, 8, 4096, 32768, 128, True), (1, 4, 1, 2048, 2048, 128, True),
+]
+
+
+def run_sweep(steps: int) -> int:
+    """fa_fwd and fa_bwd on SWEEP_SHAPES: median CUDA-event time per call (L2 flushed
+    before each), TFLOP/s over the visible (query, key) pairs (4 d per pair and head,
+    x2.5 for the backward), and the key / query splits each call takes.  One JSON line
+    per shape."""
+    import torch
+    import exact_attention_114_b200 as fa
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(2 * 126 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def med(fn):
+        ts = []
+        for i in range(steps + 3):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    for i, (B, Hq, Hkv, Nq, Nk, d, causal) in enumerate(SWEEP_SHAPES):
+        w = synth.Workload("sweep", B, Hq, Hkv, Nq, Nk, d, causal, 5000 + i)
+        x = {k: v.to(dev) for k, v in synth.make_inputs(w).items()}
+        o = torch.empty_like(x["q"])
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
+        g = [torch.empty_like(x[k]) for k in ("q", "k", "v")]
+        ws = torch.empty(fa.fa_bwd_workspace_size(B, Hq, Hkv, Nq, Nk, d), dtype=torch.uint8, device=dev)
+        f_ms = med(lambda: fa.fa_fwd(x["q"], x["k"], x["v"], o, lse, causal=causal, scale=w.scale))
+        b_ms = med(lambda: fa.fa_bwd(x["q"], x["k"], x["v"], o, x["dout"], lse, *g, causal=causal,
+                                     scale=w.scale, workspace=ws))
+        fa.fa_check_device_status()
+        vis = (sum(min(max(r + Nk - Nq + 1, 0), Nk) for r in range(Nq)) if causal else Nq * Nk)
+        fl = 4.0 * B * Hq * vis * d
+        print(json.dumps({"sweep": {"B": B, "Hq": Hq, "Hkv": Hkv, "Nq": Nq, "Nk": Nk, "d": d, "causal": causal},
+                          "fwd_ms": f_ms, "fwd_tflops": fl / (f_ms * 1e-3) / 1e12,
+                          "bwd_ms": b_ms, "bwd_tflops": 2.5 * fl / (b_ms * 1e-3) / 1e12,
+                          "fwd_kv_split": fa.fa_fwd_kv_split(B, Hq, Hkv, Nq, Nk, d, causal),
+                          "bwd_query_split": fa.fa_bwd_query_split(B, Hq, Hkv, Nq, Nk, d, causal)}),
+              flush=True)
+        del x, o, lse, g, ws
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -808,11 +866,15 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", choices=sorted(PROFILE_CASES),
                     help="run a few launches of one call on a reduced shape (for ncu) and exit")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time fa_fwd / fa_bwd over a grid of shapes (one JSON line each) and exit")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
     if args.profile:
         return run_profile(args.profile)
+    if args.sweep:
+        return run_sweep(max(5, args.steps // 2))
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         # one process per GPU: start the ranks here and let rank 0 print the line
         return spawn_replicas(args.gpus, sys.argv[1:] if argv is None else list(argv))
