@@ -295,7 +295,10 @@ int host_blocks_for_tile(int qt, int rows, int Nq, int Nk, int causal)
 // A tail split keeps to 2 shares when K and V take more than 64 MB: the whole units of a kv
 // head stream its keys together and mostly hit in L2, while the shares of one unit read
 // different key ranges at once (4 shares on a 2048-row chunk against 32K keys: no gain, with
-// 8% in the simulation).  The choice depends only on the sizes and the SM count, and is cached.
+// 8% in the simulation).  The choice depends only on the units' key-block counts, the head
+// size, the SM count and whether K / V pass 64 MB; it is cached under those (up to 4096 entries,
+// then the cache starts over).  Candidates whose even-spread lower bound cannot beat the best so
+// far are not simulated, and a plan of at most one tile per SM needs no simulation.
 struct FwdSplit {
     int shares, full;
 };
@@ -305,51 +308,63 @@ FwdSplit fwd_split_plan(const FwdGeom& g, int B, int Hkv, int Nq, int Nk, int d,
     const long long n_units = (long long)g.n_pairs * g.n_bh;
     if (n_units > 8LL * sms || n_units < 1)
         return {1, (int)n_units};
+    const int kt = kernel_d(d) == 256 ? 1 : 2;
+    // the plan depends on the sizes only through the units' key-block counts
+    const double kv_bytes = 4.0 * B * Hkv * (double)Nk * d;   // K and V, 16-bit
+    const bool kv_beyond_l2 = kv_bytes > 64.0 * (1 << 20);
+    std::vector<long long> key{g.n_bh, kt, d, sms, kv_beyond_l2};
+    for (int pr = 0; pr < g.n_pairs; ++pr) {
+        int n = 0;
+        for (int t = 0; t < kt; ++t)
+            n = std::max(n, host_blocks_for_tile(pr * 128 * kt + 128 * t, g.rows, Nq, Nk, causal));
+        key.push_back(n);
+    }
     static std::mutex mu;
     static std::map<std::vector<long long>, FwdSplit> cache;
-    const std::vector<long long> key{g.n_pairs, g.n_bh, g.rows, B, Hkv, Nq, Nk, d, causal, sms};
-    const double kv_bytes = 4.0 * B * Hkv * (double)Nk * d;   // K and V, 16-bit
     {
         std::lock_guard<std::mutex> lk(mu);
         auto it = cache.find(key);
         if (it != cache.end())
             return it->second;
     }
-    const int kt = kernel_d(d) == 256 ? 1 : 2;
-    std::vector<int> pair_len((size_t)g.n_pairs);
-    for (int pr = 0; pr < g.n_pairs; ++pr) {
-        int n = 0;
-        for (int t = 0; t < kt; ++t)
-            n = std::max(n, host_blocks_for_tile(pr * 128 * kt + 128 * t, g.rows, Nq, Nk, causal));
-        pair_len[(size_t)pr] = n;
-    }
-    auto unit_len = [&](long long u) { return pair_len[(size_t)(g.n_pairs - 1 - u / g.n_bh)]; };
+    auto unit_len = [&](long long u) { return (int)key[5 + (size_t)(g.n_pairs - 1 - u / g.n_bh)]; };
     const double fixed = 2.0, merge_fixed = 8.0, bytes_per_block = 13.0e6;
-    // greedy claiming of the work tiles in order on `sms` CTAs: the last finish
-    auto simulate = [&](long long full, int sh) {
-        std::priority_queue<double, std::vector<double>, std::greater<double>> done;
+    std::vector<double> lens;
+    // the work tiles of a plan, in claim order
+    auto items = [&](long long full, int sh) {
+        lens.clear();
+        for (long long u = 0; u < n_units; ++u) {
+            const int n = unit_len(u);
+            if (u < full || sh == 1) {
+                lens.push_back(n + fixed);
+            } else {
+                for (int k = 0; k < sh; ++k)
+                    lens.push_back((double)(((long long)(k + 1) * n) / sh - ((long long)k * n) / sh) + fixed);
+            }
+        }
+    };
+    // greedy claiming on `sms` CTAs: the last finish (one round: the longest tile)
+    auto simulate = [&]() {
         double last = 0;
-        auto take = [&](double len) {
+        if ((int)lens.size() <= sms) {
+            for (double x : lens)
+                last = std::max(last, x);
+            return last;
+        }
+        std::priority_queue<double, std::vector<double>, std::greater<double>> done;
+        for (double x : lens) {
             double start = 0;
             if ((int)done.size() == sms) {
                 start = done.top();
                 done.pop();
             }
-            done.push(start + len + fixed);
-            last = std::max(last, start + len + fixed);
-        };
-        for (long long u = 0; u < n_units; ++u) {
-            const int n = unit_len(u);
-            if (u < full || sh == 1) {
-                take(n);
-            } else {
-                for (int k = 0; k < sh; ++k)
-                    take((double)(((long long)(k + 1) * n) / sh - ((long long)k * n) / sh));
-            }
+            done.push(start + x);
+            last = std::max(last, start + x);
         }
         return last;
     };
-    const double base = simulate(n_units, 1);
+    items(n_units, 1);
+    const double base = simulate();
     FwdSplit best{1, (int)n_units};
     double best_cost = base;
     static const int kShares[] = {2, 3, 4, 6, 8, 12, 16};
@@ -358,14 +373,26 @@ FwdSplit fwd_split_plan(const FwdGeom& g, int B, int Hkv, int Nq, int Nk, int d,
         if (full >= n_units || (full > 0 && full == fulls[0]))
             continue;
         int longest = 0;
-        for (long long u = full; u < n_units; ++u)
-            longest = std::max(longest, unit_len(u));
+        double total = 0;
+        for (long long u = 0; u < n_units; ++u) {
+            total += unit_len(u);
+            if (u >= full)
+                longest = std::max(longest, unit_len(u));
+        }
         for (int sh : kShares) {
             const double part_bytes = (double)(n_units - full) * sh * 128 * kt * d * 4.0;
             if (longest < 2 * sh || part_bytes > 256.0 * (1 << 20) ||
-                (full > 0 && sh > 2 && kv_bytes > 64.0 * (1 << 20)))
+                (full > 0 && sh > 2 && kv_beyond_l2))
                 break;
-            const double cost = simulate(full, sh) + merge_fixed + 2.0 * part_bytes / bytes_per_block;
+            const double extra = merge_fixed + 2.0 * part_bytes / bytes_per_block;
+            // no plan beats its lower bound, the work spread evenly over all SMs, and
+            // the bound grows with the share count
+            const double n_items = (double)full + (double)(n_units - full) * sh;
+            const double bound = (total + n_items * fixed) / sms + extra;
+            if (bound >= best_cost || bound >= 0.95 * base)
+                break;
+            items(full, sh);
+            const double cost = simulate() + extra;
             if (cost < best_cost && cost < 0.95 * base) {
                 best = {sh, (int)full};
                 best_cost = cost;
@@ -373,6 +400,8 @@ FwdSplit fwd_split_plan(const FwdGeom& g, int B, int Hkv, int Nq, int Nk, int d,
         }
     }
     std::lock_guard<std::mutex> lk(mu);
+    if (cache.size() >= 4096)
+        cache.clear();
     cache[key] = best;
     return best;
 }

@@ -301,3 +301,20 @@ def test_forward_key_split_rule():
     assert ks(1, 3, 2, 64, 64, 64, 0) == 0            # Hq not a multiple of Hkv
     assert ks(1, 2, 1, 64, 64, 80, 0) == 0            # head size not a multiple of 32
     assert fa.lib().fa_fwd_kv_split(1, 2, 1, 64, 64, 64, 2) == 0
+
+
+def test_forward_key_split_plan_cache():
+    """The planner's cache: a context that grows by one key at a time (a new shape
+    per call, more than the cache keeps) gives the same plans as the first calls
+    on those shapes, and the known plans still hold after the cache started over."""
+    if _sm_count() != 148:
+        pytest.skip("the expected shares are for 148 SMs")
+    ks = fa.fa_fwd_kv_split
+    first = [ks(1, 32, 8, 512, nk, 128, 1) for nk in range(100, 6000)]
+    for i in range(5000):   # 5000 different key-block counts
+        ks(1, 8, 2, 300 + 7 * i, 1000 + 128 * i, 64, 1)
+    again = [ks(1, 32, 8, 512, nk, 128, 1) for nk in range(100, 6000)]
+    assert first == again
+    assert ks(1, 32, 8, 512, 32768, 128, 1) == 2
+    assert ks(1, 32, 8, 4096, 32768, 128, 1) == 2
+    assert ks(1, 2, 1, 300, 5000, 64, 1) == 16
