@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdParams p)
     // one warp per two rows of B * Hq * Nq_pad (both rows' loads issued before
     // either is reduced); lane l owns columns E*l .. E*l+E-1
     constexpr int E = D / 32;   // elements per lane
+    griddep_launch_dependents();   // bwd_main may start its set-up and K / V loads
     const int lane = threadIdx.x & 31;
     const int total = p.B * p.Hq * p.Nq_pad;
     const int row0 = (int)(blockIdx.x * 16 + (threadIdx.x >> 5) * 2);
@@ -191,6 +192,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdParams p)
 template <int D, typename T = __nv_bfloat16>
 __global__ void __launch_bounds__(256) bwd_post_kernel(BwdParams p)
 {
+    griddep_wait();   // the accumulator is complete once bwd_main has finished
     const int lane = threadIdx.x & 31;
     const long long BH = (long long)p.B * p.Hq;
     const int i_step = (int)gridDim.x * 16;
@@ -323,6 +325,7 @@ __global__ void __launch_bounds__(384, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* split_word = reinterpret_cast<int*>(bars + 22);   // query split: the ticket, to the compute warps
 
+    griddep_launch_dependents();   // bwd_post may take the SMs this launch frees
     const int warp = warp_id(), lane = lane_id();
     const int nsp = SPLIT ? p.q_split : 1;                         // CTAs per unit
     const int units = p.B * p.Hkv * C::kFeatSplit;                 // units per key block
@@ -377,6 +380,12 @@ __global__ void __launch_bounds__(384, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // The launch may overlap the end of bwd_pre (programmatic launch), which writes -lse_log2,
+    // -delta, the zeroed dQ accumulator and the split counters: every thread waits for it
+    // here, except the TMA thread, which first issues the K / V loads (inputs bwd_pre leaves
+    // alone) and then waits.
+    if (warp != 8 || lane != 0)
+        griddep_wait();
 
     auto step_coords = [&](int it, int& h, int& qb) {
         const int g = it_lo + it;
@@ -397,6 +406,7 @@ __global__ void __launch_bounds__(384, 1)
                 tma_load_3d(smem + C::kOffK + pn * C::kKPanel, &tmK, bar_kv, pn * 64, kb * 128, kvh);
                 tma_load_3d(smem + C::kOffV + pn * C::kKPanel, &tmV, bar_kv, pn * 64, kb * 128, kvh);
             }
+            griddep_wait();
             if constexpr (C::kHalves) {
                 // part 0: the other CTA's feature half (Q and dO), read only by the step's
                 // S^T / dP^T; part 1: this CTA's Q half (buffer st & 1) with the step's

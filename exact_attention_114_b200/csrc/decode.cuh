@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(160, 2)   // two CTAs per SM (shared memory al
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         DecodeParams p)
 {
+    griddep_launch_dependents();   // the combine may be scheduled
     const int d_io = NARROW ? p.d_io : 128;
     using C = DecCfg;
     extern __shared__ uint8_t smem_raw[];
@@ -342,6 +343,7 @@ __global__ void __launch_bounds__(160, 2)   // two CTAs per SM (shared memory al
 template <typename T = __nv_bfloat16>
 __global__ void __launch_bounds__(128) decode_combine_kernel(DecodeParams p)
 {
+    griddep_wait();   // the partials are complete once the split pass has finished
     const int warp = (int)(blockIdx.x * 4 + (threadIdx.x >> 5));
     const int lane = threadIdx.x & 31;
     const int total = p.B * p.Hkv * p.R;

@@ -19,6 +19,7 @@
 #include <vector>
 #include <string>
 #include <type_traits>
+#include <utility>
 
 #include "bwd.cuh"
 #include "decode.cuh"
@@ -212,6 +213,31 @@ fa_status_t check_launch(const char* what)
     if (e != cudaSuccess)
         return cuda_fail(e, what);
     return FA_OK;
+}
+
+// Launch `kern` as a programmatic dependent of the kernel before it on the stream, which
+// is always one of this library's own launches of the same call: its blocks may be
+// scheduled, and run their set-up, while that kernel's last blocks finish.  Each such
+// kernel calls griddep_wait() before it reads anything that kernel writes, and the
+// kernel before it calls griddep_launch_dependents() at its start.
+template <typename... P, typename... A>
+fa_status_t launch_dependent(const char* what, void (*kern)(P...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t stream, A&&... args)
+{
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+    if (e != cudaSuccess)
+        return cuda_fail(e, what);
+    return check_launch(what);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -451,8 +477,8 @@ fa_status_t launch_fwd_tiles(Kern kern, int threads, int smem, const CUtensorMap
     if (p.kv_split > 1) {
         if (st == FA_OK) {
             const long long rows = (long long)p.n_bh * p.rows;
-            fa::fwd_combine_kernel<T><<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(p);
-            st = check_launch("fwd_combine_kernel launch");
+            st = launch_dependent("fwd_combine_kernel launch", fa::fwd_combine_kernel<T>,
+                                  dim3((unsigned)((rows + 3) / 4)), dim3(128), 0, stream, p);
         }
         cudaError_t e = cudaFreeAsync(ws, stream);
         if (e != cudaSuccess && st == FA_OK)
@@ -696,8 +722,9 @@ fa_status_t launch_decode_t(const void* q, const void* k, const void* v, void* o
     if ((st = check_launch("decode_split_kernel launch")) != FA_OK) return st;
     if (pl.splits > 1) {
         const long long rows = (long long)B * Hkv * p.R;
-        fa::decode_combine_kernel<T><<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(p);
-        if ((st = check_launch("decode_combine_kernel launch")) != FA_OK) return st;
+        if ((st = launch_dependent("decode_combine_kernel launch", fa::decode_combine_kernel<T>,
+                                   dim3((unsigned)((rows + 3) / 4)), dim3(128), 0, stream, p)) != FA_OK)
+            return st;
     }
     return FA_OK;
 }
@@ -924,14 +951,14 @@ fa_status_t launch_bwd(const fa::BwdParams& p, const void* q, const void* k, con
     auto kern = p.q_split > 1 ? fa::bwd_main_kernel<D, CAUSAL, T, true> : fa::bwd_main_kernel<D, CAUSAL, T, false>;
     if ((st = ensure_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes)) != FA_OK) return st;
     const long long grid = (long long)((p.Nk + 127) / 128) * p.B * p.Hkv * C::kFeatSplit * p.q_split;
-    kern<<<(unsigned)grid, C::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mdo, p);
-    if ((st = check_launch("bwd_main_kernel launch")) != FA_OK) return st;
+    if ((st = launch_dependent("bwd_main_kernel launch", kern, dim3((unsigned)grid), dim3(C::kThreads),
+                               C::kSmemBytes, stream, mq, mk, mv, mdo, p)) != FA_OK)
+        return st;
 
     // 16 rows per block; the y dimension walks batch * head (looping past 65535)
     const dim3 pgrid((unsigned)std::max(1, std::min((p.Nq + 15) / 16, 4096)),
                      (unsigned)std::max<long long>(1, std::min<long long>((long long)p.B * p.Hq, 65535)));
-    fa::bwd_post_kernel<D, T><<<pgrid, 256, 0, stream>>>(p);
-    return check_launch("bwd_post_kernel launch");
+    return launch_dependent("bwd_post_kernel launch", fa::bwd_post_kernel<D, T>, pgrid, dim3(256), 0, stream, p);
 }
 
 template <typename T>

@@ -212,6 +212,7 @@ __global__ void __launch_bounds__(384, 1)
                const __grid_constant__ CUtensorMap tmV, FwdParams p)
 {
     using C = FwdCfg<D, F8>;
+    griddep_launch_dependents();   // the merge of a key split may be scheduled
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -837,6 +838,7 @@ __global__ void __launch_bounds__(384, 1)
 template <typename T = __nv_bfloat16>
 __global__ void __launch_bounds__(128) fwd_combine_kernel(FwdParams p)
 {
+    griddep_wait();   // the partials are complete once the forward has finished
     const long long row = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= (long long)p.n_bh * p.rows)

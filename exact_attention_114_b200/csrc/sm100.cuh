@@ -580,6 +580,15 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* ptr)
     return v;
 }
 
+// Programmatic dependent launch (PTX griddepcontrol).  A kernel launched with
+// programmatic stream serialisation may start while the kernel before it on the stream
+// finishes; griddep_wait() returns once that kernel has completed and its memory
+// operations are visible.  griddep_launch_dependents() lets the next such kernel start
+// once every block of this one has issued it or exited.  In a plain launch both are
+// no-ops.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // barrier over a subset of the block's warps (ids 1..15; 0 is __syncthreads)
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads)
 {

@@ -4,6 +4,8 @@ GPU has SMs, each tile's key blocks are cut into contiguous shares that run as
 separate tiles, and a second kernel merges their fp32 partials by their LSE.
 Each case checks O and LSE (every row, or sampled rows at the long append
 shapes) and that O repeats bitwise from call to call."""
+import functools
+
 import numpy as np
 import pytest
 import torch
@@ -135,6 +137,55 @@ def test_fwd_tail_split_full(shape):
     assert torch.equal(o, o2) and torch.equal(lse, l2)
     o_ref, lse_ref = oracle.fwd(x["q"], x["k"], x["v"], w.scale, w.causal)
     G.assert_o(G.f64(o), o_ref, o_abs=G.o_abs_ref(x["q"], x["k"], x["v"], w.scale, w.causal))
+    G.assert_lse(G.f64(lse), lse_ref)
+
+
+# Seeded random shapes on which the planner splits the keys: units (query-tile pairs x heads,
+# Nq >= 300 so no group rows) at most the SM count, where every unit runs in shares, or beyond
+# it, where the units after the last full round do (a tail split).  Drawn at run time (the
+# plan depends on the device's SM count), within a budget the oracle finishes in about a
+# second; every O and LSE element is compared.
+@functools.lru_cache(maxsize=None)
+def _draw_split_shapes(tail, n=6, seed=20261205):
+    rng = np.random.default_rng(seed + int(tail))
+    sms, out = _sms(), []
+    for _ in range(20000):
+        if len(out) == n:
+            break
+        d = int(rng.choice([64, 128]))
+        Hkv = int(rng.choice([2, 4, 8] if tail else [1, 2, 4, 8]))
+        G_ = int(rng.choice([2, 3, 4, 8] if tail else [1, 2, 4]))
+        B = int(rng.integers(1, 3))
+        Hq = Hkv * G_
+        Nq = int(rng.integers(300, 2200 if tail else 2600))
+        Nk = int(rng.integers(300, 3000 if tail else 4000))
+        causal = bool(rng.integers(0, 2))
+        units = B * Hq * ((Nq + 255) // 256)
+        pairs = B * Hq * Nq * Nk * (0.5 if causal else 1.0)
+        if (units > sms) != tail or pairs * d > 6e9:
+            continue
+        shares = fa.fa_fwd_kv_split(B, Hq, Hkv, Nq, Nk, d, causal)
+        if shares > 1:
+            out.append((B, Hq, Hkv, Nq, Nk, d, causal, shares))
+    return tuple(out)
+
+
+@pytest.mark.parametrize("tail", [False, True], ids=["every_unit", "tail"])
+@pytest.mark.parametrize("i", range(6))
+def test_fwd_split_random(tail, i):
+    shapes = _draw_split_shapes(tail)
+    if i >= len(shapes):
+        pytest.skip(f"only {len(shapes)} split shapes drawn on this device")
+    B, Hq, Hkv, Nq, Nk, d, causal, shares = shapes[i]
+    w = synth.Workload("fwd_split_random", B, Hq, Hkv, Nq, Nk, d, causal, 9870 + 10 * int(tail) + i)
+    dtype = torch.float16 if i % 3 == 2 else torch.bfloat16
+    x = synth.make_inputs(w, dout=False, dtype=dtype)
+    xd = {k: v.cuda() for k, v in x.items()}
+    o, lse, o2, l2 = _forward_twice(w, xd)
+    assert torch.equal(o, o2) and torch.equal(lse, l2)
+    xr = {k: v.double() for k, v in x.items()}
+    o_ref, lse_ref = oracle.fwd(xr["q"], xr["k"], xr["v"], w.scale, w.causal)
+    G.assert_o(G.f64(o), o_ref, o_abs=G.o_abs_ref(xr["q"], xr["k"], xr["v"], w.scale, w.causal))
     G.assert_lse(G.f64(lse), lse_ref)
 
 
