@@ -33,7 +33,13 @@
  *    Nq = Nk this is the usual lower triangle).  A query row that sees no key
  *    gets O = 0, LSE = -inf and zero gradients.
  *  - stream is a cudaStream_t (NULL = the legacy default stream).  All work is
- *    enqueued on it; no call synchronises the stream or the device.
+ *    enqueued on it; no call synchronises the stream or the device.  A call's
+ *    first kernel is a plain launch: it starts after all earlier work on the
+ *    stream.  Its later kernels (the backward's main and post passes, the merge of
+ *    split partials) are programmatic dependent launches.  They may start their
+ *    set-up while the kernel before them finishes, but they read nothing that
+ *    kernel writes until it has completed.  Later work on the stream starts after
+ *    the whole call, as usual.
  *  - Ownership: the caller owns every buffer; the library keeps no pointer
  *    after a call returns and frees nothing it did not allocate.
  *  - Scratch: a call that allocates its own scratch (workspace NULL, or the
