@@ -814,8 +814,8 @@ SWEEP_SHAPES = [
 def run_sweep(steps: int) -> int:
     """fa_fwd and fa_bwd on SWEEP_SHAPES: median CUDA-event time per call (L2 flushed
     before each), TFLOP/s over the visible (query, key) pairs (4 d per pair and head,
-    x2.5 for the backward), and the key / query splits each call takes.  One JSON line
-    per shape."""
+    x2.5 for the backward), the key / query splits each call takes and the SM clocks
+    sampled while the shape ran.  One JSON line per shape."""
     import torch
     import exact_attention_114_b200 as fa
     dev = torch.device("cuda", 0)
@@ -841,9 +841,10 @@ def run_sweep(steps: int) -> int:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
         g = [torch.empty_like(x[k]) for k in ("q", "k", "v")]
         ws = torch.empty(fa.fa_bwd_workspace_size(B, Hq, Hkv, Nq, Nk, d), dtype=torch.uint8, device=dev)
-        f_ms = med(lambda: fa.fa_fwd(x["q"], x["k"], x["v"], o, lse, causal=causal, scale=w.scale))
-        b_ms = med(lambda: fa.fa_bwd(x["q"], x["k"], x["v"], o, x["dout"], lse, *g, causal=causal,
-                                     scale=w.scale, workspace=ws))
+        with ClockSampler(0) as clk:
+            f_ms = med(lambda: fa.fa_fwd(x["q"], x["k"], x["v"], o, lse, causal=causal, scale=w.scale))
+            b_ms = med(lambda: fa.fa_bwd(x["q"], x["k"], x["v"], o, x["dout"], lse, *g, causal=causal,
+                                         scale=w.scale, workspace=ws))
         fa.fa_check_device_status()
         vis = (sum(min(max(r + Nk - Nq + 1, 0), Nk) for r in range(Nq)) if causal else Nq * Nk)
         fl = 4.0 * B * Hq * vis * d
@@ -851,7 +852,8 @@ def run_sweep(steps: int) -> int:
                           "fwd_ms": f_ms, "fwd_tflops": fl / (f_ms * 1e-3) / 1e12,
                           "bwd_ms": b_ms, "bwd_tflops": 2.5 * fl / (b_ms * 1e-3) / 1e12,
                           "fwd_kv_split": fa.fa_fwd_kv_split(B, Hq, Hkv, Nq, Nk, d, causal),
-                          "bwd_query_split": fa.fa_bwd_query_split(B, Hq, Hkv, Nq, Nk, d, causal)}),
+                          "bwd_query_split": fa.fa_bwd_query_split(B, Hq, Hkv, Nq, Nk, d, causal),
+                          "clocks": clk.summary()}),
               flush=True)
         del x, o, lse, g, ws
     return 0
