@@ -91,3 +91,72 @@ def test_graph_replay_matches_eager(shape):
     G.assert_grad(G.f64(got["dq"]), rq, "dQ")
     G.assert_grad(G.f64(got["dk"]), rk, "dK")
     G.assert_grad(G.f64(got["dv"]), rv, "dV")
+
+
+def _programmatic_edges(fn):
+    """A CUDA graph captured (relaxed mode) from the work fn enqueues on a fresh stream,
+    never launched: (programmatic edges from a kernel node to a kernel node, kernel nodes,
+    the node types at both ends of every programmatic edge)."""
+    from cuda.bindings import runtime as rt
+    ok = rt.cudaError_t.cudaSuccess
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        err, = rt.cudaStreamBeginCapture(stream.cuda_stream,
+                                         rt.cudaStreamCaptureMode.cudaStreamCaptureModeRelaxed)
+        assert err == ok, err
+        try:
+            fn()
+        finally:
+            err, graph = rt.cudaStreamEndCapture(stream.cuda_stream)
+    assert err == ok, err
+    try:
+        res = rt.cudaGraphGetEdges_v2(graph, 0)
+        assert res[0] == ok, res[0]
+        err, src, dst, data, n = rt.cudaGraphGetEdges_v2(graph, res[-1])
+        assert err == ok, err
+        kernel = rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+        kind = lambda nd: rt.cudaGraphNodeGetType(nd)[1]
+        # a programmatic edge: its type, or its source port (programmatic / launch completion)
+        prog = [(kind(a), kind(b)) for a, b, e in zip(src[:n], dst[:n], data[:n])
+                if int(e.type) == int(rt.cudaGraphDependencyType.cudaGraphDependencyTypeProgrammatic)
+                or int(e.from_port) != int(rt.cudaGraphKernelNodePortDefault)]
+        err, _, m = rt.cudaGraphGetNodes(graph, 0)
+        err, nodes, m = rt.cudaGraphGetNodes(graph, m)
+        kernels = sum(1 for nd in nodes[:m] if kind(nd) == kernel)
+        return sum(1 for a, b in prog if a == kernel and b == kernel), kernels, prog
+    finally:
+        rt.cudaGraphDestroy(graph)
+
+
+def test_capture_records_programmatic_edges():
+    """A call's later kernels are programmatic dependents of the kernel before them:
+    the backward's main and post passes (2 kernel-to-kernel edges), the merge of a
+    key-split forward and of a split-KV decode (1 each); a plain forward has none."""
+    w = synth.Workload("graph_edges", 1, 4, 1, 2048, 2048, 128, True, 9460)
+    x = {k: v.cuda() for k, v in synth.make_inputs(w).items()}
+    o, lse = fa.fa_fwd(x["q"], x["k"], x["v"], causal=True)
+    ws = torch.empty(fa.fa_bwd_workspace_size(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d), dtype=torch.uint8,
+                     device="cuda")
+    g = [torch.empty_like(x[k]) for k in ("q", "k", "v")]
+    torch.cuda.synchronize()
+    prog, kern, edges = _programmatic_edges(
+        lambda: fa.fa_bwd(x["q"], x["k"], x["v"], o, x["dout"], lse, *g, causal=True, workspace=ws))
+    assert (prog, kern) == (2, 3), edges
+    assert fa.fa_fwd_kv_split(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, True) > 1
+    prog, kern, edges = _programmatic_edges(lambda: fa.fa_fwd(x["q"], x["k"], x["v"], o, lse, causal=True))
+    assert (prog, kern) == (1, 2), edges
+    w2 = synth.Workload("graph_edges_plain", 1, 32, 8, 2048, 2048, 128, True, 9461, backward=False)
+    x2 = {k: v.cuda() for k, v in synth.make_inputs(w2, dout=False).items()}
+    assert fa.fa_fwd_kv_split(w2.B, w2.Hq, w2.Hkv, w2.Nq, w2.Nk, w2.d, True) == 1
+    o2, lse2 = fa.fa_fwd(x2["q"], x2["k"], x2["v"], causal=True)
+    prog, kern, edges = _programmatic_edges(
+        lambda: fa.fa_fwd(x2["q"], x2["k"], x2["v"], o2, lse2, causal=True))
+    assert (prog, kern) == (0, 1), edges
+    w3 = synth.Workload("graph_edges_decode", 2, 8, 2, 1, 3000, 128, True, 9462, backward=False)
+    x3 = {k: v.cuda() for k, v in synth.make_inputs(w3, dout=False).items()}
+    o3, lse3 = fa.fa_fwd_splitkv(x3["q"], x3["k"], x3["v"], causal=True, num_splits=4)
+    torch.cuda.synchronize()
+    prog, kern, edges = _programmatic_edges(
+        lambda: fa.fa_fwd_splitkv(x3["q"], x3["k"], x3["v"], o3, lse3, causal=True, num_splits=4))
+    assert (prog, kern) == (1, 2), edges
