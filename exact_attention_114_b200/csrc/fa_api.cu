@@ -459,7 +459,8 @@ fa_status_t fwd_tile_counter(unsigned** ctr, unsigned* tag)
 // go to stream-ordered scratch and fwd_combine_kernel merges them into o / lse.
 template <typename T, typename Kern>
 fa_status_t launch_fwd_tiles(Kern kern, int threads, int smem, const CUtensorMap& mq, const CUtensorMap& mk,
-                             const CUtensorMap& mv, fa::FwdParams& p, cudaStream_t stream)
+                             const CUtensorMap& mv, fa::FwdParams& p, cudaStream_t stream,
+                             bool after_kernel = false)
 {
     void* ws = nullptr;
     if (p.kv_split > 1) {
@@ -472,8 +473,15 @@ fa_status_t launch_fwd_tiles(Kern kern, int threads, int smem, const CUtensorMap
         p.part_o = static_cast<float*>(ws);
         p.part_lse = reinterpret_cast<float*>(static_cast<char*>(ws) + o_bytes);
     }
-    kern<<<fwd_grid(p), threads, smem, stream>>>(mq, mk, mv, p);
-    fa_status_t st = check_launch("fwd_kernel launch");
+    fa_status_t st;
+    if (after_kernel && p.kv_split <= 1) {
+        // straight after a kernel of the same call (the e4m3 V transpose)
+        st = launch_dependent("fwd_kernel launch", kern, dim3(fwd_grid(p)), dim3(threads), (size_t)smem, stream,
+                              mq, mk, mv, p);
+    } else {
+        kern<<<fwd_grid(p), threads, smem, stream>>>(mq, mk, mv, p);
+        st = check_launch("fwd_kernel launch");
+    }
     if (p.kv_split > 1) {
         if (st == FA_OK) {
             const long long rows = (long long)p.n_bh * p.rows;
@@ -585,7 +593,7 @@ fa_status_t launch_fwd_fp8(const void* q, const void* k, const void* v, void* vt
     p.part_lse = nullptr;
     if ((st = fwd_tile_counter(&p.tile_ctr, &p.tile_tag)) != FA_OK)
         return st;
-    return launch_fwd_tiles<__nv_bfloat16>(kern, C::kThreads, C::kSmemBytes, mq, mk, mv, p, stream);
+    return launch_fwd_tiles<__nv_bfloat16>(kern, C::kThreads, C::kSmemBytes, mq, mk, mv, p, stream, true);
 }
 
 template <typename T>

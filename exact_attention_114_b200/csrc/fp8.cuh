@@ -10,6 +10,8 @@
 
 #include <cstdint>
 
+#include "sm100.cuh"
+
 namespace fa {
 
 // grid (Nk_pad / 64 rounded up, B * Hkv), 256 threads; D = 128
@@ -18,6 +20,7 @@ __global__ void __launch_bounds__(256) fp8_vt_kernel(const uint8_t* __restrict__
                                                      int Nk, int Nk_pad)
 {
     __shared__ __align__(16) uint8_t tile[64][D + 16];   // 64 keys x D bytes (+16: fewer bank conflicts)
+    griddep_launch_dependents();   // the forward may start its set-up
     const int kb = (int)blockIdx.x * 64;
     const size_t bh = blockIdx.y;
     const uint8_t* src = v + bh * (size_t)Nk * D;

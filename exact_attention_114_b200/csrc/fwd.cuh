@@ -277,6 +277,9 @@ __global__ void __launch_bounds__(384, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // after the e4m3 V transpose the kernel is a programmatic dependent of it: V^T (and
+    // everything else) is read only once that kernel has completed; a no-op in a plain launch
+    griddep_wait();
     FwdTile w;
 
     // Each role runs inside the branch that sets its register budget.

@@ -36,7 +36,8 @@
  *    enqueued on it; no call synchronises the stream or the device.  A call's
  *    first kernel is a plain launch: it starts after all earlier work on the
  *    stream.  Its later kernels (the backward's main and post passes, the merge of
- *    split partials) are programmatic dependent launches.  They may start their
+ *    split partials, the e4m3 forward after its V transpose) are programmatic
+ *    dependent launches.  They may start their
  *    set-up while the kernel before them finishes, but they read nothing that
  *    kernel writes until it has completed.  Later work on the stream starts after
  *    the whole call, as usual.

@@ -132,7 +132,8 @@ def _programmatic_edges(fn):
 def test_capture_records_programmatic_edges():
     """A call's later kernels are programmatic dependents of the kernel before them:
     the backward's main and post passes (2 kernel-to-kernel edges), the merge of a
-    key-split forward and of a split-KV decode (1 each); a plain forward has none."""
+    key-split forward and of a split-KV decode (1 each), the e4m3 forward kernel after
+    its V transpose (1); a plain forward has none."""
     w = synth.Workload("graph_edges", 1, 4, 1, 2048, 2048, 128, True, 9460)
     x = {k: v.cuda() for k, v in synth.make_inputs(w).items()}
     o, lse = fa.fa_fwd(x["q"], x["k"], x["v"], causal=True)
@@ -159,4 +160,16 @@ def test_capture_records_programmatic_edges():
     torch.cuda.synchronize()
     prog, kern, edges = _programmatic_edges(
         lambda: fa.fa_fwd_splitkv(x3["q"], x3["k"], x3["v"], o3, lse3, causal=True, num_splits=4))
+    assert (prog, kern) == (1, 2), edges
+    # e4m3: the forward kernel after the V transpose (no key split at this size)
+    w4 = synth.Workload("graph_edges_fp8", 1, 32, 8, 2048, 2048, 128, True, 9463, backward=False)
+    assert fa.fa_fwd_kv_split(w4.B, w4.Hq, w4.Hkv, w4.Nq, w4.Nk, w4.d, True) == 1
+    x4 = {k: v.cuda() for k, v in synth.make_inputs_fp8(w4).items()}
+    ds = synth.FP8_DESCALE
+    vt = torch.empty(fa.fa_fwd_fp8_workspace_size(w4.B, w4.Hkv, w4.Nk, w4.d), dtype=torch.uint8, device="cuda")
+    o4, lse4 = fa.fa_fwd_fp8(x4["q"], x4["k"], x4["v"], ds["q"], ds["k"], ds["v"], causal=True, workspace=vt)
+    torch.cuda.synchronize()
+    prog, kern, edges = _programmatic_edges(
+        lambda: fa.fa_fwd_fp8(x4["q"], x4["k"], x4["v"], ds["q"], ds["k"], ds["v"], o4, lse4, causal=True,
+                              workspace=vt))
     assert (prog, kern) == (1, 2), edges
