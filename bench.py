@@ -315,7 +315,7 @@ def bwd_main_steps(w) -> int:
 # launch list of this bench command on the current kernel (dram__bytes_read.sum +
 # dram__bytes_write.sum, mean of the six warm-up and timed-step launches); to be
 # taken again whenever the kernel changes.
-BWD_MAIN_DRAM_BYTES = 677.65e6 + 320.94e6
+BWD_MAIN_DRAM_BYTES = 720.38e6 + 341.18e6
 
 
 def run_libfa(args, rank, world, local):
